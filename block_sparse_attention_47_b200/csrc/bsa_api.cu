@@ -1,0 +1,394 @@
+// The extern "C" entry points of libbsa.so: host-side validation of every
+// argument (nothing is launched on error), derived sizes, TMA tensor maps,
+// and the launches on the caller's stream.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "bsa_internal.cuh"
+
+namespace bsa {
+size_t select_smem_bytes(const Geo& g);
+}
+
+namespace {
+
+using bsa::Geo;
+
+thread_local char g_last_error[512] = "";
+
+bsa_status fail(bsa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// library-owned fallback status word for callers that pass dev_status = NULL
+__device__ int32_t g_dev_status_sink;
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+bsa_status make_geo(const bsa_problem* p, Geo* g) {
+  if (!p) return fail(BSA_ERR_INVALID_ARG, "problem is NULL");
+  if (p->B < 1 || p->heads < 1) return fail(BSA_ERR_SHAPE, "B and heads must be >= 1");
+  if (p->head_dim != 64 && p->head_dim != 128)
+    return fail(BSA_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", p->head_dim);
+  if (p->block_mode != BSA_BLOCK_FIXED_444 && p->block_mode != BSA_BLOCK_DYNAMIC_888)
+    return fail(BSA_ERR_INVALID_ARG, "block_mode %d is not a bsa_block_mode", p->block_mode);
+  const int unit = p->block_mode == BSA_BLOCK_DYNAMIC_888 ? 8 : 4;
+  const int max_pad = p->block_mode == BSA_BLOCK_DYNAMIC_888 ? 1 : 3;
+  const int dims[3] = {p->T, p->H, p->W};
+  const int valid[3] = {p->T_valid, p->H_valid, p->W_valid};
+  for (int a = 0; a < 3; ++a) {
+    if (dims[a] < unit || dims[a] % unit)
+      return fail(BSA_ERR_SHAPE, "grid extent %d must be a positive multiple of %d", dims[a], unit);
+    if (valid[a] < 1 || valid[a] > dims[a] || dims[a] - valid[a] > max_pad)
+      return fail(BSA_ERR_SHAPE,
+                  "valid extent %d of %d: at most %d trailing pad rows allowed so that no "
+                  "block is all pad",
+                  valid[a], dims[a], max_pad);
+  }
+  if (p->n_prefix_segments < 0 || p->n_prefix_segments > BSA_MAX_PREFIX_SEGMENTS)
+    return fail(BSA_ERR_SHAPE, "n_prefix_segments %d outside 0..%d", p->n_prefix_segments,
+                BSA_MAX_PREFIX_SEGMENTS);
+  if (!(std::isfinite(p->softmax_scale) && p->softmax_scale > 0.f))
+    return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (p->block_mode == BSA_BLOCK_DYNAMIC_888 && !(std::isfinite(p->dyn_tau) && p->dyn_tau >= 1.f))
+    return fail(BSA_ERR_INVALID_ARG, "dyn_tau must be finite and >= 1 in dynamic mode");
+
+  std::memset(g, 0, sizeof(*g));
+  g->B = p->B;
+  g->h = p->heads;
+  g->d = p->head_dim;
+  g->T = p->T;
+  g->H = p->H;
+  g->W = p->W;
+  g->Tv = p->T_valid;
+  g->Hv = p->H_valid;
+  g->Wv = p->W_valid;
+  g->nseg = p->n_prefix_segments;
+  int64_t P = 0;
+  for (int i = 0; i < g->nseg; ++i) {
+    if (p->prefix_len[i] < 1) return fail(BSA_ERR_SHAPE, "prefix_len[%d] must be >= 1", i);
+    g->seg_len[i] = p->prefix_len[i];
+    g->seg_off[i] = int(P);
+    P += (int64_t(p->prefix_len[i]) + 63) / 64 * 64;
+    if (P > (int64_t(1) << 28)) return fail(BSA_ERR_SHAPE, "prefix too long");
+  }
+  const int64_t Nv = int64_t(p->T) * p->H * p->W;
+  const int64_t N = P + Nv;
+  if (N > (int64_t(1) << 28)) return fail(BSA_ERR_SHAPE, "too many tokens (%lld)", (long long)N);
+  if (int64_t(p->B) * p->heads * N * p->head_dim > (int64_t(1) << 40))
+    return fail(BSA_ERR_SHAPE, "tensor too large");
+  g->P = int(P);
+  g->Nv = int(Nv);
+  g->N = int(N);
+  g->nbp = int(P / 64);
+  g->nbv = int(Nv / 64);
+  g->nb = g->nbp + g->nbv;
+  if (p->keep_blocks < 1 || p->keep_blocks > g->nbv)
+    return fail(BSA_ERR_SHAPE, "keep_blocks %d outside 1..%d", p->keep_blocks, g->nbv);
+  g->keep = p->keep_blocks;
+  g->kcap = g->nbp + g->keep;
+  g->mode = p->block_mode;
+  g->nreg = p->block_mode == BSA_BLOCK_DYNAMIC_888 ? (p->T / 8) * (p->H / 8) * (p->W / 8) : 0;
+  g->tau = p->dyn_tau;
+  g->scale = p->softmax_scale;
+  if (int64_t(p->B) * p->heads > 65535) return fail(BSA_ERR_SHAPE, "B*heads must be <= 65535");
+  if (bsa::select_smem_bytes(*g) > kMaxSmem)
+    return fail(BSA_ERR_UNSUPPORTED, "too many video blocks (%d) for on-chip selection", g->nbv);
+  return BSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bsa_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(BSA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(BSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return BSA_OK;
+}
+
+bsa_status check_strides(const Geo& g, int64_t sb, int64_t sn, int64_t sh, const char* name) {
+  // elements; every (b, n, h) row of head_dim bf16 must start 16-byte aligned
+  if (sb < 0 || sn < 0 || sh < 0 || (sb % 8) || (sn % 8) || (sh % 8))
+    return fail(BSA_ERR_INVALID_ARG, "%s strides must be non-negative multiples of 8 elements",
+                name);
+  (void)g;  // overlapping views are the caller's business; only alignment is checked
+  return BSA_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B*heads, N, d] bf16 block-order tensor, box = 64 columns x rows x 1
+bsa_status make_map(CUtensorMap* m, const Geo& g, const void* ptr, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {cuuint64_t(g.d), cuuint64_t(g.N), cuuint64_t(g.B) * g.h};
+  cuuint64_t strides[2] = {cuuint64_t(g.d) * 2, cuuint64_t(g.N) * g.d * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return BSA_OK;
+}
+
+bsa_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(BSA_ERR_UNSUPPORTED, "device is sm_%d%d; libbsa is built for sm_100a", major,
+                minor);
+  return BSA_OK;
+}
+
+#define BSA_TRY(x)                 \
+  do {                             \
+    bsa_status _s = (x);           \
+    if (_s != BSA_OK) return _s;   \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int32_t bsa_keep_count(int32_t n_blocks, double keep_ratio) {
+  if (n_blocks < 1 || !std::isfinite(keep_ratio) || keep_ratio < 0.0 || keep_ratio > 1.0)
+    return -1;
+  double k = std::ceil(keep_ratio * double(n_blocks) - 1e-9);
+  if (k < 1.0) k = 1.0;
+  if (k > double(n_blocks)) k = double(n_blocks);
+  return int32_t(k);
+}
+
+bsa_status bsa_query_sizes(const bsa_problem* prob, bsa_sizes* out) {
+  g_last_error[0] = 0;
+  if (!out) return fail(BSA_ERR_INVALID_ARG, "out is NULL");
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  out->n_tokens = g.N;
+  out->n_prefix_tokens = g.P;
+  out->n_blocks = g.nb;
+  out->n_prefix_blocks = g.nbp;
+  out->n_video_blocks = g.nbv;
+  out->n_regions = g.nreg;
+  out->list_capacity = g.kcap;
+  out->layout_bytes = bsa::layout_map(g).total;
+  out->perm_tensor_bytes = size_t(g.B) * g.h * g.N * g.d * 2;
+  out->raster_tensor_bytes = out->perm_tensor_bytes;
+  out->pool_bytes = size_t(g.B) * g.h * g.nb * g.d * 4;
+  out->idx_bytes = size_t(g.B) * g.h * g.nb * g.kcap * 4;
+  out->cnt_bytes = size_t(g.B) * g.h * g.nb * 4;
+  return BSA_OK;
+}
+
+bsa_status bsa_layout(const bsa_problem* prob, const void* k_raster, int64_t stride_b,
+                      int64_t stride_n, int64_t stride_h, void* layout_buf, void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  if (g.mode == BSA_BLOCK_DYNAMIC_888) {
+    BSA_TRY(check_ptr(k_raster, "k_raster"));
+    BSA_TRY(check_strides(g, stride_b, stride_n, stride_h, "k_raster"));
+  }
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_layout(g, static_cast<const __nv_bfloat16*>(k_raster), stride_b,
+                                     stride_n, stride_h, bsa::layout_ptrs(g, layout_buf),
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_layout launch");
+}
+
+bsa_status bsa_permute(const bsa_problem* prob, const void* layout_buf, const void* x_raster,
+                       int64_t stride_b, int64_t stride_n, int64_t stride_h, void* x_perm,
+                       void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(x_raster, "x_raster"));
+  BSA_TRY(check_ptr(x_perm, "x_perm"));
+  BSA_TRY(check_strides(g, stride_b, stride_n, stride_h, "x_raster"));
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_permute(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
+                                      static_cast<const __nv_bfloat16*>(x_raster), stride_b,
+                                      stride_n, stride_h, static_cast<__nv_bfloat16*>(x_perm),
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_permute launch");
+}
+
+bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void* q_perm,
+                    const void* k_perm, float* q_pool, float* k_pool, void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(q_perm, "q_perm"));
+  BSA_TRY(check_ptr(k_perm, "k_perm"));
+  BSA_TRY(check_ptr(q_pool, "q_pool"));
+  BSA_TRY(check_ptr(k_pool, "k_pool"));
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_pool(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
+                                   static_cast<const __nv_bfloat16*>(q_perm),
+                                   static_cast<const __nv_bfloat16*>(k_perm), q_pool, k_pool,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_pool launch");
+}
+
+bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const float* k_pool,
+                           int32_t* idx, int32_t* cnt, void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(q_pool, "q_pool"));
+  BSA_TRY(check_ptr(k_pool, "k_pool"));
+  BSA_TRY(check_ptr(idx, "idx"));
+  BSA_TRY(check_ptr(cnt, "cnt"));
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_select(g, q_pool, k_pool, idx, cnt, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_select_topk launch");
+}
+
+static bsa_status attention_common(const bsa_problem* prob, const void* layout_buf,
+                                   const void* q_perm, const void* k_perm, const void* v_perm,
+                                   const int32_t* idx, const int32_t* cnt, void* o_perm,
+                                   int32_t* dev_status, bool dense, void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(q_perm, "q_perm"));
+  BSA_TRY(check_ptr(k_perm, "k_perm"));
+  BSA_TRY(check_ptr(v_perm, "v_perm"));
+  BSA_TRY(check_ptr(o_perm, "o_perm"));
+  if (!dense) {
+    BSA_TRY(check_ptr(idx, "idx"));
+    BSA_TRY(check_ptr(cnt, "cnt"));
+  }
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+    return fail(BSA_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  BSA_TRY(check_device());
+  CUtensorMap maps[3];
+  BSA_TRY(make_map(&maps[0], g, q_perm, 128));
+  BSA_TRY(make_map(&maps[1], g, k_perm, 64));
+  BSA_TRY(make_map(&maps[2], g, v_perm, 64));
+  int32_t* status = dev_status;
+  if (!status) {
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dev_status_sink);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status sink)");
+  }
+  cudaError_t e = bsa::launch_attention(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
+                                        maps, idx, cnt, static_cast<__nv_bfloat16*>(o_perm),
+                                        status, dense, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "attention launch");
+}
+
+bsa_status bsa_sparse_attn_fwd(const bsa_problem* prob, const void* layout_buf,
+                               const void* q_perm, const void* k_perm, const void* v_perm,
+                               const int32_t* idx, const int32_t* cnt, void* o_perm,
+                               int32_t* dev_status, void* stream) {
+  return attention_common(prob, layout_buf, q_perm, k_perm, v_perm, idx, cnt, o_perm, dev_status,
+                          false, stream);
+}
+
+bsa_status bsa_dense_attn_fwd(const bsa_problem* prob, const void* layout_buf,
+                              const void* q_perm, const void* k_perm, const void* v_perm,
+                              void* o_perm, int32_t* dev_status, void* stream) {
+  return attention_common(prob, layout_buf, q_perm, k_perm, v_perm, nullptr, nullptr, o_perm,
+                          dev_status, true, stream);
+}
+
+bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const void* o_perm,
+                         void* o_raster, int64_t stride_b, int64_t stride_n, int64_t stride_h,
+                         void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(o_perm, "o_perm"));
+  BSA_TRY(check_ptr(o_raster, "o_raster"));
+  BSA_TRY(check_strides(g, stride_b, stride_n, stride_h, "o_raster"));
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_unpermute(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
+                                        static_cast<const __nv_bfloat16*>(o_perm),
+                                        static_cast<__nv_bfloat16*>(o_raster), stride_b,
+                                        stride_n, stride_h, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_unpermute launch");
+}
+
+bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int64_t hist7[7],
+                            void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  if (!hist7) return fail(BSA_ERR_INVALID_ARG, "hist7 is NULL");
+  for (int i = 0; i < 7; ++i) hist7[i] = 0;
+  if (g.mode == BSA_BLOCK_FIXED_444) {
+    hist7[0] = int64_t(g.B) * g.nbv;
+    return BSA_OK;
+  }
+  BSA_TRY(check_device());
+  const size_t n = size_t(g.B) * g.nreg;
+  unsigned char* host = static_cast<unsigned char*>(malloc(n));
+  if (!host) return fail(BSA_ERR_INVALID_ARG, "host allocation of %zu bytes failed", n);
+  const char* src = static_cast<const char*>(layout_buf) + bsa::layout_map(g).codes;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(host, src, n, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    free(host);
+    return cuda_fail(e, "bsa_layout_stats copy");
+  }
+  for (size_t i = 0; i < n; ++i) hist7[host[i] < 7 ? host[i] : 0] += 8;
+  free(host);
+  return BSA_OK;
+}
+
+const char* bsa_status_string(bsa_status s) {
+  switch (s) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+    case BSA_ERR_SHAPE: return "BSA_ERR_SHAPE";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
+    case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+  }
+  return "BSA_ERR_UNKNOWN";
+}
+
+const char* bsa_last_error(void) { return g_last_error; }
+
+}  // extern "C"

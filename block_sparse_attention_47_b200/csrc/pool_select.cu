@@ -1,0 +1,219 @@
+// Block mean pooling and top-k key-block selection.
+//
+// Pooling (Prism / Kandinsky 6 speed ablation, oh-my-gpu.com, section
+// "같은 계산량 안에서 볼 곳을 고르는 Prism": a block is judged by the mean of
+// its 64 tokens): pad slots are zero in block order, so the mean is the sum
+// of the 64 rows divided by the block's valid count.  HBM-bound.
+//
+// Selection (same section: keep the most relevant key blocks, 25 % at
+// sparsity 0.75; Ref2VA VSA, pulmap.app, section "조건 토큰은 왜 다르게
+// 다루나": the conditioning prefix is always kept and top-k runs over video
+// key blocks only).  Scores are fp32 dot products of the pooled means; the
+// k-th largest is found by an exact 4-pass radix select on order-preserving
+// 32-bit keys, then a warp compacts the winners in ascending index order, so
+// ties at the threshold go to the lowest indices and the list comes out
+// sorted.  The score matrix never leaves shared memory.
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+// ---- pooling --------------------------------------------------------------
+// One CTA per (block, head, batch) for both Q and K: thread (r, v) sums rows
+// r, r+16, r+32, r+48 of 16-byte channel vector v, then a shared reduction.
+constexpr int kPoolThreads = 256;
+
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(
+    Geo g, const int32_t* __restrict__ bcount, const __nv_bfloat16* __restrict__ qp,
+    const __nv_bfloat16* __restrict__ kp, float* __restrict__ qpool, float* __restrict__ kpool) {
+  const int j = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int vec = g.d / 8;            // 16 (d=128) or 8 (d=64)
+  const int groups = kPoolThreads / vec;  // row groups
+  const int v = threadIdx.x % vec, rg = threadIdx.x / vec;
+  const int64_t row0 = (int64_t(b) * g.h + hh) * g.N + int64_t(j) * kBlock;
+  __shared__ float red[2][kPoolThreads / 8][129];
+  for (int which = 0; which < 2; ++which) {
+    const __nv_bfloat16* x = which ? kp : qp;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int r = rg; r < kBlock; r += groups) {
+      const uint4 u = *reinterpret_cast<const uint4*>(x + (row0 + r) * g.d + v * 8);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[which][rg][v * 8 + i] = acc[i];
+  }
+  __syncthreads();
+  const float inv = 1.0f / float(bcount[int64_t(b) * g.nb + j]);
+  const int64_t out0 = ((int64_t(b) * g.h + hh) * g.nb + j) * g.d;
+  for (int c = threadIdx.x; c < 2 * g.d; c += kPoolThreads) {
+    const int which = c / g.d, ch = c % g.d;
+    float s = 0.f;
+    for (int r = 0; r < groups; ++r) s += red[which][r][ch];
+    (which ? kpool : qpool)[out0 + ch] = s * inv;
+  }
+}
+
+// ---- selection --------------------------------------------------------------
+constexpr int kSelThreads = 256;
+constexpr int kSelRows = 8;  // query blocks per CTA, one per warp in the top-k phase
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// dynamic smem: q rows [kSelRows][d] fp32, keys [kSelRows][nbv] u32,
+// histograms [8 warps][256] u32
+__global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, const float* __restrict__ qpool,
+                                                             const float* __restrict__ kpool,
+                                                             int32_t* __restrict__ idx,
+                                                             int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* sq = reinterpret_cast<float*>(smem);
+  uint32_t* skey = reinterpret_cast<uint32_t*>(sq + kSelRows * g.d);
+  uint32_t* shist = skey + kSelRows * g.nbv;
+
+  const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * kSelRows;  // first video query block of this CTA
+  const int rows = min(kSelRows, g.nbv - i0);
+  const int64_t pool0 = int64_t(bh) * g.nb * g.d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // prefix query blocks attend densely: mark them once per (b, h)
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < g.nbp; i += kSelThreads) cnt[int64_t(bh) * g.nb + i] = -1;
+
+  for (int e = threadIdx.x; e < kSelRows * g.d; e += kSelThreads) {
+    const int r = e / g.d, c = e % g.d;
+    sq[e] = r < rows ? qpool[pool0 + int64_t(g.nbp + i0 + r) * g.d + c] : 0.f;
+  }
+  __syncthreads();
+
+  // scores: thread per key block, all rows of the CTA at once
+  for (int jv = threadIdx.x; jv < g.nbv; jv += kSelThreads) {
+    const float4* kr = reinterpret_cast<const float4*>(kpool + pool0 + int64_t(g.nbp + jv) * g.d);
+    float acc[kSelRows];
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
+    for (int c4 = 0; c4 < g.d / 4; ++c4) {
+      const float4 kv = __ldg(kr + c4);
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r) {
+        const float4 qv = reinterpret_cast<const float4*>(sq + r * g.d)[c4];
+        acc[r] = fmaf(qv.x, kv.x, acc[r]);
+        acc[r] = fmaf(qv.y, kv.y, acc[r]);
+        acc[r] = fmaf(qv.z, kv.z, acc[r]);
+        acc[r] = fmaf(qv.w, kv.w, acc[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r) skey[r * g.nbv + jv] = order_key(acc[r]);
+  }
+  __syncthreads();
+
+  // top-k: one warp per query row
+  if (warp < rows) {
+    const uint32_t* key = skey + warp * g.nbv;
+    uint32_t* hist = shist + warp * 256;
+    uint32_t prefix = 0;  // high bits decided so far
+    int want = g.keep;    // how many still to take among keys matching prefix
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      const uint32_t hi_mask = pass ? (0xFFFFFFFFu << (32 - 8 * pass)) : 0u;
+      for (int i = lane; i < 256; i += 32) hist[i] = 0;
+      __syncwarp();
+      for (int jv = lane; jv < g.nbv; jv += 32) {
+        const uint32_t u = key[jv];
+        if ((u & hi_mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFF], 1u);
+      }
+      __syncwarp();
+      // find the digit D: count(digit > D) < want <= count(digit >= D).
+      // lane l owns digits [8*(31-l), 8*(31-l)+8), scanned from the top.
+      uint32_t local[8];
+      uint32_t tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        local[q] = hist[8 * (31 - lane) + (7 - q)];  // descending digits
+        tot += local[q];
+      }
+      uint32_t incl = tot;  // inclusive prefix over lanes (higher digits first)
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      const uint32_t excl = incl - tot;
+      const bool mine = (excl < uint32_t(want)) && (incl >= uint32_t(want));
+      const uint32_t who = __ballot_sync(0xffffffffu, mine);
+      const int src = __ffs(who) - 1;
+      int digit = 0, above = 0;
+      if (mine) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (run + local[q] >= uint32_t(want)) {
+            digit = 8 * (31 - lane) + (7 - q);
+            above = int(run);
+            break;
+          }
+          run += local[q];
+        }
+      }
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      want -= above;
+      prefix |= uint32_t(digit) << shift;
+      __syncwarp();
+    }
+    // prefix is now the exact key of the k-th best; `want` ties are needed
+    const uint32_t thr = prefix;
+    const int64_t row = int64_t(bh) * g.nb + g.nbp + i0 + warp;
+    int32_t* out = idx + row * g.kcap;
+    for (int p = lane; p < g.nbp; p += 32) out[p] = p;
+    int written = g.nbp, ties = 0;
+    for (int base = 0; base < g.nbv; base += 32) {
+      const int jv = base + lane;
+      const uint32_t u = jv < g.nbv ? key[jv] : 0u;
+      const bool tie = (jv < g.nbv) && (u == thr);
+      const uint32_t tie_bal = __ballot_sync(0xffffffffu, tie);
+      const int tie_rank = ties + __popc(tie_bal & ((1u << lane) - 1u));
+      const bool take = (jv < g.nbv) && (u > thr || (tie && tie_rank < want));
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      if (take) out[written + __popc(bal & ((1u << lane) - 1u))] = g.nbp + jv;
+      written += __popc(bal);
+      ties += __popc(tie_bal);
+    }
+    if (lane == 0) cnt[row] = g.nbp + g.keep;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* qp,
+                        const __nv_bfloat16* kp, float* qpool, float* kpool, cudaStream_t st) {
+  pool_kernel<<<dim3(g.nb, g.h, g.B), kPoolThreads, 0, st>>>(g, lp.bcount, qp, kp, qpool, kpool);
+  return cudaGetLastError();
+}
+
+size_t select_smem_bytes(const Geo& g) {
+  return sizeof(float) * kSelRows * g.d + sizeof(uint32_t) * kSelRows * g.nbv +
+         sizeof(uint32_t) * (kSelThreads / 32) * 256;
+}
+
+cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, int32_t* idx,
+                          int32_t* cnt, cudaStream_t st) {
+  const size_t smem = select_smem_bytes(g);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  const int ctas = (g.nbv + kSelRows - 1) / kSelRows;
+  select_kernel<<<dim3(ctas, g.B * g.h), kSelThreads, smem, st>>>(g, qpool, kpool, idx, cnt);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

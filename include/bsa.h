@@ -1,0 +1,197 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) block-sparse video self-attention
+ * library, libbsa.so.
+ *
+ * What the library computes.  Tokens of a video latent lie on a T x H x W
+ * grid (Prism / Kandinsky 6 speed ablation, oh-my-gpu.com, section
+ * "토큰 수의 제곱으로 느는 어텐션 비용": 720p, 121 frames -> 32 x 48 x 80,
+ * 122,880 tokens with padding).  They are grouped into 64-token blocks,
+ * either fixed 4x4x4 cubes or, per 8x8x8 region, a 64-token box whose
+ * short side lies on the axis along which K changes most (same page,
+ * section "같은 계산량 안에서 볼 곳을 고르는 Prism").  Q and K are mean-pooled
+ * per block; every query block keeps the key blocks with the highest
+ * pooled score (sparsity 0.75 keeps 25 %, 480 of 1,920), and attention runs
+ * over the kept 64 x 64 tiles only, so empty tiles are skipped outright
+ * (Sparse VideoGen on TPU, aibase.it, section "이론적 sparsity와 물리적
+ * sparsity의 차이").  An optional conditioning prefix (text, reference
+ * image, reference audio) sits in segment-pure blocks that every query
+ * keeps and whose queries attend densely (Ref2VA VSA, pulmap.app, section
+ * "조건 토큰은 왜 다르게 다루나").
+ *
+ * The call sequence for one attention layer:
+ *   bsa_layout -> bsa_permute (Q, K, V) -> bsa_pool -> bsa_select_topk
+ *   -> bsa_sparse_attn_fwd -> bsa_unpermute
+ * bsa_dense_attn_fwd is the same attention kernel over every tile (the
+ * speed-up denominator).
+ *
+ * Conventions (every entry point):
+ *   - The caller owns all memory.  The library allocates no device memory;
+ *     sizes of every buffer come from bsa_query_sizes.
+ *   - Device pointers must be 16-byte aligned; the innermost (head_dim)
+ *     dimension of every tensor is contiguous.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*; NULL = legacy default stream).  Arguments are validated on the
+ *     host before anything is launched: on any error nothing is launched and
+ *     a bsa_status other than BSA_OK is returned; bsa_last_error() then
+ *     gives a message (per calling thread).
+ *   - Errors found on the device (a bounded wait that ran out) are written
+ *     to the optional `dev_status` int32 device word as a bsa_status value;
+ *     the word is never cleared by the library.
+ *   - Token order "raster": prefix segment s occupies
+ *     [off_s, off_s + pad64(prefix_len[s])) with its pad tokens at the end,
+ *     then video token (t, y, x) sits at P + (t*H + y)*W + x, where
+ *     P = sum of padded segment lengths and N = P + T*H*W.
+ *     Token order "perm" (block order): slot s of block j = j*64 + s; the
+ *     prefix keeps raster order; video blocks follow the layout.
+ *   - Raster tensors are [B, N, heads, head_dim] bf16 addressed with element
+ *     strides (stride_b, stride_n, stride_h); permuted tensors are
+ *     contiguous [B, heads, N, head_dim] bf16.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSA_MAX_PREFIX_SEGMENTS 8
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad scalar */
+  BSA_ERR_SHAPE = 2,       /* grid, block or prefix geometry not allowed */
+  BSA_ERR_UNSUPPORTED = 3, /* head_dim other than 64 or 128, no sm_100 GPU */
+  BSA_ERR_WORKSPACE = 4,   /* a caller buffer is too small */
+  BSA_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
+  BSA_ERR_TIMEOUT = 6      /* device-side bounded wait ran out */
+} bsa_status;
+
+typedef enum {
+  BSA_BLOCK_FIXED_444 = 0,  /* 4x4x4 token cubes, blocks in (bt,bh,bw) raster order */
+  BSA_BLOCK_DYNAMIC_888 = 1 /* one of 7 64-token shapes per 8x8x8 region */
+} bsa_block_mode;
+
+/* One attention call.  Every field must be set; there are no defaults. */
+typedef struct {
+  int32_t B, heads, head_dim;    /* head_dim in {64, 128} */
+  int32_t T, H, W;               /* padded grid; multiples of 4 (8 in dynamic mode) */
+  int32_t T_valid, H_valid, W_valid; /* valid extents; trailing indices are pad.
+                                        T-T_valid etc. < 4 (fixed) / < 2 (dynamic)
+                                        so that no block is all pad */
+  int32_t n_prefix_segments;     /* 0..BSA_MAX_PREFIX_SEGMENTS */
+  int32_t prefix_len[BSA_MAX_PREFIX_SEGMENTS]; /* valid tokens per segment (>= 1) */
+  int32_t keep_blocks;           /* video key blocks kept per video query block,
+                                    1..n_video_blocks (see bsa_keep_count) */
+  int32_t block_mode;            /* bsa_block_mode */
+  float dyn_tau;                 /* dynamic mode: a region keeps 4x4x4 when
+                                    max(v) < dyn_tau*min(v); finite, >= 1 */
+  float softmax_scale;           /* logit scale, finite and > 0 (1/sqrt(head_dim)
+                                    for standard attention) */
+} bsa_problem;
+
+/* Sizes derived from a problem (all byte counts are for the whole batch). */
+typedef struct {
+  int64_t n_tokens;          /* N = P + T*H*W */
+  int64_t n_prefix_tokens;   /* P */
+  int64_t n_blocks;          /* nb = N / 64 */
+  int64_t n_prefix_blocks;   /* nbp = P / 64 */
+  int64_t n_video_blocks;    /* nbv = T*H*W / 64 */
+  int64_t n_regions;         /* dynamic mode: (T/8)(H/8)(W/8); else 0 */
+  int64_t list_capacity;     /* kcap = nbp + keep_blocks: ints per index-list row */
+  size_t layout_bytes;       /* layout buffer (bsa_layout output) */
+  size_t perm_tensor_bytes;  /* one permuted tensor [B, heads, N, head_dim] bf16 */
+  size_t raster_tensor_bytes;/* one dense raster tensor [B, N, heads, head_dim] bf16 */
+  size_t pool_bytes;         /* one pooled tensor [B, heads, nb, head_dim] fp32 */
+  size_t idx_bytes;          /* index lists [B, heads, nb, kcap] int32 */
+  size_t cnt_bytes;          /* list lengths [B, heads, nb] int32 */
+} bsa_sizes;
+
+/* Kept video key blocks per video query block for a keep ratio r = 1 - sparsity:
+ * max(1, ceil(r*n - 1e-9)), at most n (Prism speed ablation, section
+ * "같은 계산량 안에서 볼 곳을 고르는 Prism": sparsity 0.75 -> 480 of 1,920).
+ * Returns -1 for n < 1 or r outside [0, 1] or not finite.  Host only. */
+int32_t bsa_keep_count(int32_t n_blocks, double keep_ratio);
+
+/* Validate `prob` and fill `out`.  Host only; no CUDA call. */
+bsa_status bsa_query_sizes(const bsa_problem* prob, bsa_sizes* out);
+
+/* Build the block layout into `layout_buf` (layout_bytes, caller-owned).
+ * Fixed mode: a closed-form permutation; k_raster may be NULL.
+ * Dynamic mode (the Prism section on 8x8x8 regions): per (batch, region)
+ *   v_a = mean |K(p+e_a) - K(p)| over heads, channels and adjacent valid
+ *   in-region token pairs along axis a (fp32 sums); the region keeps 4x4x4
+ *   when max(v) < dyn_tau*min(v) or max(v) == 0, otherwise the axes ranked
+ *   by (v descending, t<h<w) get block sides 2, 4, 8.  The shape is shared
+ *   by all heads.  k_raster is K in raster order with element strides
+ *   (stride_b, stride_n, stride_h).
+ * layout_buf holds: slot->raster and raster->slot maps (int32 [B, N], bit 31
+ * set for pad tokens), per-block valid-slot masks (uint64 [B, nb]) and
+ * counts (int32 [B, nb]), and shape codes (uint8 [B, n_regions]). */
+bsa_status bsa_layout(const bsa_problem* prob, const void* k_raster, int64_t stride_b,
+                      int64_t stride_n, int64_t stride_h, void* layout_buf, void* stream);
+
+/* Gather one raster tensor into block order: x_perm[b, h, s, :] =
+ * x_raster[b, perm[b][s], h, :], pad slots written as 0 (token permutation,
+ * Sparse VideoGen on TPU, section "실무에서 배울 최적화 기준"). */
+bsa_status bsa_permute(const bsa_problem* prob, const void* layout_buf, const void* x_raster,
+                       int64_t stride_b, int64_t stride_n, int64_t stride_h, void* x_perm,
+                       void* stream);
+
+/* Block means of Q and K over each block's valid tokens, fp32
+ * [B, heads, nb, head_dim] (Prism section: a block is judged by the mean of
+ * its 64 tokens). */
+bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void* q_perm,
+                    const void* k_perm, float* q_pool, float* k_pool, void* stream);
+
+/* Per (batch, head) and video query block i: scores S[i, j] = q_pool[i] .
+ * k_pool[j] (fp32) over video key blocks j; keep the keep_blocks best by
+ * (score descending, index ascending).  Row i of idx [B, heads, nb, kcap]
+ * receives every prefix block then the kept video blocks, ascending;
+ * cnt[i] = nbp + keep_blocks.  Prefix query blocks attend densely:
+ * cnt = -1 and their idx row is left untouched (Ref2VA VSA, section
+ * "조건 토큰은 왜 다르게 다루나"). */
+bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const float* k_pool,
+                           int32_t* idx, int32_t* cnt, void* stream);
+
+/* Block-sparse attention over the kept tiles: for each query block i and
+ * each key block j in idx row i (all blocks when cnt[i] == -1), logits
+ * softmax_scale * q.k over the valid keys of j, online softmax, O = P V,
+ * normalised; pad query rows are written as 0.  Inputs and output are in
+ * block order [B, heads, N, head_dim] bf16; accumulation is fp32.
+ * Index rows must be strictly ascending with entries in [0, nb). */
+bsa_status bsa_sparse_attn_fwd(const bsa_problem* prob, const void* layout_buf,
+                               const void* q_perm, const void* k_perm, const void* v_perm,
+                               const int32_t* idx, const int32_t* cnt, void* o_perm,
+                               int32_t* dev_status, void* stream);
+
+/* The same attention over every tile (pad keys masked): the dense comparator. */
+bsa_status bsa_dense_attn_fwd(const bsa_problem* prob, const void* layout_buf,
+                              const void* q_perm, const void* k_perm, const void* v_perm,
+                              void* o_perm, int32_t* dev_status, void* stream);
+
+/* Scatter block-ordered rows back to raster order: o_raster[b, n, h, :] =
+ * o_perm[b, h, iperm[b][n], :]; pad tokens written as 0. */
+bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const void* o_perm,
+                         void* o_raster, int64_t stride_b, int64_t stride_n, int64_t stride_h,
+                         void* stream);
+
+/* Histogram of video blocks by shape code over the whole batch (hist7[0]
+ * counts 4x4x4 blocks; each dynamic region adds 8 blocks of its code), the
+ * block-shape log of the Prism speed ablation (section "동적 블록을 켜도
+ * 그대로였던 속도").  Dynamic mode synchronises `stream` and copies the codes
+ * to the host.  Fixed mode: hist7[0] = B * n_video_blocks, no CUDA call. */
+bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int64_t hist7[7],
+                            void* stream);
+
+/* Name of a status code. */
+const char* bsa_status_string(bsa_status status);
+/* Message of the last failed call on this thread ("" if none). */
+const char* bsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H */

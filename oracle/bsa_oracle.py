@@ -164,7 +164,7 @@ def dynamic_perm(geo, codes):
     return np.asarray(perm, dtype=np.int64)
 
 
-def region_variation(geo, k_raster_b):
+def region_variation(geo, k_raster_b, regions=None):
     """float64 [n_regions, 3]: per-axis mean |delta K| of each 8x8x8 region.
 
     k_raster_b: one batch element of K, [N, heads, d] (any float dtype).
@@ -172,16 +172,21 @@ def region_variation(geo, k_raster_b):
     adjacent in-region tokens along axis a that are both valid ([PRISM]
     Prism section: the change along t, h, w is measured per region).
     A region with no valid pair along some axis reports NaN for that axis.
+    With `regions` given, only those rows are evaluated (the others are 0).
     """
     T, H, W = geo.T, geo.H, geo.W
     valid = geo.token_valid()[geo.P:].reshape(T, H, W)
     vid = k_raster_b[geo.P:]
     nr_t, nr_h, nr_w = T // 8, H // 8, W // 8
     out = np.zeros((nr_t * nr_h * nr_w, 3))
-    r = 0
+    wanted = None if regions is None else set(int(r) for r in regions)
+    r = -1
     for rt in range(nr_t):
         for rh in range(nr_h):
             for rw in range(nr_w):
+                r += 1
+                if wanted is not None and r not in wanted:
+                    continue
                 idx = np.array([[[(8 * rt + a) * H * W + (8 * rh + b) * W + 8 * rw + c
                                   for c in range(8)] for b in range(8)] for a in range(8)])
                 x = np.asarray(vid[idx.reshape(-1)], dtype=np.float64)
@@ -197,7 +202,6 @@ def region_variation(geo, k_raster_b):
                         out[r, axis] = np.nan
                     else:
                         out[r, axis] = diff[pair_ok].mean()
-                r += 1
     return out
 
 
@@ -294,19 +298,23 @@ def topk_row(scores_row, k):
     return sorted(order[:k])
 
 
-def select(geo, q_pool, k_pool, keep):
+def select(geo, q_pool, k_pool, keep, rows=None):
     """Kept key-block lists for every query block of one (batch, head).
 
     Returns a list of length nb; entry i is a sorted int64 array of kept key
     blocks.  Prefix query blocks keep every block; video query blocks keep
     every prefix block plus their top-`keep` video blocks ([PRISM] Prism
-    section; [REF2VA] condition-token section).
+    section; [REF2VA] condition-token section).  With `rows` given, only
+    those query blocks are evaluated (the others are None).
     """
     S = block_scores_f32(geo, q_pool, k_pool)
     lists = []
     every = np.arange(geo.nb, dtype=np.int64)
+    wanted = None if rows is None else set(int(r) for r in rows)
     for i in range(geo.nb):
-        if i < geo.nbp:
+        if wanted is not None and i not in wanted:
+            lists.append(None)
+        elif i < geo.nbp:
             lists.append(every)
         else:
             vid = np.asarray(topk_row(S[i - geo.nbp], keep), dtype=np.int64) + geo.nbp

@@ -1,0 +1,142 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads and
+exports every symbol include/bsa.h declares, sizes match the workload
+arithmetic, the keep-count closed form agrees with the oracle's exact
+rational version, and invalid arguments are rejected before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import block_sparse_attention_47_b200 as bsa
+from gen import CONFIGS, SWEEP_KEEP_RATIOS, config, derived_sizes
+from oracle import bsa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from block_sparse_attention_47_b200 import build
+    build.build()
+    return bsa.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) == 12, names
+    for n in names:
+        assert hasattr(bsa.lib(), n), n
+    assert set(names) == set(bsa._SIGS), "binding and header disagree"
+
+
+def test_struct_layout_matches_header():
+    # 10 int32 + 8 int32 prefix + keep + mode + 2 floats
+    assert ctypes.sizeof(bsa.Problem) == 4 * (10 + 8 + 2 + 2)
+    assert ctypes.sizeof(bsa.Sizes) == 8 * 13
+
+
+def test_keep_count_matches_oracle():
+    for n in (1, 2, 3, 7, 32, 504, 1440, 1920, 2016, 5000):
+        for r in (0.0, 0.001, 0.01, 0.03, 0.05, 0.0625, 0.0664, 0.0793, 0.1, 0.25, 0.5, 0.75, 1.0):
+            assert bsa.keep_count(n, r) == O.keep_count(n, r), (n, r)
+    assert bsa.keep_count(0, 0.5) == -1
+    assert bsa.keep_count(10, 1.5) == -1
+    assert bsa.keep_count(10, float("nan")) == -1
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_query_sizes_match_workload(name):
+    cfg = config(name)
+    p = bsa.Problem.make(**cfg)
+    s = bsa.query_sizes(p)
+    d = derived_sizes(cfg)
+    assert (s.n_tokens, s.n_prefix_tokens, s.n_blocks, s.n_prefix_blocks, s.n_video_blocks) == \
+        (d["N"], d["P"], d["nb"], d["nbp"], d["nbv"])
+    assert s.list_capacity == d["nbp"] + O.keep_count(d["nbv"], cfg["keep_ratio"])
+    assert s.perm_tensor_bytes == cfg["B"] * cfg["heads"] * d["N"] * cfg["head_dim"] * 2
+    assert s.idx_bytes == cfg["B"] * cfg["heads"] * d["nb"] * s.list_capacity * 4
+    if cfg["block_mode"] == 1:
+        assert s.n_regions == (cfg["T"] // 8) * (cfg["H"] // 8) * (cfg["W"] // 8)
+
+
+def test_sweep_keep_counts():
+    nbv = derived_sizes(config("sweep"))["nbv"]
+    assert [bsa.keep_count(nbv, r) for r in SWEEP_KEEP_RATIOS] == [360, 144, 115, 96, 72, 44, 15]
+
+
+def base(**kw):
+    d = dict(B=1, heads=2, head_dim=64, T=8, H=16, W=16, keep_blocks=8)
+    d.update(kw)
+    return bsa.Problem.make(**d)
+
+
+BAD_PROBLEMS = [
+    (dict(head_dim=96), 3), (dict(head_dim=0), 3), (dict(B=0), 2), (dict(heads=0), 2),
+    (dict(T=6), 2), (dict(W=0), 2), (dict(H_valid=12), 2), (dict(T_valid=0), 2),
+    (dict(T_valid=9), 2), (dict(keep_blocks=0), 2), (dict(keep_blocks=33), 2),
+    (dict(block_mode=2), 1), (dict(block_mode=1, W=12), 2), (dict(block_mode=1, H_valid=14), 2),
+    (dict(block_mode=1, dyn_tau=float("nan")), 1), (dict(block_mode=1, dyn_tau=0.5), 1),
+    (dict(softmax_scale=0.0), 1), (dict(softmax_scale=float("inf")), 1),
+    (dict(prefix=(0,)), 2),
+]
+
+
+@pytest.mark.parametrize("kw,status", BAD_PROBLEMS, ids=[str(k) for k, _ in BAD_PROBLEMS])
+def test_invalid_problems_rejected(kw, status):
+    p = base(**kw)
+    s = bsa.Sizes()
+    rc = bsa.lib().bsa_query_sizes(ctypes.byref(p), ctypes.byref(s))
+    assert rc == status, (rc, bsa.lib().bsa_last_error())
+    assert bsa.lib().bsa_last_error().decode()
+    # every entry point rejects it the same way, before touching CUDA
+    rc2 = bsa.lib().bsa_permute(ctypes.byref(p), 16, 16, 8, 8, 8, 16, None)
+    assert rc2 == status
+
+
+def test_too_many_prefix_segments():
+    p = base()
+    p.n_prefix_segments = 9
+    assert bsa.lib().bsa_query_sizes(ctypes.byref(p), ctypes.byref(bsa.Sizes())) == 2
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = base()
+    L = bsa.lib()
+    assert L.bsa_permute(ctypes.byref(p), None, 16, 8, 8, 8, 16, None) == 1
+    assert b"layout_buf" in L.bsa_last_error()
+    assert L.bsa_permute(ctypes.byref(p), 16, 24, 8, 8, 8, 16, None) == 1
+    assert b"aligned" in L.bsa_last_error()
+    assert L.bsa_permute(ctypes.byref(p), 16, 16, 8, 12, 8, 16, None) == 1  # stride not %8
+    assert L.bsa_sparse_attn_fwd(ctypes.byref(p), 16, 16, 16, 16, None, 16, 16, None, None) == 1
+    assert L.bsa_sparse_attn_fwd(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, 2, None) == 1
+    assert L.bsa_select_topk(ctypes.byref(p), 16, 16, 16, None, None) == 1
+    assert L.bsa_pool(ctypes.byref(p), 16, 16, 16, 16, 8, None) == 1
+    assert L.bsa_unpermute(ctypes.byref(p), 16, 16, None, 8, 8, 8, None) == 1
+    assert L.bsa_layout(None, None, 0, 0, 0, 16, None) == 1
+    hist = (ctypes.c_int64 * 7)()
+    assert L.bsa_layout_stats(ctypes.byref(p), 16, None, None) == 1
+    # fixed-mode stats need no device
+    assert L.bsa_layout_stats(ctypes.byref(p), 16, hist, None) == 0
+    assert list(hist) == [32, 0, 0, 0, 0, 0, 0]
+
+
+def test_status_strings():
+    for code, name in bsa.STATUS.items():
+        assert bsa.lib().bsa_status_string(code).decode() == name
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_call_without_gpu_reports_cuda_error():
+    p = base()
+    rc = bsa.lib().bsa_permute(ctypes.byref(p), 16, 16, 8, 8, 8, 16, None)
+    assert rc == 5
+    with pytest.raises(bsa.BSAError):
+        bsa._check(rc)

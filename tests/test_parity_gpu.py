@@ -1,0 +1,219 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle on
+seeded inputs small enough for the oracle to finish in seconds, spanning
+several tiles, a ragged tail (odd block count, padded grid, padded prefix
+segments), keep = 1, keep = everything, dynamic block shapes and d = 64/128.
+
+Bars: bit-exact for maps, permutation and index lists (lists up to the
+documented near-tie band); max-abs <= 2e-2 and relative L2 <= 5e-3 for
+attention outputs against fp64."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_47_b200 as bsa
+from gen import config
+from oracle import bsa_oracle as O
+from parity_helpers import (GpuRun, assert_close, check_list_row, decode_map, lists_to_device,
+                            oracle_bh, problem, scale_of, seeded_inputs, to_np64)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": config("tiny"),
+    "ragged": dict(config("tiny"), B=2, heads=3, head_dim=128, T=8, H=12, W=20, T_valid=7,
+                   H_valid=10, W_valid=17, prefix=(40, 64, 1), keep_ratio=0.3, name="ragged"),
+    "dyn": dict(config("tiny"), B=2, heads=2, head_dim=128, T=8, H=16, W=24, T_valid=8,
+                H_valid=16, W_valid=24, block_mode=1, blobs=2, keep_ratio=0.25, name="dyn"),
+    "dyn_pad": dict(config("tiny"), B=1, heads=2, head_dim=64, T=8, H=16, W=16, T_valid=7,
+                    H_valid=15, W_valid=16, block_mode=1, blobs=1, prefix=(100,),
+                    keep_ratio=0.4, name="dyn_pad"),
+    "keep1": dict(config("tiny"), keep_ratio=0.0, name="keep1"),
+    "keepall": dict(config("tiny"), keep_ratio=1.0, prefix=(64, 10), name="keepall"),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built(cuda_ok):
+    from block_sparse_attention_47_b200 import build
+    build.build()
+    bsa.lib()
+
+
+@pytest.fixture(scope="module", params=sorted(SMALL))
+def case(request):
+    cfg = SMALL[request.param]
+    (q, k, v), (qn, kn, vn) = seeded_inputs(cfg, seed=42000 + len(request.param))
+    run = GpuRun(cfg, q, k, v)
+    geo = O.Geometry(cfg)
+    lay = O.layout(cfg, kn)
+    return dict(cfg=cfg, geo=geo, run=run, dev=(q, k, v), host=(qn, kn, vn), lay=lay)
+
+
+def test_layout_maps_bit_exact(case):
+    geo, run = case["geo"], case["run"]
+    valid = geo.token_valid()
+    for b in range(geo.B):
+        operm = case["lay"][b][0]
+        ocodes = case["lay"][b][1]
+        if ocodes is not None and not np.array_equal(ocodes, run.codes[b]):
+            pytest.fail("shape codes differ (see test_dynamic_codes)")
+        gperm, gpad = decode_map(run.perm[b])
+        assert np.array_equal(gperm, operm)
+        assert np.array_equal(gpad, ~valid[operm])
+        ginv, ipad = decode_map(run.iperm[b])
+        assert np.array_equal(ginv[operm], np.arange(geo.N))
+        assert np.array_equal(ipad, ~valid)
+        ok = O.slot_valid(geo, operm).reshape(geo.nb, 64)
+        want_mask = (ok.astype(np.uint64) << np.arange(64, dtype=np.uint64)).sum(axis=1)
+        assert np.array_equal(run.bmask[b].view(np.uint64), want_mask)
+        assert np.array_equal(run.bcount[b], ok.sum(axis=1))
+
+
+def test_dynamic_codes(case):
+    cfg, geo, run = case["cfg"], case["geo"], case["run"]
+    if cfg["block_mode"] != 1:
+        pytest.skip("fixed layout")
+    kn = case["host"][1]
+    for b in range(geo.B):
+        v = O.region_variation(geo, kn[b])
+        want = np.array([O.shape_code(v[r], cfg["dyn_tau"]) for r in range(len(v))])
+        got = run.codes[b].astype(np.int64)
+        for r in np.nonzero(got != want)[0]:
+            vr = v[r]
+            top = vr.max()
+            near = (abs(top - cfg["dyn_tau"] * vr.min()) < 1e-4 * top
+                    or np.sort(np.abs(vr[:, None] - vr[None, :]).ravel())[3] < 1e-4 * top)
+            assert near, "region %d: code %d vs oracle %d, v=%s" % (r, got[r], want[r], vr)
+    hist = bsa.layout_stats(run.prob, run.attn.layout_buf)
+    assert sum(hist) == geo.B * geo.nbv
+    assert hist == [8 * int((run.codes == c).sum()) for c in range(7)]
+
+
+def test_permute_bit_exact(case):
+    geo, run = case["geo"], case["run"]
+    qn, kn, vn = case["host"]
+    gq, gk, gv = (to_np64(t) for t in (run.attn.qp, run.attn.kp, run.attn.vp))
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        for hh in range(geo.h):
+            oq, ok_, ov = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            assert np.array_equal(gq[b, hh], oq)
+            assert np.array_equal(gk[b, hh], ok_)
+            assert np.array_equal(gv[b, hh], ov)
+
+
+def test_pool(case):
+    geo, run = case["geo"], case["run"]
+    qn, kn, vn = case["host"]
+    gq, gk = run.attn.q_pool.cpu().numpy(), run.attn.k_pool.cpu().numpy()
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        for hh in range(geo.h):
+            oq, ok_, _ = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            np.testing.assert_allclose(gq[b, hh], O.pool(geo, perm, oq), rtol=1e-5, atol=1e-5)
+            np.testing.assert_allclose(gk[b, hh], O.pool(geo, perm, ok_), rtol=1e-5, atol=1e-5)
+
+
+def test_select_lists(case):
+    cfg, geo, run = case["cfg"], case["geo"], case["run"]
+    qn, kn, vn = case["host"]
+    keep = run.prob.keep_blocks
+    idx, cnt = run.attn.idx.cpu().numpy(), run.attn.cnt.cpu().numpy()
+    exact = total = 0
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        for hh in range(geo.h):
+            oq, ok_, _ = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            S = O.block_scores_f32(geo, O.pool(geo, perm, oq), O.pool(geo, perm, ok_))
+            assert np.all(cnt[b, hh, :geo.nbp] == -1)
+            assert np.all(cnt[b, hh, geo.nbp:] == geo.nbp + keep)
+            for i in range(geo.nbp, geo.nb):
+                exact += check_list_row(idx[b, hh, i, :geo.nbp + keep], S[i - geo.nbp], keep, geo.nbp)
+                total += 1
+    assert exact >= 0.99 * total, "%d of %d lists differ from the oracle (near ties)" % (total - exact, total)
+
+
+def oracle_lists(case):
+    geo = case["geo"]
+    qn, kn, vn = case["host"]
+    keep = O.keep_count(geo.nbv, case["cfg"]["keep_ratio"])
+    out = []
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        per = []
+        for hh in range(geo.h):
+            oq, ok_, _ = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            per.append(O.select(geo, O.pool(geo, perm, oq), O.pool(geo, perm, ok_), keep))
+        out.append(per)
+    return out
+
+
+def test_attention_kernel_on_oracle_inputs(case):
+    """bsa_sparse_attn_fwd alone: permuted inputs and lists built by the
+    oracle, output compared block by block with the fp64 oracle."""
+    cfg, geo, run = case["cfg"], case["geo"], case["run"]
+    qn, kn, vn = case["host"]
+    lists = oracle_lists(case)
+    idx, cnt = lists_to_device(geo, lists, run.attn.sizes.list_capacity)
+    perm_t = [torch.empty_like(run.attn.qp) for _ in range(3)]
+    want = np.zeros((geo.B, geo.h, geo.N, geo.d))
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        for hh in range(geo.h):
+            parts = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            for t, x in zip(perm_t, parts):
+                t[b, hh] = torch.from_numpy(x).to(torch.bfloat16)
+            blocks = O.block_sparse_attention(geo, perm, *parts, lists[b][hh], scale_of(cfg))
+            want[b, hh] = np.concatenate([blocks[i] for i in range(geo.nb)])
+    o = torch.full_like(run.attn.qp, float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bsa.sparse_attn_fwd(run.prob, run.attn.layout_buf, *perm_t, idx, cnt, o, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = to_np64(o)
+    assert np.isfinite(got).all()
+    assert_close(got, want, cfg["name"])
+
+
+def test_end_to_end_raster(case):
+    cfg, geo, run = case["cfg"], case["geo"], case["run"]
+    qn, kn, vn = case["host"]
+    want, _, _, lists = O.forward(cfg, qn, kn, vn)
+    got = to_np64(run.out)
+    idx, cnt = run.attn.idx.cpu().numpy(), run.attn.cnt.cpu().numpy()
+    keep_rows = np.ones((geo.B, geo.h, geo.N), dtype=bool)  # raster tokens to compare
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        for hh in range(geo.h):
+            for i in range(geo.nbp, geo.nb):
+                if list(idx[b, hh, i, :cnt[b, hh, i]]) != list(lists[b][hh][i]):
+                    keep_rows[b, hh, perm[i * 64:(i + 1) * 64]] = False
+    assert keep_rows.mean() > 0.99
+    g = got.transpose(0, 2, 1, 3)[keep_rows]
+    w = want.transpose(0, 2, 1, 3)[keep_rows]
+    assert_close(g, w, cfg["name"])
+    valid = geo.token_valid()
+    assert not got[:, ~valid].any(), "pad tokens must come out as 0"
+
+
+def test_dense_kernel_matches_oracle_and_full_keep(case):
+    cfg, geo, run = case["cfg"], case["geo"], case["run"]
+    qn, kn, vn = case["host"]
+    o = torch.empty_like(run.attn.qp)
+    bsa.dense_attn_fwd(run.prob, run.attn.layout_buf, run.attn.qp, run.attn.kp, run.attn.vp, o)
+    torch.cuda.synchronize()
+    got = to_np64(o)
+    every = [[[np.arange(geo.nb)] * geo.nb for _ in range(geo.h)] for _ in range(geo.B)]
+    for b in range(geo.B):
+        perm = case["lay"][b][0]
+        for hh in range(geo.h):
+            parts = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            blocks = O.block_sparse_attention(geo, perm, *parts, every[b][hh], scale_of(cfg))
+            assert_close(got[b, hh], np.concatenate([blocks[i] for i in range(geo.nb)]), "dense")
+    if cfg["name"] == "keepall":
+        # keeping every block walks the same tiles in the same order
+        assert torch.equal(o, run.attn.op)
+
+
+def test_status_word_untouched(case):
+    assert int(case["run"].attn.status.item()) == 0
