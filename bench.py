@@ -1,0 +1,486 @@
+"""Benchmark of block-sparse video self-attention on B200.
+
+One step = one whole attention call over one batch of synthetic inputs:
+layout -> permute Q, K, V -> pool -> top-k select -> sparse attention ->
+unpermute, all through libbsa.so on one stream.  Default workload: the 720p
+121-frame clip (B=2 CFG pair, 24 heads of 128, 32x48x80 = 122,880 tokens,
+fixed 4x4x4 blocks, sparsity 0.75 = keep 480 of 1,920).  Metric: effective
+TFLOP/s counted on kept 64x64 tiles only (4*64*64*d FLOP per tile), plus
+ms per call and the fraction of the measured bf16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config 720p|720p_dyn|ref_prefix|lowres|sweep] [--keep-ratio r]
+                    [--sweep]   # keep-ratio sweep on the 1152x640 grid instead
+
+N > 1 runs under torchrun: each rank processes its own independent call
+(its own seeded inputs; the (batch, head) problems share nothing), no
+collective on the data path; `value` = all ranks' kept-tile FLOPs / the
+slowest rank's time (weak scaling).
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (one (batch, head), a seeded subset of query
+blocks per step) and reports the same metric for that sample.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "ms/call & effective TFLOP/s (kept tiles) at 122,880 tok, s=0.75; % BF16 peak"
+
+
+# ----------------------------------------------------------------------------
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kept_tiles(cfg, keep):
+    """64x64 tiles attention touches: video query blocks keep every prefix
+    block plus `keep` video blocks; prefix query blocks keep every block."""
+    s = derived_sizes(cfg)
+    per_bh = s["nbv"] * (s["nbp"] + keep) + s["nbp"] * s["nb"]
+    return cfg["B"] * cfg["heads"] * per_bh
+
+
+def dense_tiles(cfg):
+    s = derived_sizes(cfg)
+    return cfg["B"] * cfg["heads"] * s["nb"] * s["nb"]
+
+
+def tile_flops(cfg):
+    return 4 * 64 * 64 * cfg["head_dim"]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.tmp = None
+        self.target = self._gpu_id(device_index)
+
+    @staticmethod
+    def _gpu_id(i):
+        try:
+            u = str(torch.cuda.get_device_properties(i).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return str(i)
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.target, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:7]))
+                except ValueError:
+                    continue
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+def dist_setup(want_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != want_gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (want_gpus, world))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+STAGES = ("layout", "permute", "pool", "select", "attention", "unpermute")
+
+
+def run_step(bsa, attn, q, k, v, out, ev):
+    """One call; ev (list of 7 events or None) brackets the six stages."""
+    p, L = attn.prob, attn.layout_buf
+    if ev:
+        ev[0].record()
+    bsa.layout(p, k, L)
+    if ev:
+        ev[1].record()
+    bsa.permute(p, L, q, attn.qp)
+    bsa.permute(p, L, k, attn.kp)
+    bsa.permute(p, L, v, attn.vp)
+    if ev:
+        ev[2].record()
+    bsa.pool(p, L, attn.qp, attn.kp, attn.q_pool, attn.k_pool)
+    if ev:
+        ev[3].record()
+    bsa.select_topk(p, attn.q_pool, attn.k_pool, attn.idx, attn.cnt)
+    if ev:
+        ev[4].record()
+    bsa.sparse_attn_fwd(p, L, attn.qp, attn.kp, attn.vp, attn.idx, attn.cnt, attn.op, attn.status)
+    if ev:
+        ev[5].record()
+    bsa.unpermute(p, L, attn.op, out)
+    if ev:
+        ev[6].record()
+
+
+def launches_per_step(cfg):
+    return (2 if cfg["block_mode"] == 1 else 1) + 3 + 1 + 1 + 1 + 1
+
+
+def measure(cfg, keep, steps, warmup, world, rank, local, do_e2e, do_dense):
+    import block_sparse_attention_47_b200 as bsa
+    from block_sparse_attention_47_b200 import build
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    prob = bsa.Problem.make(**dict(cfg, keep_blocks=keep))
+    q, k, v = make_qkv(cfg, 42002 + 1000 * rank, pad_fill=0.0, device=dev)
+    attn = bsa.BlockSparseAttention(prob, device=dev)
+    out = torch.empty_like(q)
+    torch.cuda.synchronize()
+
+    flops = kept_tiles(cfg, keep) * tile_flops(cfg)
+    for _ in range(warmup):
+        run_step(bsa, attn, q, k, v, out, None)
+    torch.cuda.synchronize()
+    attn.check_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        run_step(bsa, attn, q, k, v, out, evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    attn.check_status()
+    ms_total = t0.elapsed_time(t1)
+    ms_step = max_over_ranks(ms_total / steps, world)
+    stage_ms = {}
+    for si, name in enumerate(STAGES):
+        stage_ms[name] = statistics.median(e[si].elapsed_time(e[si + 1]) for e in evs)
+    attn_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
+
+    res = dict(ms_step=ms_step, flops=flops, stage_ms=stage_ms, attn_ms=attn_ms, clocks=clocks)
+
+    if do_dense:
+        o = torch.empty_like(attn.op)
+        bsa.dense_attn_fwd(prob, attn.layout_buf, attn.qp, attn.kp, attn.vp, o, attn.status)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(2):
+            bsa.dense_attn_fwd(prob, attn.layout_buf, attn.qp, attn.kp, attn.vp, o, attn.status)
+        b_.record()
+        torch.cuda.synchronize()
+        res["dense_ms"] = a.elapsed_time(b_) / 2
+        res["dense_flops"] = dense_tiles(cfg) * tile_flops(cfg)
+        del o
+
+    if do_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dout = torch.empty_like(q)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            attn(dq, dk, dv, out=dout)
+            hout.copy_(dout, non_blocking=True)
+
+        for _ in range(max(1, min(warmup, 2))):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(2, min(steps, 5))
+        barrier(world)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        b_.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(a.elapsed_time(b_) / n_e2e, world)
+        nbytes = q.numel() * q.element_size()
+        res["e2e"] = dict(ms=e2e_ms, h2d=3 * nbytes, d2h=nbytes)
+        del hq, hk, hv, hout, dq, dk, dv, dout
+    return res
+
+
+# ----------------------------------------------------------------------------
+def oracle_sample(cfg, keep, n_query_blocks, seed, inputs=None):
+    """Run the fp64 oracle on one (batch, head) of the workload for a seeded
+    sample of query blocks; returns (seconds, kept tiles processed)."""
+    from oracle import bsa_oracle as O
+    geo = O.Geometry(cfg)
+    if inputs is None:
+        q, k, v = make_qkv(dict(cfg, B=1, heads=1), seed, pad_fill=0.0)
+        inputs = [t[0, :, 0].float().numpy().astype(np.float64) for t in (q, k, v)]
+    qn, kn, vn = inputs
+    rng = np.random.default_rng(seed)
+    blocks = sorted(set(rng.choice(geo.nb, size=min(n_query_blocks, geo.nb), replace=False).tolist()))
+    t0 = time.perf_counter()
+    if cfg["block_mode"] == 0:
+        perm = O.fixed_perm(geo)
+    else:
+        kk = kn[None, :, None, :] if kn.ndim == 2 else kn
+        v_ = O.region_variation(geo, kk[0])
+        perm = O.dynamic_perm(geo, [O.shape_code(v_[r], cfg["dyn_tau"]) for r in range(len(v_))])
+    qp, kp, vp = (O.permute(geo, perm, x) for x in (qn, kn, vn))
+    lists = O.select(geo, O.pool(geo, perm, qp), O.pool(geo, perm, kp), keep, rows=blocks)
+    O.block_sparse_attention(geo, perm, qp, kp, vp, lists, 1 / math.sqrt(geo.d), blocks)
+    secs = time.perf_counter() - t0
+    return secs, sum(len(lists[i]) for i in blocks), inputs
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, keep, budget_s=15.0):
+    n = 32
+    secs, tiles, inputs = oracle_sample(cfg, keep, n, 4242)
+    # grow the sample to roughly the time budget (one more run)
+    if secs < budget_s / 3:
+        n = int(n * min(budget_s / max(secs, 1e-3), 16))
+        secs, tiles, _ = oracle_sample(cfg, keep, n, 4243, inputs)
+    tflops = tiles * tile_flops(cfg) / secs / 1e12
+    return {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": "fp64 numpy oracle, one (batch, head) of %s: layout, permute, pool, full "
+                      "block scores, top-k and attention for %d seeded query blocks (%d kept "
+                      "tiles) in %.1f s; value = kept-tile FLOPs / wall time"
+                      % (cfg.get("name", "?"), n, tiles, secs)}
+
+
+# ----------------------------------------------------------------------------
+def reference_arm(args, cfg, keep, world, rank):
+    if rank != 0:
+        return
+    n_blocks = 48
+    _, _, inputs = oracle_sample(cfg, keep, 1, 7)
+    for i in range(args.warmup):
+        oracle_sample(cfg, keep, n_blocks, 100 + i, inputs)
+    tiles = 0
+    secs = 0.0
+    for i in range(args.steps):
+        s, t, _ = oracle_sample(cfg, keep, n_blocks, 200 + i, inputs)
+        secs += s
+        tiles += t
+    value = tiles * tile_flops(cfg) / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(cfg, keep, args),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+                             "kind": "oracle",
+                             "sample": "per step: one (batch, head), %d seeded query blocks of "
+                                       "the workload through the fp64 oracle" % n_blocks},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def workload_config(cfg, keep, args):
+    s = derived_sizes(cfg)
+    return {"workload": "%s: B=%d heads=%d d=%d grid %dx%dx%d%s = %d tokens, %d blocks, keep %d "
+                        "(%s blocks)" % (cfg.get("name"), cfg["B"], cfg["heads"], cfg["head_dim"],
+                                         cfg["T"], cfg["H"], cfg["W"],
+                                         " + prefix %s" % (list(cfg["prefix"]),) if cfg["prefix"] else "",
+                                         s["N"], s["nb"], keep,
+                                         "dynamic 8x8x8" if cfg["block_mode"] else "fixed 4x4x4"),
+            "global_batch": cfg["B"] * args.gpus, "seq_len": s["N"], "keep_blocks": keep,
+            "keep_ratio": cfg["keep_ratio"], "parallelism": "independent calls per GPU (dp%d)" % args.gpus,
+            "l2": "inputs larger than L2 (Q, K, V %.2f GB each); no flush" %
+                  (cfg["B"] * s["N"] * cfg["heads"] * cfg["head_dim"] * 2 / 1e9)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--config", default="720p")
+    ap.add_argument("--keep-ratio", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None, help="override heads (profiling runs)")
+    ap.add_argument("--batch", type=int, default=None, help="override B (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="keep-ratio sweep on the 1152x640 grid")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    cfg = config(args.config)
+    if args.keep_ratio is not None:
+        cfg["keep_ratio"] = args.keep_ratio
+    if args.heads is not None:
+        cfg["heads"] = args.heads
+    if args.batch is not None:
+        cfg["B"] = args.batch
+    import block_sparse_attention_47_b200 as bsa
+    from block_sparse_attention_47_b200 import build
+    build.build()
+    keep = bsa.keep_count(derived_sizes(cfg)["nbv"], cfg["keep_ratio"])
+
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            reference_arm(args, cfg, keep, world, rank)
+            return
+        if args.sweep:
+            sweep(args, world, rank, local)
+            return
+        res = measure(cfg, keep, args.steps, args.warmup, world, rank, local,
+                      not args.no_e2e, not args.no_dense and world == 1)
+        if rank != 0:
+            return
+        pk, pk_kind = peaks()
+        value = world * res["flops"] / (res["ms_step"] / 1e3) / 1e12
+        attn_tflops = res["flops"] / (res["attn_ms"] / 1e3) / 1e12
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded smooth field + noise, no weights)",
+            "config": workload_config(cfg, keep, args),
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                         "kernel": "attn_fwd_kernel<128,false> (sparse attention)",
+                         "peak_kind": "%s bf16 sustained" % pk_kind,
+                         "frac_of_burst": attn_tflops / pk["bf16_tflops"]},
+            "stage_ms": res["stage_ms"],
+            "gpu_launches": launches_per_step(cfg) * args.steps,
+        }
+        if "dense_ms" in res:
+            line["dense"] = {"ms": res["dense_ms"],
+                             "tflops": res["dense_flops"] / (res["dense_ms"] / 1e3) / 1e12,
+                             "speedup_sparse_attention_vs_dense": res["dense_ms"] / res["attn_ms"],
+                             "speedup_full_call_vs_dense": res["dense_ms"] / res["ms_step"]}
+        if "e2e" in res:
+            e = res["e2e"]
+            line["e2e"] = {"value": world * res["flops"] / (e["ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+                           "ms_per_step": e["ms"], "h2d_bytes_per_step": e["h2d"],
+                           "d2h_bytes_per_step": e["d2h"]}
+        if res["clocks"]:
+            line["clocks"] = res["clocks"]
+        if world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_baseline(cfg, keep)
+        print(json.dumps(line))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+def sweep(args, world, rank, local):
+    """ms per call and the layout/permute/pool/select overhead as the keep
+    ratio falls, on the 1152x640 grid (plus the 40-layer schedule)."""
+    from gen import layer_keep_schedule
+    base = config("sweep")
+    nbv = derived_sizes(base)["nbv"]
+    rows = []
+    import block_sparse_attention_47_b200 as bsa
+    for r in SWEEP_KEEP_RATIOS:
+        keep = bsa.keep_count(nbv, r)
+        cfg = dict(base, keep_ratio=r)
+        res = measure(cfg, keep, args.steps, args.warmup, world, rank, local, False, False)
+        st = res["stage_ms"]
+        overhead = sum(st[s] for s in ("layout", "permute", "pool", "select", "unpermute"))
+        rows.append({"keep_ratio": r, "keep": keep, "ms_per_call": res["ms_step"],
+                     "attention_ms": st["attention"], "overhead_ms": overhead,
+                     "overhead_share": overhead / res["ms_step"],
+                     "tflops_kept": res["flops"] / (res["ms_step"] / 1e3) / 1e12,
+                     "stage_ms": st})
+    sched = layer_keep_schedule()
+    by_ratio = {row["keep_ratio"]: row["ms_per_call"] for row in rows}
+    if rank == 0:
+        print(json.dumps({"sweep": "1152x640 grid, 92,160 tokens, 24 heads, d=128",
+                          "rows": rows,
+                          "layer_schedule_40": {"keep_ratios": sched,
+                                                "ms_total": sum(by_ratio[r] for r in sched)}}))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,25 +1,36 @@
 // Block-sparse attention forward on sm_100a: TMA-fed tcgen05 tiles with the
-// accumulators in tensor memory, walking a per-query-block list of kept key
-// blocks so that only kept 64x64 tiles are ever loaded or multiplied
-// (Sparse VideoGen on TPU, aibase.it, section "이론적 sparsity와 물리적
-// sparsity의 차이": skipping empty tiles is where the speed comes from).
+// accumulators and the A operands in tensor memory, walking a per-query-block
+// list of kept key blocks so that only kept 64x64 tiles are ever loaded or
+// multiplied (Sparse VideoGen on TPU, aibase.it, section "이론적 sparsity와
+// 물리적 sparsity의 차이": skipping empty tiles is where the speed comes
+// from).
 //
 // CTA = two adjacent query blocks (128 query rows = the full tcgen05 M=128
 // datapath; M=64 would leave half of it idle).  The two blocks' sorted key
 // lists are merged on the fly; each merged step loads one 64-token key
-// block (K and V, 16 KB each at head_dim 128) and computes
-//     S = Q K^T      (M=128, N=64,  K=head_dim)  -> TMEM, double buffered
-//     O += P V       (M=128, N=head_dim, K=64)   -> TMEM accumulator
-// Rows of a block that did not keep the step's key block get P = 0.
+// block (K and V, 16 KB each at head_dim 128) into a shared-memory ring and
+// computes
+//     S = Q K^T   M=128, N=64,       K=head_dim  A = Q in TMEM, B = K in SMEM
+//     O += P V    M=128, N=head_dim, K=64        A = P in TMEM, B = V in SMEM
+// so shared memory only ever feeds the B operands.  Rows of a block that did
+// not keep the step's key block get P = 0.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread r owns query row r = TMEM lane r
-//   warp 4     TMA producer: Q once, then K/V per step into a ring
-//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer
-// Softmax is the exact online softmax in the exp2 domain with a lazily
-// updated running max: the O rescale is only applied when the row max grows
-// by more than 2^8, which keeps every probability below 256 (still exact
-// after the final division by the running sum).
+// Two softmax warpgroups take alternate steps, each with its own running
+// max, running sum and O accumulator (an exact split of the key set); the
+// epilogue merges them: O = (a0*O0 + a1*O1) / (a0*l0 + a1*l1),
+// a_w = 2^(m_w - max(m0, m1)).  The softmax is the exact online softmax in
+// the exp2 domain with a lazily updated running max: O is rescaled only
+// when the row max grows by more than 8 (so every probability stays below
+// 2^8), which is still exact after the final division.
+//
+// Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax warpgroup 0 / 1; thread r of a group owns
+//                    query row r = TMEM lane r (warp w reaches lanes
+//                    32*(w%4)..+31); group 0 first copies Q into TMEM
+//   warp 8           TMA producer of the K/V ring
+//   warp 9           TMEM allocator and single-thread tcgen05.mma issuer
+// Tensor memory (512 columns): Q [0,64) bf16 pairs | S0 [64,128) | S1
+// [128,192) | P0 [192,224) | P1 [224,256) | O0 [256,384) | O1 [384,512).
 //
 // Every wait is bounded (2 s); a timeout sets the caller's status word to
 // BSA_ERR_TIMEOUT, drains in-flight copies and MMAs and frees tensor memory.
@@ -32,23 +43,20 @@ namespace {
 
 template <int D>
 struct Cfg {
-  static constexpr int kThreads = 192;
-  static constexpr int BM = 128, BN = 64;
-  static constexpr int STAGES = (D == 128) ? 4 : 6;
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int Q_BOX = BM * 128;  // bytes of one 64-column Q box
-  static constexpr int KV_BOX = BN * 128;
-  static constexpr uint32_t TMEM_COLS = 256;  // S0 [0,64) S1 [64,128) O [128,128+D)
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int N_BARS = 2 * STAGES + 6;
+  static constexpr int kThreads = 320;
+  static constexpr int STAGES = (D == 128) ? 6 : 8;
+  static constexpr int KV_BYTES = 64 * D * 2;  // one K (or V) block
+  static constexpr int KV_BOX = 64 * 128;      // one 64-column TMA box of a block
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_Q = 0, COL_S = 64, COL_P = 192, COL_O = 256;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = 2 * STAGES * KV_BYTES;
+  // full[S] empty[S] qready s[2] sfree[2] p[2] o[2] drain
+  static constexpr int N_BARS = 2 * STAGES + 10;
   static constexpr int OFF_INFO = OFF_BAR + 8 * N_BARS;
-  static constexpr int OFF_MISC = OFF_INFO + 16 * STAGES;
+  static constexpr int OFF_XCH = OFF_INFO + 16 * STAGES;  // float m[2][128], l[2][128]
+  static constexpr int OFF_MISC = OFF_XCH + 4 * 4 * 128;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
 };
 
@@ -73,27 +81,34 @@ __device__ __forceinline__ void report_timeout(volatile int* abort_flag, int32_t
   atomicCAS(status, 0, int32_t(BSA_ERR_TIMEOUT));
 }
 
+__device__ __forceinline__ bool bit_of(uint32_t lo, uint32_t hi, int c) {
+  return ((c < 32 ? (lo >> c) : (hi >> (c - 32))) & 1u) != 0u;
+}
+
 template <int D, bool DENSE>
-__global__ void __launch_bounds__(192, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                    const __grid_constant__ CUtensorMap mv, Geo g,
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                    Geo g, const __nv_bfloat16* __restrict__ qperm,
                     const uint64_t* __restrict__ bmask, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ out,
                     int32_t* __restrict__ status) {
   using C = Cfg<D>;
+  constexpr int S_ = C::STAGES;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
-  const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V,
-                 sP = base + C::OFF_P, bar0 = base + C::OFF_BAR;
-  // barrier ids
-  const uint32_t bar_q = bar0 + 8 * (2 * C::STAGES);
-  const uint32_t bar_s = bar_q + 8;      // two: S buffer 0 / 1 ready
-  const uint32_t bar_p = bar_q + 24;     // P written + O corrected (128 arrivals)
-  const uint32_t bar_o = bar_q + 32;     // PV finished
-  const uint32_t bar_drain = bar_q + 40; // final MMA drain
+  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, bar0 = base + C::OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * uint32_t(s); };
+  auto empty_bar = [&](int s) { return bar0 + 8u * uint32_t(S_ + s); };
+  const uint32_t bar_qready = bar0 + 8u * (2 * S_);
+  const uint32_t bar_s = bar_qready + 8;       // [2] S of group w ready
+  const uint32_t bar_sfree = bar_qready + 24;  // [2] group w has read its S (128 arrivals)
+  const uint32_t bar_p = bar_qready + 40;      // [2] P written + O corrected (128 arrivals)
+  const uint32_t bar_o = bar_qready + 56;      // [2] PV of group w finished
+  const uint32_t bar_drain = bar_qready + 72;
   StepInfo* info = reinterpret_cast<StepInfo*>(sm + C::OFF_INFO);
+  float* xch = reinterpret_cast<float*>(sm + C::OFF_XCH);  // m[2][128] then l[2][128]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
 
@@ -101,20 +116,22 @@ __global__ void __launch_bounds__(192, 1)
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar0 + 8 * s, 1);
-      mbar_init(bar0 + 8 * (C::STAGES + s), 1);
+    for (int s = 0; s < S_; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
     }
-    mbar_init(bar_q, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_s + 8, 1);
-    mbar_init(bar_p, 128);
-    mbar_init(bar_o, 1);
+    mbar_init(bar_qready, 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bar_s + 8 * w, 1);
+      mbar_init(bar_sfree + 8 * w, 128);
+      mbar_init(bar_p + 8 * w, 128);
+      mbar_init(bar_o + 8 * w, 1);
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -122,17 +139,12 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tS = tmem, tO = tmem + 128;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&mq);
       tma_prefetch_desc(&mk);
       tma_prefetch_desc(&mv);
-      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
-      for (int bx = 0; bx < D / 64; ++bx)
-        tma_load_3d(sQ + bx * C::Q_BOX, &mq, bar_q, bx * 64, pair * 128, bh);
       ListIt it[2];
       for (int hf = 0; hf < 2; ++hf) {
         const int qb = 2 * pair + hf;
@@ -147,21 +159,22 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      int j = 0;
+      int j = 0, ends = 0;
       bool ok = true;
       for (;; ++j) {
-        const int s = j % C::STAGES;
-        if (j >= C::STAGES &&
-            !mbar_wait(bar0 + 8 * (C::STAGES + s), ((j / C::STAGES) - 1) & 1, abort_flag)) {
+        const int s = j % S_;
+        if (j >= S_ && !mbar_wait(empty_bar(s), ((j / S_) - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         const int ta = it[0].peek(), tb = it[1].peek();
         const int t = ta < tb ? ta : tb;
         if (t == INT_MAX) {
+          // two end markers: each softmax group meets one at its next step
           info[s].tile = -1;
-          mbar_arrive(bar0 + 8 * s);
-          break;
+          mbar_arrive(full_bar(s));
+          if (++ends == 2) break;
+          continue;
         }
         uint32_t flags = 0;
         if (ta == t) { flags |= 1u; ++it[0].pos; }
@@ -169,63 +182,73 @@ __global__ void __launch_bounds__(192, 1)
         info[s].tile = t;
         info[s].flags = flags;
         info[s].vmask = __ldg(bmask + int64_t(b) * g.nb + t);
-        const uint32_t full = bar0 + 8 * s;
-        mbar_arrive_expect_tx(full, 2 * C::KV_BYTES);
+        mbar_arrive_expect_tx(full_bar(s), 2 * C::KV_BYTES);
+#pragma unroll
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_3d(sK + s * C::KV_BYTES + bx * C::KV_BOX, &mk, full, bx * 64, t * 64, bh);
-          tma_load_3d(sV + s * C::KV_BYTES + bx * C::KV_BOX, &mv, full, bx * 64, t * 64, bh);
+          tma_load_3d(sK + s * C::KV_BYTES + bx * C::KV_BOX, &mk, full_bar(s), bx * 64, t * 64, bh);
+          tma_load_3d(sV + s * C::KV_BYTES + bx * C::KV_BOX, &mv, full_bar(s), bx * 64, t * 64, bh);
         }
       }
       if (!ok) {
         report_timeout(abort_flag, status);
         // let the copies already in flight land before the CTA goes away
-        for (int jj = j - 1; jj >= 0 && jj >= j - C::STAGES; --jj)
-          mbar_wait(bar0 + 8 * (jj % C::STAGES), (jj / C::STAGES) & 1, nullptr, 200000000ull);
+        for (int jj = j - 1; jj >= 0 && jj >= j - S_; --jj)
+          mbar_wait(full_bar(jj % S_), (jj / S_) & 1, nullptr, 200000000ull);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      bool ok = mbar_wait(bar_q, 0, abort_flag);
-      for (int j = 0; ok; ++j) {
-        const int s = j % C::STAGES;
-        if (!mbar_wait(bar0 + 8 * s, (j / C::STAGES) & 1, abort_flag)) {
-          ok = false;
+      auto issue_qk = [&](int j) {
+        const int s = j % S_;
+        tc_fence_after();
+        const uint32_t d = tmem + C::COL_S + 64u * uint32_t(j & 1);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t bd =
+              sdesc_sw128(sK + s * C::KV_BYTES + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
+          tc_mma_ts(d, tmem + C::COL_Q + 8u * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_s + 8 * (j & 1));
+      };
+      bool ok = mbar_wait(bar_qready, 0, abort_flag);
+      int n = INT_MAX;  // number of steps, known once an end marker is seen
+      for (int j = 0; ok && j < 2; ++j) {
+        ok = mbar_wait(full_bar(j), 0, abort_flag);
+        if (!ok) break;
+        if (*reinterpret_cast<volatile int32_t*>(&info[j].tile) < 0) {
+          n = j;
           break;
         }
-        const int tile = *reinterpret_cast<volatile int32_t*>(&info[s].tile);
-        if (tile >= 0) {
-          tc_fence_after();
-          const uint32_t dS = tS + uint32_t(j & 1) * 64u;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sQ + (kk / 4) * C::Q_BOX + (kk % 4) * 32, 16, 1024);
-            const uint64_t bd =
-                sdesc_sw128(sK + s * C::KV_BYTES + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
-            tc_mma_ss(dS, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar_s + 8 * (j & 1));
+        issue_qk(j);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int w = j & 1, s = j % S_;
+        // the next S of this group can be computed once the group has read S_j
+        const int jn = j + 2;
+        if (jn < n) {
+          ok = mbar_wait(bar_sfree + 8 * w, (j >> 1) & 1, abort_flag);
+          if (ok) ok = mbar_wait(full_bar(jn % S_), (jn / S_) & 1, abort_flag);
+          if (!ok) break;
+          if (*reinterpret_cast<volatile int32_t*>(&info[jn % S_].tile) < 0)
+            n = jn;
+          else
+            issue_qk(jn);
         }
-        if (j > 0) {
-          const int jp = j - 1, sp = jp % C::STAGES;
-          if (!mbar_wait(bar_p, jp & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        ok = mbar_wait(bar_p + 8 * w, (j >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = sdesc_sw128(sP + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sV + sp * C::KV_BYTES + kk * 2048, C::KV_BOX, 1024);
-            tc_mma_ss(tO, a, bd, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(bar_o);
-          tc_commit(bar0 + 8 * (C::STAGES + sp));
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_BOX, 1024);
+          tc_mma_ts(tmem + C::COL_O + 128u * w, tmem + C::COL_P + 32u * w + 8u * kk, bd, idesc_pv,
+                    (j >= 2 || kk > 0) ? 1u : 0u);
         }
-        if (tile < 0) break;
+        tc_commit(bar_o + 8 * w);
+        tc_commit(empty_bar(s));
       }
       if (!ok) report_timeout(abort_flag, status);
       // every MMA this thread issued has completed once bar_drain flips
@@ -235,27 +258,58 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int row = warp * 32 + lane;
-    const int half = warp >> 1;
+    const int wg = warp >> 2, quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int half = quad >> 1;
     const int qb = 2 * pair + half;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const bool q_exists = qb < g.nb;
     const bool row_valid =
         q_exists && ((__ldg(bmask + int64_t(b) * g.nb + qb) >> (row & 63)) & 1ull);
+    bool ok = true;
+
+    if (wg == 0) {
+      // Q rows into tensor memory (A operand of S = Q K^T), bf16 pairs per column
+      uint32_t qr[D / 2];
+      const int64_t qrow = int64_t(pair) * 128 + row;
+      if (qrow < g.N) {
+        const uint4* src = reinterpret_cast<const uint4*>(qperm + (int64_t(bh) * g.N + qrow) * D);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+          const uint4 u = __ldg(src + i);
+          qr[4 * i] = u.x;
+          qr[4 * i + 1] = u.y;
+          qr[4 * i + 2] = u.z;
+          qr[4 * i + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < D / 2; ++i) qr[i] = 0u;
+      }
+      if constexpr (D == 128) {
+        BSA_TMEM_ST64(tmem + C::COL_Q + lane_base, qr);
+      } else {
+        BSA_TMEM_ST32(tmem + C::COL_Q + lane_base, qr);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_qready);
+    }
+
+    const uint32_t tS = tmem + C::COL_S + 64u * wg + lane_base;
+    const uint32_t tP = tmem + C::COL_P + 32u * wg + lane_base;
+    const uint32_t tO = tmem + C::COL_O + 128u * wg + lane_base;
     const float sl2 = g.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l_sum = 0.f;
-    bool ok = true;
-    int j = 0;
-    for (;; ++j) {
-      const int s = j % C::STAGES;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar0 + 8 * s, (j / C::STAGES) & 1, abort_flag));
+    int k = 0;  // steps of this group so far
+    for (int j = wg;; j += 2, ++k) {
+      const int s = j % S_;
+      ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (j / S_) & 1, abort_flag));
       if (!ok) break;
-      const int tile = *reinterpret_cast<volatile int32_t*>(&info[s].tile);
-      if (tile < 0) break;
+      if (*reinterpret_cast<volatile int32_t*>(&info[s].tile) < 0) break;
       const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&info[s].flags);
       const uint64_t vm = *reinterpret_cast<volatile uint64_t*>(&info[s].vmask);
       const bool member = (flags >> half) & 1u;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s + 8 * (j & 1), (j >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s + 8 * wg, k & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t pk[32];
@@ -263,14 +317,21 @@ __global__ void __launch_bounds__(192, 1)
       bool rescale = false;
       if (member) {
         uint32_t r[64];
-        const uint32_t ts = tS + uint32_t(j & 1) * 64u + lane_base;
-        BSA_TMEM_LD32(ts, r);
-        BSA_TMEM_LD32(ts + 32, (r + 32));
-        float mx = -INFINITY;
+        BSA_TMEM_LD64(tS, r);
+        tc_fence_before();
+        mbar_arrive(bar_sfree + 8 * wg);
+        const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
+        const bool all_valid = (lo & hi) == 0xFFFFFFFFu;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (all_valid) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if ((vm >> c) & 1ull) mx = fmaxf(mx, __uint_as_float(r[c]));
-        const float mxs = mx * sl2;
+          for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (bit_of(lo, hi, c)) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
+        }
+        const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
         if (mxs > m_used + 8.f) {
           if (m_used != -INFINITY) {
             factor = ex2_approx(m_used - mxs);
@@ -278,103 +339,128 @@ __global__ void __launch_bounds__(192, 1)
           }
           m_used = mxs;
         }
-        float sum = 0.f;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        if (all_valid) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ((vm >> c) & 1ull) ? ex2_approx(fmaf(__uint_as_float(r[c]), sl2, -m_used)) : 0.f;
-          const float p1 =
-              ((vm >> (c + 1)) & 1ull) ? ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, -m_used)) : 0.f;
-          sum += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, -m_used));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, -m_used));
+            sum[(c >> 1) & 3] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 =
+                bit_of(lo, hi, c) ? ex2_approx(fmaf(__uint_as_float(r[c]), sl2, -m_used)) : 0.f;
+            const float p1 = bit_of(lo, hi, c + 1)
+                                 ? ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, -m_used))
+                                 : 0.f;
+            sum[(c >> 1) & 3] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
         }
-        l_sum = l_sum * factor + sum;
+        l_sum = l_sum * factor + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
       } else {
+        tc_fence_before();
+        mbar_arrive(bar_sfree + 8 * wg);
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      // P buffer and O are free once the previous PV has finished
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, abort_flag));
+      // P and O of this group are free once its previous PV has finished
+      if (k > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o + 8 * wg, (k - 1) & 1, abort_flag));
         if (!ok) break;
       }
+      tc_fence_after();
       if (__any_sync(0xffffffffu, rescale)) {
-        tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t o[32];
-          const uint32_t ta = tO + uint32_t(ch * 32) + lane_base;
-          BSA_TMEM_LD32(ta, o);
+          BSA_TMEM_LD32(tO + 32u * ch, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          BSA_TMEM_ST32(ta, o);
+          BSA_TMEM_ST32(tO + 32u * ch, o);
         }
       }
-      const uint32_t prow = sP + uint32_t(row) * 128u;
-#pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
-        const uint32_t addr = prow + (uint32_t(c16 ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c16]),
-                     "r"(pk[4 * c16 + 1]), "r"(pk[4 * c16 + 2]), "r"(pk[4 * c16 + 3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+      BSA_TMEM_ST32(tP, pk);
       tc_fence_before();
-      mbar_arrive(bar_p);
+      mbar_arrive(bar_p + 8 * wg);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, abort_flag));
+    if (ok && k > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o + 8 * wg, (k - 1) & 1, abort_flag));
+    xch[wg * 128 + row] = m_used;
+    xch[256 + wg * 128 + row] = l_sum;
+    named_bar_sync(1, 256);
+    ok = ok && !*abort_flag;
     if (!ok) {
       if (lane == 0) report_timeout(abort_flag, status);
     } else if (q_exists) {
       tc_fence_after();
-      const float inv = (row_valid && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      const float m0 = xch[row], m1 = xch[128 + row];
+      const float l0 = xch[256 + row], l1 = xch[384 + row];
+      const float m = fmaxf(m0, m1);
+      const float a0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - m);
+      const float a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
+      const float l = l0 * a0 + l1 * a1;
+      const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
+      const float f0 = a0 * inv, f1 = a1 * inv;
       __nv_bfloat16* orow = out + (int64_t(bh) * g.N + int64_t(qb) * 64 + (row & 63)) * D;
+      // group wg writes columns [wg*D/2, (wg+1)*D/2)
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t o[32];
-        BSA_TMEM_LD32(tO + uint32_t(ch * 32) + lane_base, o);
+      for (int ch = 0; ch < D / 64; ++ch) {
+        const uint32_t col = uint32_t(wg * (D / 2) + ch * 32);
+        uint32_t o0[32], o1[32];
+        BSA_TMEM_LD32(tmem + C::COL_O + col + lane_base, o0);
+        BSA_TMEM_LD32(tmem + C::COL_O + 128u + col + lane_base, o1);
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = (a0 != 0.f ? __uint_as_float(o0[2 * i]) * f0 : 0.f) +
+                           (a1 != 0.f ? __uint_as_float(o1[2 * i]) * f1 : 0.f);
+          const float x1 = (a0 != 0.f ? __uint_as_float(o0[2 * i + 1]) * f0 : 0.f) +
+                           (a1 != 0.f ? __uint_as_float(o1[2 * i + 1]) * f1 : 0.f);
+          w[i] = pack_bf16x2(x0, x1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
 template <int D, bool DENSE>
-cudaError_t launch_t(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps, const int32_t* idx,
-                     const int32_t* cnt, __nv_bfloat16* o, int32_t* status, cudaStream_t st) {
+cudaError_t launch_t(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps,
+                     const __nv_bfloat16* qp, const int32_t* idx, const int32_t* cnt,
+                     __nv_bfloat16* o, int32_t* status, cudaStream_t st) {
   using C = Cfg<D>;
   auto kern = attn_fwd_kernel<D, DENSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((g.nb + 1) / 2, g.B * g.h);
-  kern<<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], g, lp.bmask, idx, cnt, o,
-                                           status);
+  kern<<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], g, qp, lp.bmask, idx, cnt, o, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps,
-                             const int32_t* idx, const int32_t* cnt, __nv_bfloat16* o,
-                             int32_t* dev_status, bool dense, cudaStream_t st) {
+                             const __nv_bfloat16* qp, const int32_t* idx, const int32_t* cnt,
+                             __nv_bfloat16* o, int32_t* dev_status, bool dense, cudaStream_t st) {
   if (g.d == 128)
-    return dense ? launch_t<128, true>(g, lp, maps, idx, cnt, o, dev_status, st)
-                 : launch_t<128, false>(g, lp, maps, idx, cnt, o, dev_status, st);
-  return dense ? launch_t<64, true>(g, lp, maps, idx, cnt, o, dev_status, st)
-               : launch_t<64, false>(g, lp, maps, idx, cnt, o, dev_status, st);
+    return dense ? launch_t<128, true>(g, lp, maps, qp, idx, cnt, o, dev_status, st)
+                 : launch_t<128, false>(g, lp, maps, qp, idx, cnt, o, dev_status, st);
+  return dense ? launch_t<64, true>(g, lp, maps, qp, idx, cnt, o, dev_status, st)
+               : launch_t<64, false>(g, lp, maps, qp, idx, cnt, o, dev_status, st);
 }
 
 }  // namespace bsa

@@ -299,17 +299,17 @@ static bsa_status attention_common(const bsa_problem* prob, const void* layout_b
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
     return fail(BSA_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
   BSA_TRY(check_device());
-  CUtensorMap maps[3];
-  BSA_TRY(make_map(&maps[0], g, q_perm, 128));
-  BSA_TRY(make_map(&maps[1], g, k_perm, 64));
-  BSA_TRY(make_map(&maps[2], g, v_perm, 64));
+  CUtensorMap maps[2];
+  BSA_TRY(make_map(&maps[0], g, k_perm, 64));
+  BSA_TRY(make_map(&maps[1], g, v_perm, 64));
   int32_t* status = dev_status;
   if (!status) {
     cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dev_status_sink);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status sink)");
   }
   cudaError_t e = bsa::launch_attention(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
-                                        maps, idx, cnt, static_cast<__nv_bfloat16*>(o_perm),
+                                        maps, static_cast<const __nv_bfloat16*>(q_perm), idx,
+                                        cnt, static_cast<__nv_bfloat16*>(o_perm),
                                         status, dense, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "attention launch");
 }
