@@ -8,12 +8,16 @@
 // CTA = two adjacent query blocks (128 query rows = the full tcgen05 M=128
 // datapath; M=64 would leave half of it idle).  The two blocks' sorted key
 // lists are merged on the fly; each merged step loads one 64-token key
-// block (K and V, 16 KB each at head_dim 128) into a shared-memory ring and
-// computes
-//     S = Q K^T   M=128, N=64,       K=head_dim  A = Q in TMEM, B = K in SMEM
-//     O += P V    M=128, N=head_dim, K=64        A = P in TMEM, B = V in SMEM
-// so shared memory only ever feeds the B operands.  Rows of a block that did
-// not keep the step's key block get P = 0.
+// block (K and V, 16 KB each at head_dim 128) into a shared-memory ring.
+// Steps go in pairs (one per softmax warpgroup) and each pair's scores come
+// from one full-width MMA burst:
+//     [S_j | S_j+1] = Q [K_j ; K_j+1]^T   M=128, N=128, K=head_dim
+//     O_w += P_j V_j                      M=128, N=head_dim, K=64
+// with A = Q or P read from TMEM and B = K or V from shared memory.  (Every
+// MMA burst pays a pipeline-fill latency, so fewer, wider bursts keep the
+// tensor pipe busier; the K ring is laid out box-major so that the K blocks
+// of two consecutive stages are contiguous.)  Rows of a block that did not
+// keep the step's key block get P = 0.
 //
 // Two softmax warpgroups take alternate steps, each with its own running
 // max, running sum and O accumulator (an exact split of the key set); the
@@ -47,6 +51,7 @@ struct Cfg {
   static constexpr int STAGES = (D == 128) ? 6 : 8;
   static constexpr int KV_BYTES = 64 * D * 2;  // one K (or V) block
   static constexpr int KV_BOX = 64 * 128;      // one 64-column TMA box of a block
+  static_assert(STAGES % 2 == 0, "step pairs must not straddle the ring's end");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_Q = 0, COL_S = 64, COL_P = 192, COL_O = 256;
   static constexpr int OFF_K = 0;
@@ -56,7 +61,11 @@ struct Cfg {
   static constexpr int N_BARS = 2 * STAGES + 10;
   static constexpr int OFF_INFO = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_XCH = OFF_INFO + 16 * STAGES;  // float m[2][128], l[2][128]
-  static constexpr int OFF_MISC = OFF_XCH + 4 * 4 * 128;
+  static constexpr int LIST_CAP = 2048;  // index-list entries cached per query block
+  static constexpr int FULL_CAP = 8192;  // blocks whose full/partial byte is cached
+  static constexpr int OFF_LIST = OFF_XCH + 4 * 4 * 128;
+  static constexpr int OFF_FULL = OFF_LIST + 2 * 4 * LIST_CAP;
+  static constexpr int OFF_MISC = OFF_FULL + FULL_CAP;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
 };
 
@@ -66,13 +75,14 @@ struct StepInfo {
   uint64_t vmask;  // valid-slot mask of the key block
 };
 
-// Iterator over the kept key blocks of one query block.
+// Iterator over the kept key blocks of one query block (p points to the
+// shared-memory copy of the list, or to global memory for very long lists).
 struct ListIt {
   const int32_t* p;
   int n, pos, dense_n;
   __device__ int peek() const {
     if (dense_n) return pos < dense_n ? pos : INT_MAX;
-    return pos < n ? __ldg(p + pos) : INT_MAX;
+    return pos < n ? p[pos] : INT_MAX;
   }
 };
 
@@ -89,7 +99,8 @@ template <int D, bool DENSE>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                     Geo g, const __nv_bfloat16* __restrict__ qperm,
-                    const uint64_t* __restrict__ bmask, const int32_t* __restrict__ idx,
+                    const uint64_t* __restrict__ bmask, const uint8_t* __restrict__ bfull,
+                    const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ out,
                     int32_t* __restrict__ status) {
   using C = Cfg<D>;
@@ -102,7 +113,7 @@ __global__ void __launch_bounds__(320, 1)
   auto full_bar = [&](int s) { return bar0 + 8u * uint32_t(s); };
   auto empty_bar = [&](int s) { return bar0 + 8u * uint32_t(S_ + s); };
   const uint32_t bar_qready = bar0 + 8u * (2 * S_);
-  const uint32_t bar_s = bar_qready + 8;       // [2] S of group w ready
+  const uint32_t bar_s = bar_qready + 8;       // S of a step pair ready (slot 2 unused)
   const uint32_t bar_sfree = bar_qready + 24;  // [2] group w has read its S (128 arrivals)
   const uint32_t bar_p = bar_qready + 40;      // [2] P written + O corrected (128 arrivals)
   const uint32_t bar_o = bar_qready + 56;      // [2] PV of group w finished
@@ -121,8 +132,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(bar_qready, 128);
+    mbar_init(bar_s, 1);
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bar_s + 8 * w, 1);
       mbar_init(bar_sfree + 8 * w, 128);
       mbar_init(bar_p + 8 * w, 128);
       mbar_init(bar_o + 8 * w, 1);
@@ -142,23 +153,39 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&mk);
-      tma_prefetch_desc(&mv);
-      ListIt it[2];
-      for (int hf = 0; hf < 2; ++hf) {
-        const int qb = 2 * pair + hf;
-        it[hf] = {nullptr, 0, 0, 0};
-        if (qb < g.nb) {
-          const int c = DENSE ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
-          if (c < 0)
-            it[hf].dense_n = g.nb;
-          else {
-            it[hf].p = idx + (int64_t(bh) * g.nb + qb) * g.kcap;
-            it[hf].n = c;
+    // The whole warp stages both index lists and the per-block "all slots
+    // valid" bytes in shared memory; lane 0 then merges the lists and
+    // issues the K/V copies without a dependent global load per step.
+    int32_t* slist = reinterpret_cast<int32_t*>(sm + C::OFF_LIST);
+    uint8_t* sfull = sm + C::OFF_FULL;
+    const bool full_cached = g.nb <= C::FULL_CAP;
+    const uint8_t* gfull = bfull + int64_t(b) * g.nb;
+    if (full_cached)
+      for (int i = lane; i < g.nb; i += 32) sfull[i] = __ldg(gfull + i);
+    ListIt it[2];
+    for (int hf = 0; hf < 2; ++hf) {
+      const int qb = 2 * pair + hf;
+      it[hf] = {nullptr, 0, 0, 0};
+      if (qb < g.nb) {
+        const int c = DENSE ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
+        if (c < 0) {
+          it[hf].dense_n = g.nb;
+        } else {
+          const int32_t* src = idx + (int64_t(bh) * g.nb + qb) * g.kcap;
+          it[hf].n = c;
+          if (c <= C::LIST_CAP) {
+            for (int i = lane; i < c; i += 32) slist[hf * C::LIST_CAP + i] = __ldg(src + i);
+            it[hf].p = slist + hf * C::LIST_CAP;
+          } else {
+            it[hf].p = src;
           }
         }
       }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      tma_prefetch_desc(&mk);
+      tma_prefetch_desc(&mv);
       int j = 0, ends = 0;
       bool ok = true;
       for (;; ++j) {
@@ -179,13 +206,14 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t flags = 0;
         if (ta == t) { flags |= 1u; ++it[0].pos; }
         if (tb == t) { flags |= 2u; ++it[1].pos; }
+        const bool whole = full_cached ? (sfull[t] != 0) : (__ldg(gfull + t) != 0);
         info[s].tile = t;
         info[s].flags = flags;
-        info[s].vmask = __ldg(bmask + int64_t(b) * g.nb + t);
+        info[s].vmask = whole ? ~0ull : __ldg(bmask + int64_t(b) * g.nb + t);
         mbar_arrive_expect_tx(full_bar(s), 2 * C::KV_BYTES);
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_3d(sK + s * C::KV_BYTES + bx * C::KV_BOX, &mk, full_bar(s), bx * 64, t * 64, bh);
+          tma_load_3d(sK + (bx * S_ + s) * C::KV_BOX, &mk, full_bar(s), bx * 64, t * 64, bh);
           tma_load_3d(sV + s * C::KV_BYTES + bx * C::KV_BOX, &mv, full_bar(s), bx * 64, t * 64, bh);
         }
       }
@@ -200,46 +228,21 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      auto issue_qk = [&](int j) {
-        const int s = j % S_;
+      // scores of steps 2t and 2t+1 into S0 | S1 (adjacent TMEM columns)
+      auto issue_qk_pair = [&](int t) {
+        const int s0 = (2 * t) % S_;
         tc_fence_after();
-        const uint32_t d = tmem + C::COL_S + 64u * uint32_t(j & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t bd =
-              sdesc_sw128(sK + s * C::KV_BYTES + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
-          tc_mma_ts(d, tmem + C::COL_Q + 8u * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t bd = sdesc_sw128(sK + ((kk / 4) * S_ + s0) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
+          tc_mma_ts(tmem + C::COL_S, tmem + C::COL_Q + 8u * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar_s + 8 * (j & 1));
+        tc_commit(bar_s);
       };
-      bool ok = mbar_wait(bar_qready, 0, abort_flag);
-      int n = INT_MAX;  // number of steps, known once an end marker is seen
-      for (int j = 0; ok && j < 2; ++j) {
-        ok = mbar_wait(full_bar(j), 0, abort_flag);
-        if (!ok) break;
-        if (*reinterpret_cast<volatile int32_t*>(&info[j].tile) < 0) {
-          n = j;
-          break;
-        }
-        issue_qk(j);
-      }
-      for (int j = 0; ok && j < n; ++j) {
+      auto issue_pv = [&](int j) {
         const int w = j & 1, s = j % S_;
-        // the next S of this group can be computed once the group has read S_j
-        const int jn = j + 2;
-        if (jn < n) {
-          ok = mbar_wait(bar_sfree + 8 * w, (j >> 1) & 1, abort_flag);
-          if (ok) ok = mbar_wait(full_bar(jn % S_), (jn / S_) & 1, abort_flag);
-          if (!ok) break;
-          if (*reinterpret_cast<volatile int32_t*>(&info[jn % S_].tile) < 0)
-            n = jn;
-          else
-            issue_qk(jn);
-        }
-        ok = mbar_wait(bar_p + 8 * w, (j >> 1) & 1, abort_flag);
-        if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -249,6 +252,45 @@ __global__ void __launch_bounds__(320, 1)
         }
         tc_commit(bar_o + 8 * w);
         tc_commit(empty_bar(s));
+      };
+      // Two independent queues, served in whichever order they become
+      // ready: the score burst of pair tq (needs K of both steps loaded and
+      // both groups done reading the previous pair's S) and PV_jp (needs
+      // P_jp).  No step waits behind the other group's work.
+      bool ok = mbar_wait(bar_qready, 0, abort_flag);
+      int n = INT_MAX;  // number of steps, known once an end marker is seen
+      int tq = 0, jp = 0;
+      uint64_t idle_since = 0;
+      uint32_t idle = 0;
+      while (ok && jp < n) {
+        bool progress = false;
+        const int j0 = 2 * tq;
+        if (j0 < n) {
+          const int s0 = j0 % S_;
+          if ((tq == 0 || (mbar_test(bar_sfree, (tq - 1) & 1) &&
+                           mbar_test(bar_sfree + 8, (tq - 1) & 1))) &&
+              mbar_test(full_bar(s0), (j0 / S_) & 1) &&
+              mbar_test(full_bar(s0 + 1), ((j0 + 1) / S_) & 1)) {
+            if (*reinterpret_cast<volatile int32_t*>(&info[s0].tile) < 0) {
+              n = j0;
+            } else {
+              if (*reinterpret_cast<volatile int32_t*>(&info[s0 + 1].tile) < 0) n = j0 + 1;
+              issue_qk_pair(tq++);
+            }
+            progress = true;
+          }
+        }
+        if (jp < 2 * tq && jp < n && mbar_test(bar_p + 8 * (jp & 1), (jp >> 1) & 1)) {
+          issue_pv(jp++);
+          progress = true;
+        }
+        if (progress) {
+          idle = 0;
+        } else if ((++idle & 255) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (idle == 256) idle_since = now;
+          if (*abort_flag || now - idle_since > 2000000000ull) ok = false;
+        }
       }
       if (!ok) report_timeout(abort_flag, status);
       // every MMA this thread issued has completed once bar_drain flips
@@ -309,7 +351,7 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&info[s].flags);
       const uint64_t vm = *reinterpret_cast<volatile uint64_t*>(&info[s].vmask);
       const bool member = (flags >> half) & 1u;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s + 8 * wg, k & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s, k & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t pk[32];
@@ -447,7 +489,8 @@ cudaError_t launch_t(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps,
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((g.nb + 1) / 2, g.B * g.h);
-  kern<<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], g, qp, lp.bmask, idx, cnt, o, status);
+  kern<<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], g, qp, lp.bmask, lp.bfull, idx, cnt, o,
+                                           status);
   return cudaGetLastError();
 }
 

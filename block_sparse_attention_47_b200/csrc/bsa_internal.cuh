@@ -31,7 +31,7 @@ struct Geo {
 
 // Byte offsets of the sections of the layout buffer (each 256-B aligned).
 struct LayoutMap {
-  size_t perm, iperm, bmask, bcount, codes, total;
+  size_t perm, iperm, bmask, bcount, codes, bfull, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -44,6 +44,7 @@ __host__ __device__ inline LayoutMap layout_map(const Geo& g) {
   m.bmask = off;  off = align256(off + sizeof(uint64_t) * size_t(g.B) * g.nb);
   m.bcount = off; off = align256(off + sizeof(int32_t) * size_t(g.B) * g.nb);
   m.codes = off;  off = align256(off + size_t(g.B) * (g.nreg > 0 ? g.nreg : 1));
+  m.bfull = off;  off = align256(off + size_t(g.B) * g.nb);
   m.total = off;
   return m;
 }
@@ -54,6 +55,7 @@ struct LayoutPtrs {
   uint64_t* bmask;   // [B, nb] bit s: slot s of the block is a real token
   int32_t* bcount;   // [B, nb] number of real tokens in the block
   uint8_t* codes;    // [B, nreg] shape code per region
+  uint8_t* bfull;    // [B, nb] 1 when all 64 slots of the block are real tokens
 };
 
 inline LayoutPtrs layout_ptrs(const Geo& g, void* buf) {
@@ -61,7 +63,7 @@ inline LayoutPtrs layout_ptrs(const Geo& g, void* buf) {
   char* p = static_cast<char*>(buf);
   return {reinterpret_cast<int32_t*>(p + m.perm), reinterpret_cast<int32_t*>(p + m.iperm),
           reinterpret_cast<uint64_t*>(p + m.bmask), reinterpret_cast<int32_t*>(p + m.bcount),
-          reinterpret_cast<uint8_t*>(p + m.codes)};
+          reinterpret_cast<uint8_t*>(p + m.codes), reinterpret_cast<uint8_t*>(p + m.bfull)};
 }
 
 // shape code -> (t, h, w) sides; code 0 is the 4x4x4 cube, codes 1..6 are
@@ -122,6 +124,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
+}
+// non-blocking probe of an mbarrier phase
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;

@@ -142,7 +142,8 @@ __global__ void __launch_bounds__(64) build_maps_kernel(Geo g, const uint8_t* __
                                                         int32_t* __restrict__ perm,
                                                         int32_t* __restrict__ iperm,
                                                         uint64_t* __restrict__ bmask,
-                                                        int32_t* __restrict__ bcount) {
+                                                        int32_t* __restrict__ bcount,
+                                                        uint8_t* __restrict__ bfull) {
   const int j = blockIdx.x, b = blockIdx.y, s = threadIdx.x;
   const int slot = j * kBlock + s;
   int raster;
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(64) build_maps_kernel(Geo g, const uint8_t* __
     const uint64_t m = uint64_t(s_bal[0]) | (uint64_t(s_bal[1]) << 32);
     bmask[int64_t(b) * g.nb + j] = m;
     bcount[int64_t(b) * g.nb + j] = __popcll(m);
+    bfull[int64_t(b) * g.nb + j] = (m == ~0ull) ? 1 : 0;
   }
 }
 
@@ -203,7 +205,7 @@ cudaError_t launch_layout(const Geo& g, const __nv_bfloat16* k, int64_t sb, int6
     if (e != cudaSuccess) return e;
   }
   build_maps_kernel<<<dim3(g.nb, g.B), 64, 0, st>>>(g, lp.codes, lp.perm, lp.iperm, lp.bmask,
-                                                    lp.bcount);
+                                                    lp.bcount, lp.bfull);
   return cudaGetLastError();
 }
 
