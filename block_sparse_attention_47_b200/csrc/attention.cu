@@ -7,17 +7,21 @@
 //
 // CTA = two adjacent query blocks (128 query rows = the full tcgen05 M=128
 // datapath; M=64 would leave half of it idle).  The two blocks' sorted key
-// lists are merged on the fly; each merged step loads one 64-token key
-// block (K and V, 16 KB each at head_dim 128) into a shared-memory ring.
-// Steps go in pairs (one per softmax warpgroup) and each pair's scores come
-// from one full-width MMA burst:
+// lists are merged on the fly into a sequence of steps, one 64-token key
+// block each.  Steps go in pairs (one per softmax warpgroup) and each pair's
+// scores come from one full-width MMA burst:
 //     [S_j | S_j+1] = Q [K_j ; K_j+1]^T   M=128, N=128, K=head_dim
 //     O_w += P_j V_j                      M=128, N=head_dim, K=64
-// with A = Q or P read from TMEM and B = K or V from shared memory.  (Every
+// with A = Q or P read from TMEM and B = K or V from shared memory.  Every
 // MMA burst pays a pipeline-fill latency, so fewer, wider bursts keep the
-// tensor pipe busier; the K ring is laid out box-major so that the K blocks
-// of two consecutive stages are contiguous.)  Rows of a block that did not
-// keep the step's key block get P = 0.
+// tensor pipe busier.  Rows of a block that did not keep the step's key
+// block get P = 0.
+//
+// K and V sit in separate shared-memory rings: a K stage is recycled as
+// soon as its score burst has run, a V stage after its PV, so K is fetched
+// several steps ahead of its use and the TMA latency (far L2 partition or
+// HBM) stays hidden.  The K ring is box-major so that the K blocks of two
+// consecutive stages are contiguous (one B operand for the pair burst).
 //
 // Two softmax warpgroups take alternate steps, each with its own running
 // max, running sum and O accumulator (an exact split of the key set); the
@@ -27,12 +31,17 @@
 // when the row max grows by more than 8 (so every probability stays below
 // 2^8), which is still exact after the final division.
 //
-// Warp roles (320 threads):
+// Warp roles (416 threads):
 //   warps 0-3 / 4-7  softmax warpgroup 0 / 1; thread r of a group owns
 //                    query row r = TMEM lane r (warp w reaches lanes
 //                    32*(w%4)..+31); group 0 first copies Q into TMEM
-//   warp 8           TMA producer of the K/V ring
+//   warp 8           stages the index lists, merges them, publishes each
+//                    step and copies box 0 (head_dim 0-63) of its K block
 //   warp 9           TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-12      copy K box 1, V box 0, V box 1 of each step
+// Each copy stream has its own issuing warp because one thread's stream of
+// bulk tensor copies is limited to about 25 bytes per clock on this part;
+// four streams keep up with the tensor pipe.
 // Tensor memory (512 columns): Q [0,64) bf16 pairs | S0 [64,128) | S1
 // [128,192) | P0 [192,224) | P1 [224,256) | O0 [256,384) | O1 [384,512).
 //
@@ -47,42 +56,81 @@ namespace {
 
 template <int D>
 struct Cfg {
-  static constexpr int kThreads = 320;
-  static constexpr int STAGES = (D == 128) ? 6 : 8;
-  static constexpr int KV_BYTES = 64 * D * 2;  // one K (or V) block
-  static constexpr int KV_BOX = 64 * 128;      // one 64-column TMA box of a block
-  static_assert(STAGES % 2 == 0, "step pairs must not straddle the ring's end");
+  static constexpr int kThreads = 416;
+  static constexpr int KB = D / 64;  // 64-column boxes per block (copy streams per ring)
+  static constexpr int KS = 6;                    // K ring stages (even: pairs)
+  static constexpr int VS = 6;                    // V ring stages
+  static constexpr int IR = 16;                   // step-info ring entries
+  static constexpr int BLK_BYTES = 64 * D * 2;    // one K (or V) block
+  static constexpr int BOX = 64 * 128;            // one 64-column TMA box of a block
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_Q = 0, COL_S = 64, COL_P = 192, COL_O = 256;
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = 2 * STAGES * KV_BYTES;
-  // full[S] empty[S] qready s[2] sfree[2] p[2] o[2] drain
-  static constexpr int N_BARS = 2 * STAGES + 10;
+  static constexpr int OFF_V = KS * BLK_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * BLK_BYTES;
+  // kfull[KS] kempty[KS] vfull[VS] vempty[VS] qready s sfree[2] p[2] o[2] drain
+  static constexpr int N_BARS = 2 * KS + 2 * VS + 10;
   static constexpr int OFF_INFO = OFF_BAR + 8 * N_BARS;
-  static constexpr int OFF_XCH = OFF_INFO + 16 * STAGES;  // float m[2][128], l[2][128]
+  static constexpr int OFF_XCH = OFF_INFO + 24 * IR;  // float m[2][128], l[2][128]
   static constexpr int LIST_CAP = 2048;  // index-list entries cached per query block
   static constexpr int FULL_CAP = 8192;  // blocks whose full/partial byte is cached
   static constexpr int OFF_LIST = OFF_XCH + 4 * 4 * 128;
   static constexpr int OFF_FULL = OFF_LIST + 2 * 4 * LIST_CAP;
   static constexpr int OFF_MISC = OFF_FULL + FULL_CAP;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
+  static_assert(KS % 2 == 0, "step pairs must not straddle the K ring's end");
+  // A step's info entry is overwritten only after the score burst of the
+  // step KS later has run, which needs both groups past step j+KS-2.
+  static_assert(IR > KS + 2 && IR <= 32, "step-info ring size");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 struct StepInfo {
+  int32_t tag;     // j+1 once the entry describes step j (0 = none yet)
   int32_t tile;    // key block, or -1 = no more steps
   uint32_t flags;  // bit 0: first query block keeps it; bit 1: second one
+  uint32_t pad;
   uint64_t vmask;  // valid-slot mask of the key block
 };
+static_assert(sizeof(StepInfo) == 24, "StepInfo layout");
 
-// Iterator over the kept key blocks of one query block (p points to the
-// shared-memory copy of the list, or to global memory for very long lists).
+// Iterator over the kept key blocks of one query block, in rotated order:
+// blocks >= `start` ascending, then the blocks below `start` ascending.
+// CTAs working on the same head start at different blocks, so they do not
+// all fetch the same K/V tiles at the same moment (the online softmax does
+// not depend on the order of its steps).  p points to the shared-memory
+// copy of the list, or to global memory for very long lists; a dense row
+// walks every block.  peek() returns the rotated key (block - start) mod nb
+// of the next block, INT_MAX when done.
 struct ListIt {
   const int32_t* p;
-  int n, pos, dense_n;
+  int n;       // list length (every block for a dense row)
+  bool dense;
+  int first;   // position of the first block >= start
+  int taken;   // blocks handed out so far
+  int start, nb;
+  __device__ void init(int start_, int nb_) {
+    start = start_;
+    nb = nb_;
+    taken = 0;
+    if (dense) {
+      first = start;
+      return;
+    }
+    int lo = 0, hi = n;  // lower_bound(p, p+n, start)
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (p[mid] < start) lo = mid + 1; else hi = mid;
+    }
+    first = lo;
+  }
+  __device__ int block_at(int i) const { return dense ? i : p[i]; }
   __device__ int peek() const {
-    if (dense_n) return pos < dense_n ? pos : INT_MAX;
-    return pos < n ? p[pos] : INT_MAX;
+    if (taken >= n) return INT_MAX;
+    int i = first + taken;
+    if (i >= n) i -= n;
+    const int v = block_at(i);
+    return v >= start ? v - start : v + nb - start;
   }
 };
 
@@ -95,29 +143,44 @@ __device__ __forceinline__ bool bit_of(uint32_t lo, uint32_t hi, int c) {
   return ((c < 32 ? (lo >> c) : (hi >> (c - 32))) & 1u) != 0u;
 }
 
+// Idle bookkeeping for the polling loops: expired() turns true once no
+// progress was made for 2 s or another role has aborted.
+struct IdleClock {
+  uint32_t idle = 0;
+  uint64_t since = 0;
+  __device__ void progress() { idle = 0; }
+  __device__ bool expired(volatile int* abort_flag) {
+    if ((++idle & 255) != 0) return false;
+    const uint64_t now = global_timer_ns();
+    if (idle == 256) since = now;
+    return *abort_flag || now - since > 2000000000ull;
+  }
+};
+
 template <int D, bool DENSE>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(416, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                     Geo g, const __nv_bfloat16* __restrict__ qperm,
                     const uint64_t* __restrict__ bmask, const uint8_t* __restrict__ bfull,
-                    const int32_t* __restrict__ idx,
-                    const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ out,
-                    int32_t* __restrict__ status) {
+                    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
+                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ status) {
   using C = Cfg<D>;
-  constexpr int S_ = C::STAGES;
+  constexpr int KS = C::KS, VS = C::VS, IR = C::IR;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
   const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, bar0 = base + C::OFF_BAR;
-  auto full_bar = [&](int s) { return bar0 + 8u * uint32_t(s); };
-  auto empty_bar = [&](int s) { return bar0 + 8u * uint32_t(S_ + s); };
-  const uint32_t bar_qready = bar0 + 8u * (2 * S_);
-  const uint32_t bar_s = bar_qready + 8;       // S of a step pair ready (slot 2 unused)
-  const uint32_t bar_sfree = bar_qready + 24;  // [2] group w has read its S (128 arrivals)
-  const uint32_t bar_p = bar_qready + 40;      // [2] P written + O corrected (128 arrivals)
-  const uint32_t bar_o = bar_qready + 56;      // [2] PV of group w finished
-  const uint32_t bar_drain = bar_qready + 72;
+  auto kfull = [&](int s) { return bar0 + 8u * uint32_t(s); };
+  auto kempty = [&](int s) { return bar0 + 8u * uint32_t(KS + s); };
+  auto vfull = [&](int s) { return bar0 + 8u * uint32_t(2 * KS + s); };
+  auto vempty = [&](int s) { return bar0 + 8u * uint32_t(2 * KS + VS + s); };
+  const uint32_t bar_qready = bar0 + 8u * (2 * KS + 2 * VS);
+  const uint32_t bar_s = bar_qready + 8;       // S of a step pair ready
+  const uint32_t bar_sfree = bar_qready + 16;  // [2] group w has read its S (128 arrivals)
+  const uint32_t bar_p = bar_qready + 32;      // [2] P written + O corrected (128 arrivals)
+  const uint32_t bar_o = bar_qready + 48;      // [2] PV of group w finished
+  const uint32_t bar_drain = bar_qready + 64;
   StepInfo* info = reinterpret_cast<StepInfo*>(sm + C::OFF_INFO);
   float* xch = reinterpret_cast<float*>(sm + C::OFF_XCH);  // m[2][128] then l[2][128]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
@@ -127,9 +190,13 @@ __global__ void __launch_bounds__(320, 1)
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S_; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(kfull(s), C::KB);
+      mbar_init(kempty(s), 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(vfull(s), C::KB);
+      mbar_init(vempty(s), 1);
     }
     mbar_init(bar_qready, 128);
     mbar_init(bar_s, 1);
@@ -142,6 +209,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 8 && lane < IR) info[lane].tag = 0;
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
@@ -152,10 +220,12 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 8) {
-    // ------------------------------------------------------------ producer
+    // ---------------------------------------------- list merge + K box 0
     // The whole warp stages both index lists and the per-block "all slots
-    // valid" bytes in shared memory; lane 0 then merges the lists and
-    // issues the K/V copies without a dependent global load per step.
+    // valid" bytes in shared memory; lane 0 then merges the lists, publishes
+    // step j once K stage j%KS is free (so an info entry is never reused
+    // before every reader is past it) and copies box 0 of K_j.  After the
+    // last step it publishes two end markers (steps n and n+1).
     int32_t* slist = reinterpret_cast<int32_t*>(sm + C::OFF_LIST);
     uint8_t* sfull = sm + C::OFF_FULL;
     const bool full_cached = g.nb <= C::FULL_CAP;
@@ -165,11 +235,14 @@ __global__ void __launch_bounds__(320, 1)
     ListIt it[2];
     for (int hf = 0; hf < 2; ++hf) {
       const int qb = 2 * pair + hf;
-      it[hf] = {nullptr, 0, 0, 0};
+      it[hf].p = nullptr;
+      it[hf].n = 0;
+      it[hf].dense = false;
       if (qb < g.nb) {
         const int c = DENSE ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
         if (c < 0) {
-          it[hf].dense_n = g.nb;
+          it[hf].dense = true;
+          it[hf].n = g.nb;
         } else {
           const int32_t* src = idx + (int64_t(bh) * g.nb + qb) * g.kcap;
           it[hf].n = c;
@@ -186,42 +259,99 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       tma_prefetch_desc(&mk);
       tma_prefetch_desc(&mv);
+      const int start = int((uint32_t(pair) * 61u + uint32_t(bh) * 17u) % uint32_t(g.nb));
+      it[0].init(start, g.nb);
+      it[1].init(start, g.nb);
       int j = 0, ends = 0;
       bool ok = true;
       for (;; ++j) {
-        const int s = j % S_;
-        if (j >= S_ && !mbar_wait(empty_bar(s), ((j / S_) - 1) & 1, abort_flag)) {
+        const int s = j % KS;
+        if (j >= KS && !mbar_wait(kempty(s), ((j / KS) - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        const int ta = it[0].peek(), tb = it[1].peek();
-        const int t = ta < tb ? ta : tb;
-        if (t == INT_MAX) {
-          // two end markers: each softmax group meets one at its next step
-          info[s].tile = -1;
-          mbar_arrive(full_bar(s));
-          if (++ends == 2) break;
-          continue;
+        StepInfo& e = info[j % IR];
+        int t = INT_MAX;
+        if (ends == 0) {
+          const int ra = it[0].peek(), rb = it[1].peek();
+          const int r = ra < rb ? ra : rb;
+          if (r != INT_MAX) {
+            t = r + start < g.nb ? r + start : r + start - g.nb;
+            uint32_t flags = 0;
+            if (ra == r) { flags |= 1u; ++it[0].taken; }
+            if (rb == r) { flags |= 2u; ++it[1].taken; }
+            const bool whole = full_cached ? (sfull[t] != 0) : (__ldg(gfull + t) != 0);
+            e.tile = t;
+            e.flags = flags;
+            e.vmask = whole ? ~0ull : __ldg(bmask + int64_t(b) * g.nb + t);
+          }
         }
-        uint32_t flags = 0;
-        if (ta == t) { flags |= 1u; ++it[0].pos; }
-        if (tb == t) { flags |= 2u; ++it[1].pos; }
-        const bool whole = full_cached ? (sfull[t] != 0) : (__ldg(gfull + t) != 0);
-        info[s].tile = t;
-        info[s].flags = flags;
-        info[s].vmask = whole ? ~0ull : __ldg(bmask + int64_t(b) * g.nb + t);
-        mbar_arrive_expect_tx(full_bar(s), 2 * C::KV_BYTES);
-#pragma unroll
-        for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_3d(sK + (bx * S_ + s) * C::KV_BOX, &mk, full_bar(s), bx * 64, t * 64, bh);
-          tma_load_3d(sV + s * C::KV_BYTES + bx * C::KV_BOX, &mv, full_bar(s), bx * 64, t * 64, bh);
+        if (t == INT_MAX) e.tile = -1;
+        __threadfence_block();
+        *reinterpret_cast<volatile int32_t*>(&e.tag) = j + 1;
+        if (t == INT_MAX) {
+          mbar_arrive(kfull(s));
+          if (++ends == 2) break;
+        } else {
+          mbar_arrive_expect_tx(kfull(s), C::BOX);
+          tma_load_3d(sK + s * C::BOX, &mk, kfull(s), 0, t * 64, bh);
         }
       }
       if (!ok) {
         report_timeout(abort_flag, status);
-        // let the copies already in flight land before the CTA goes away
-        for (int jj = j - 1; jj >= 0 && jj >= j - S_; --jj)
-          mbar_wait(full_bar(jj % S_), (jj / S_) & 1, nullptr, 200000000ull);
+        for (int jj = j - 1; jj >= 0 && jj >= j - KS; --jj)
+          mbar_wait(kfull(jj % KS), (jj / KS) & 1, nullptr, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 10) {
+    // ---------------------------------------------- K box 1, V boxes 0 / 1
+    const bool is_k = warp == 10;
+    const int bx = is_k ? 1 : warp - 11;
+    if (lane == 0 && bx < C::KB) {
+      const int RS = is_k ? KS : VS;
+      int j = 0, ends = 0;
+      bool ok = true;
+      for (;; ++j) {
+        // sleep on the ring first; the step is normally published by then
+        const int s = j % RS;
+        const uint32_t emp = is_k ? kempty(s) : vempty(s);
+        const uint32_t ful = is_k ? kfull(s) : vfull(s);
+        if (j >= RS && !mbar_wait(emp, ((j / RS) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const StepInfo& e = info[j % IR];
+        {
+          bool seen = false;
+          IdleClock clk;
+          for (;;) {
+            seen = *reinterpret_cast<const volatile int32_t*>(&e.tag) == j + 1;
+            if (seen || clk.expired(abort_flag)) break;
+          }
+          if (!seen) {
+            ok = false;
+            break;
+          }
+        }
+        __threadfence_block();
+        const int t = *reinterpret_cast<const volatile int32_t*>(&e.tile);
+        if (t < 0 && !is_k) break;
+        if (t < 0) {
+          mbar_arrive(ful);
+          if (++ends == 2) break;
+          continue;
+        }
+        mbar_arrive_expect_tx(ful, C::BOX);
+        if (is_k)
+          tma_load_3d(sK + (bx * KS + s) * C::BOX, &mk, ful, 64 * bx, t * 64, bh);
+        else
+          tma_load_3d(sV + s * C::BLK_BYTES + bx * C::BOX, &mv, ful, 64 * bx, t * 64, bh);
+      }
+      if (!ok) {
+        report_timeout(abort_flag, status);
+        for (int jj = j - 1; jj >= 0 && jj >= j - RS; --jj)
+          mbar_wait(is_k ? kfull(jj % RS) : vfull(jj % RS), (jj / RS) & 1, nullptr, 200000000ull);
       }
     }
     __syncwarp();
@@ -232,65 +362,71 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       // scores of steps 2t and 2t+1 into S0 | S1 (adjacent TMEM columns)
       auto issue_qk_pair = [&](int t) {
-        const int s0 = (2 * t) % S_;
+        const int s0 = (2 * t) % KS;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(sK + ((kk / 4) * S_ + s0) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd =
+              sdesc_sw128(sK + ((kk / 4) * KS + s0) * C::BOX + (kk % 4) * 32, 16, 1024);
           tc_mma_ts(tmem + C::COL_S, tmem + C::COL_Q + 8u * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar_s);
+        tc_commit(kempty(s0));
+        tc_commit(kempty(s0 + 1));
       };
       auto issue_pv = [&](int j) {
-        const int w = j & 1, s = j % S_;
+        const int w = j & 1, s = j % VS;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_BOX, 1024);
+          const uint64_t bd = sdesc_sw128(sV + s * C::BLK_BYTES + kk * 2048, C::BOX, 1024);
           tc_mma_ts(tmem + C::COL_O + 128u * w, tmem + C::COL_P + 32u * w + 8u * kk, bd, idesc_pv,
                     (j >= 2 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar_o + 8 * w);
-        tc_commit(empty_bar(s));
+        tc_commit(vempty(s));
       };
-      // Two independent queues, served in whichever order they become
-      // ready: the score burst of pair tq (needs K of both steps loaded and
-      // both groups done reading the previous pair's S) and PV_jp (needs
-      // P_jp).  No step waits behind the other group's work.
+      // Three independent queues, served in whichever order they become
+      // ready: the score burst of pair tq (needs K of both steps and both
+      // groups done reading the previous pair's S) and, per softmax group,
+      // its next PV (needs that group's P and the step's V).  No step waits
+      // behind the other group's work.
       bool ok = mbar_wait(bar_qready, 0, abort_flag);
       int n = INT_MAX;  // number of steps, known once an end marker is seen
-      int tq = 0, jp = 0;
-      uint64_t idle_since = 0;
-      uint32_t idle = 0;
-      while (ok && jp < n) {
+      int tq = 0;
+      int jp[2] = {0, 1};  // next PV step of each group
+      IdleClock clk;
+      while (ok && (jp[0] < n || jp[1] < n)) {
         bool progress = false;
         const int j0 = 2 * tq;
         if (j0 < n) {
-          const int s0 = j0 % S_;
+          const int s0 = j0 % KS;
           if ((tq == 0 || (mbar_test(bar_sfree, (tq - 1) & 1) &&
                            mbar_test(bar_sfree + 8, (tq - 1) & 1))) &&
-              mbar_test(full_bar(s0), (j0 / S_) & 1) &&
-              mbar_test(full_bar(s0 + 1), ((j0 + 1) / S_) & 1)) {
-            if (*reinterpret_cast<volatile int32_t*>(&info[s0].tile) < 0) {
+              mbar_test(kfull(s0), (j0 / KS) & 1) && mbar_test(kfull(s0 + 1), ((j0 + 1) / KS) & 1)) {
+            if (*reinterpret_cast<volatile int32_t*>(&info[j0 % IR].tile) < 0) {
               n = j0;
             } else {
-              if (*reinterpret_cast<volatile int32_t*>(&info[s0 + 1].tile) < 0) n = j0 + 1;
+              if (*reinterpret_cast<volatile int32_t*>(&info[(j0 + 1) % IR].tile) < 0) n = j0 + 1;
               issue_qk_pair(tq++);
             }
             progress = true;
           }
         }
-        if (jp < 2 * tq && jp < n && mbar_test(bar_p + 8 * (jp & 1), (jp >> 1) & 1)) {
-          issue_pv(jp++);
-          progress = true;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int j = jp[w];
+          if (j < 2 * tq && j < n && mbar_test(bar_p + 8 * w, (j >> 1) & 1) &&
+              mbar_test(vfull(j % VS), (j / VS) & 1)) {
+            issue_pv(j);
+            jp[w] = j + 2;
+            progress = true;
+          }
         }
-        if (progress) {
-          idle = 0;
-        } else if ((++idle & 255) == 0) {
-          const uint64_t now = global_timer_ns();
-          if (idle == 256) idle_since = now;
-          if (*abort_flag || now - idle_since > 2000000000ull) ok = false;
-        }
+        if (progress)
+          clk.progress();
+        else if (clk.expired(abort_flag))
+          ok = false;
       }
       if (!ok) report_timeout(abort_flag, status);
       // every MMA this thread issued has completed once bar_drain flips
@@ -344,12 +480,22 @@ __global__ void __launch_bounds__(320, 1)
     float m_used = -INFINITY, l_sum = 0.f;
     int k = 0;  // steps of this group so far
     for (int j = wg;; j += 2, ++k) {
-      const int s = j % S_;
-      ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (j / S_) & 1, abort_flag));
-      if (!ok) break;
-      if (*reinterpret_cast<volatile int32_t*>(&info[s].tile) < 0) break;
-      const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&info[s].flags);
-      const uint64_t vm = *reinterpret_cast<volatile uint64_t*>(&info[s].vmask);
+      // the producer publishes step j's info (tag j+1) before its K copy
+      const StepInfo& e = info[j % IR];
+      {
+        bool seen = false;
+        IdleClock clk;
+        for (;;) {
+          seen = *reinterpret_cast<const volatile int32_t*>(&e.tag) == j + 1;
+          if (seen || clk.expired(abort_flag)) break;
+        }
+        ok = __all_sync(0xffffffffu, seen);
+        if (!ok) break;
+      }
+      __threadfence_block();
+      if (*reinterpret_cast<const volatile int32_t*>(&e.tile) < 0) break;
+      const uint32_t flags = *reinterpret_cast<const volatile uint32_t*>(&e.flags);
+      const uint64_t vm = *reinterpret_cast<const volatile uint64_t*>(&e.vmask);
       const bool member = (flags >> half) & 1u;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s, k & 1, abort_flag));
       if (!ok) break;
