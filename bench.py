@@ -41,6 +41,27 @@ import torch  # noqa: E402
 from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) per sparse-attention launch from one ncu capture
+# (profiles/attn_fwd_720p_b1h4.md: 2.239 GB for B=1 x 4 heads, scaled by the
+# number of (batch, head) problems).  Valid only for the kernel source it was
+# measured on and the 720p keep-480 fixed-block workload; null otherwise.
+ATTN_TRAFFIC = {"sha256": "7b03ac153a81a5d4b0e389f4338f6509c38bcf0cc68288524e6d2db4e3dee0e4",
+                "bytes_per_bh": 2.239e9 / 4, "workload": ("720p", 0.25, 0)}
+
+
+def attn_traffic(cfg, keep_ratio):
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_attention_47_b200", "csrc", "attention.cu")
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if digest != ATTN_TRAFFIC["sha256"]:
+        return None
+    if (cfg.get("name"), keep_ratio, cfg["block_mode"]) != ATTN_TRAFFIC["workload"]:
+        return None
+    return ATTN_TRAFFIC["bytes_per_bh"] * cfg["B"] * cfg["heads"]
 METRIC = "ms/call & effective TFLOP/s (kept tiles) at 122,880 tok, s=0.75; % BF16 peak"
 
 
@@ -427,7 +448,8 @@ def main():
             "data": "synthetic (seeded smooth field + noise, no weights)",
             "config": workload_config(cfg, keep, args),
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
-                         "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                         "traffic": attn_traffic(cfg, cfg["keep_ratio"]),
                          "kernel": "attn_fwd_kernel<128,false> (sparse attention)",
                          "peak_kind": "%s bf16 sustained" % pk_kind,
                          "frac_of_burst": attn_tflops / pk["bf16_tflops"]},

@@ -35,9 +35,11 @@ CONFIGS = {
     # 720p 121-frame clip, CFG cond/uncond stacked as B=2
     "720p": dict(_BASE, B=2, T=32, H=48, W=80, T_valid=32, H_valid=48,
                  W_valid=80, keep_ratio=0.25),
-    # same grid with dynamic per-region block shapes and moving objects
+    # same grid with dynamic per-region block shapes and moving objects; the
+    # blob count is calibrated so that about 40 % of the 8x8x8 regions pick a
+    # non-default shape at tau = 1.25 (64 blobs: 38 % for the K of batch 0)
     "720p_dyn": dict(_BASE, B=2, T=32, H=48, W=80, T_valid=32, H_valid=48,
-                     W_valid=80, keep_ratio=0.25, block_mode=1, blobs=4),
+                     W_valid=80, keep_ratio=0.25, block_mode=1, blobs=64),
     # 1344x768 clip behind a 512 text + 2048 image + 256 audio prefix
     "ref_prefix": dict(_BASE, T=32, H=48, W=84, T_valid=32, H_valid=48,
                        W_valid=84, prefix=(512, 2048, 256), keep_ratio=0.25),

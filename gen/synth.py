@@ -9,9 +9,9 @@ Value recipe per tensor (Q, K, V drawn from independent seeded streams):
                  with (kt, ky, kx) in {0,1,2}^3 drawn per (head, channel) and
                  phi ~ U[0, 2*pi) drawn per (batch, head, channel): a smooth
                  low-frequency field, so block means carry structure;
-  moving blobs   (optional) Gaussian blobs of sigma 4 tokens and amplitude 2,
-                 each moving 2 tokens per frame on the (periodic) frame, added
-                 with a random sign per (head, channel);
+  moving blobs   (optional, Q and K only) Gaussian blobs of sigma 4 tokens and
+                 amplitude 2, each moving 2 tokens per frame on the (periodic)
+                 frame, added with a random sign per (head, channel);
   prefix tokens  i.i.d. 0.5*N(0,1);
   pad tokens     a constant fill (1e4 in correctness runs, so that any pad
                  leaking into a result is visible; 0 in timing runs).
@@ -74,7 +74,10 @@ def make_tensor(cfg, seed, tensor_id, pad_fill=1e4, device="cpu"):
                           + yy[:, None, None] * kvec[1] / cfg["H"]
                           + xx[:, None, None] * kvec[2] / cfg["W"])  # [Nv,h,d]
     blob = None
-    if cfg.get("blobs", 0):
+    # moving objects go into Q and K (what block pooling and the dynamic
+    # shape rule look at); V keeps the base recipe so that outputs stay in
+    # the few-unit range where a bf16 result is accurate to ~1e-2 absolute
+    if cfg.get("blobs", 0) and tensor_id in (0, 1):
         gb = _gen(seed, 100 + tensor_id, device)
         field = _blob_field(cfg, cfg["blobs"], gb, device)
         sign = torch.randint(0, 2, (h, d), generator=gb, device=device).float() * 2 - 1
