@@ -31,14 +31,18 @@
 // when the row max grows by more than 8 (so every probability stays below
 // 2^8), which is still exact after the final division.
 //
-// Warp roles (416 threads):
+// Warp roles (448 threads):
 //   warps 0-3 / 4-7  softmax warpgroup 0 / 1; thread r of a group owns
 //                    query row r = TMEM lane r (warp w reaches lanes
 //                    32*(w%4)..+31); group 0 first copies Q into TMEM
 //   warp 8           stages the index lists, merges them, publishes each
 //                    step and copies box 0 (head_dim 0-63) of its K block
-//   warp 9           TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 9           TMEM allocator; one thread issues the score bursts
 //   warps 10-12      copy K box 1, V box 0, V box 1 of each step
+//   warp 13          one thread issues the PV MMAs of both softmax groups
+// tcgen05.mma blocks its issuing thread while the tensor pipe is busy, so
+// score bursts and PVs come from two threads and never queue behind each
+// other.
 // Each copy stream has its own issuing warp because one thread's stream of
 // bulk tensor copies is limited to about 25 bytes per clock on this part;
 // four streams keep up with the tensor pipe.
@@ -56,10 +60,10 @@ namespace {
 
 template <int D>
 struct Cfg {
-  static constexpr int kThreads = 416;
+  static constexpr int kThreads = 448;
   static constexpr int KB = D / 64;  // 64-column boxes per block (copy streams per ring)
-  static constexpr int KS = 6;                    // K ring stages (even: pairs)
-  static constexpr int VS = 6;                    // V ring stages
+  static constexpr int KS = 8;                    // K ring stages (even: pairs)
+  static constexpr int VS = 5;                    // V ring stages
   static constexpr int IR = 16;                   // step-info ring entries
   static constexpr int BLK_BYTES = 64 * D * 2;    // one K (or V) block
   static constexpr int BOX = 64 * 128;            // one 64-column TMA box of a block
@@ -68,12 +72,12 @@ struct Cfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = KS * BLK_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * BLK_BYTES;
-  // kfull[KS] kempty[KS] vfull[VS] vempty[VS] qready s sfree[2] p[2] o[2] drain
-  static constexpr int N_BARS = 2 * KS + 2 * VS + 10;
+  // kfull[KS] kempty[KS] vfull[VS] vempty[VS] qready s sfree[2] p[2] o[2] drain[2]
+  static constexpr int N_BARS = 2 * KS + 2 * VS + 11;
   static constexpr int OFF_INFO = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_XCH = OFF_INFO + 24 * IR;  // float m[2][128], l[2][128]
-  static constexpr int LIST_CAP = 2048;  // index-list entries cached per query block
-  static constexpr int FULL_CAP = 8192;  // blocks whose full/partial byte is cached
+  static constexpr int LIST_CAP = 1024;  // index-list entries cached per query block
+  static constexpr int FULL_CAP = 2560;  // blocks whose full/partial byte is cached
   static constexpr int OFF_LIST = OFF_XCH + 4 * 4 * 128;
   static constexpr int OFF_FULL = OFF_LIST + 2 * 4 * LIST_CAP;
   static constexpr int OFF_MISC = OFF_FULL + FULL_CAP;
@@ -158,7 +162,7 @@ struct IdleClock {
 };
 
 template <int D, bool DENSE>
-__global__ void __launch_bounds__(416, 1)
+__global__ void __launch_bounds__(448, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                     Geo g, const __nv_bfloat16* __restrict__ qperm,
                     const uint64_t* __restrict__ bmask, const uint8_t* __restrict__ bfull,
@@ -180,7 +184,7 @@ __global__ void __launch_bounds__(416, 1)
   const uint32_t bar_sfree = bar_qready + 16;  // [2] group w has read its S (128 arrivals)
   const uint32_t bar_p = bar_qready + 32;      // [2] P written + O corrected (128 arrivals)
   const uint32_t bar_o = bar_qready + 48;      // [2] PV of group w finished
-  const uint32_t bar_drain = bar_qready + 64;
+  const uint32_t bar_drain = bar_qready + 64;  // [2] score issuer, PV issuer
   StepInfo* info = reinterpret_cast<StepInfo*>(sm + C::OFF_INFO);
   float* xch = reinterpret_cast<float*>(sm + C::OFF_XCH);  // m[2][128] then l[2][128]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
@@ -206,6 +210,7 @@ __global__ void __launch_bounds__(416, 1)
       mbar_init(bar_o + 8 * w, 1);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_drain + 8, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(416, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 10) {
+  } else if (warp >= 10 && warp <= 12) {
     // ---------------------------------------------- K box 1, V boxes 0 / 1
     const bool is_k = warp == 10;
     const int bx = is_k ? 1 : warp - 11;
@@ -356,13 +361,21 @@ __global__ void __launch_bounds__(416, 1)
     }
     __syncwarp();
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score bursts
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      // scores of steps 2t and 2t+1 into S0 | S1 (adjacent TMEM columns)
-      auto issue_qk_pair = [&](int t) {
-        const int s0 = (2 * t) % KS;
+      bool ok = mbar_wait(bar_qready, 0, abort_flag);
+      // pair t: scores of steps 2t and 2t+1 into S0 | S1 (adjacent TMEM
+      // columns); needs K of both steps and both groups done reading the
+      // previous pair's S
+      for (int t = 0; ok; ++t) {
+        const int j0 = 2 * t, s0 = j0 % KS;
+        if (t > 0) ok = mbar_wait(bar_sfree, (t - 1) & 1, abort_flag) &&
+                        mbar_wait(bar_sfree + 8, (t - 1) & 1, abort_flag);
+        if (ok) ok = mbar_wait(kfull(s0), (j0 / KS) & 1, abort_flag) &&
+                     mbar_wait(kfull(s0 + 1), ((j0 + 1) / KS) & 1, abort_flag);
+        if (!ok) break;
+        if (*reinterpret_cast<volatile int32_t*>(&info[j0 % IR].tile) < 0) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -373,55 +386,53 @@ __global__ void __launch_bounds__(416, 1)
         tc_commit(bar_s);
         tc_commit(kempty(s0));
         tc_commit(kempty(s0 + 1));
-      };
-      auto issue_pv = [&](int j) {
-        const int w = j & 1, s = j % VS;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(sV + s * C::BLK_BYTES + kk * 2048, C::BOX, 1024);
-          tc_mma_ts(tmem + C::COL_O + 128u * w, tmem + C::COL_P + 32u * w + 8u * kk, bd, idesc_pv,
-                    (j >= 2 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar_o + 8 * w);
-        tc_commit(vempty(s));
-      };
-      // Three independent queues, served in whichever order they become
-      // ready: the score burst of pair tq (needs K of both steps and both
-      // groups done reading the previous pair's S) and, per softmax group,
-      // its next PV (needs that group's P and the step's V).  No step waits
-      // behind the other group's work.
-      bool ok = mbar_wait(bar_qready, 0, abort_flag);
-      int n = INT_MAX;  // number of steps, known once an end marker is seen
-      int tq = 0;
-      int jp[2] = {0, 1};  // next PV step of each group
+        if (*reinterpret_cast<volatile int32_t*>(&info[(j0 + 1) % IR].tile) < 0) break;
+      }
+      if (!ok) report_timeout(abort_flag, status);
+      // every MMA this thread issued has completed once its drain barrier flips
+      tc_commit(bar_drain);
+      mbar_wait(bar_drain, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 13) {
+    // ------------------------------------------------------------ PV issuer
+    // Two independent queues (one per softmax group), served in whichever
+    // order they become ready: PV_j needs P_j and V_j.  A group is done at
+    // its first end marker.
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      int jp[2] = {0, 1};
+      bool done[2] = {false, false};
+      bool ok = true;
       IdleClock clk;
-      while (ok && (jp[0] < n || jp[1] < n)) {
+      while (ok && !(done[0] && done[1])) {
         bool progress = false;
-        const int j0 = 2 * tq;
-        if (j0 < n) {
-          const int s0 = j0 % KS;
-          if ((tq == 0 || (mbar_test(bar_sfree, (tq - 1) & 1) &&
-                           mbar_test(bar_sfree + 8, (tq - 1) & 1))) &&
-              mbar_test(kfull(s0), (j0 / KS) & 1) && mbar_test(kfull(s0 + 1), ((j0 + 1) / KS) & 1)) {
-            if (*reinterpret_cast<volatile int32_t*>(&info[j0 % IR].tile) < 0) {
-              n = j0;
-            } else {
-              if (*reinterpret_cast<volatile int32_t*>(&info[(j0 + 1) % IR].tile) < 0) n = j0 + 1;
-              issue_qk_pair(tq++);
-            }
-            progress = true;
-          }
-        }
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
+          if (done[w]) continue;
           const int j = jp[w];
-          if (j < 2 * tq && j < n && mbar_test(bar_p + 8 * w, (j >> 1) & 1) &&
-              mbar_test(vfull(j % VS), (j / VS) & 1)) {
-            issue_pv(j);
-            jp[w] = j + 2;
+          const StepInfo& e = info[j % IR];
+          if (*reinterpret_cast<const volatile int32_t*>(&e.tag) != j + 1) continue;
+          __threadfence_block();
+          if (*reinterpret_cast<const volatile int32_t*>(&e.tile) < 0) {
+            done[w] = true;
             progress = true;
+            continue;
           }
+          const int s = j % VS;
+          if (!mbar_test(bar_p + 8 * w, (j >> 1) & 1) || !mbar_test(vfull(s), (j / VS) & 1))
+            continue;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_sw128(sV + s * C::BLK_BYTES + kk * 2048, C::BOX, 1024);
+            tc_mma_ts(tmem + C::COL_O + 128u * w, tmem + C::COL_P + 32u * w + 8u * kk, bd,
+                      idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar_o + 8 * w);
+          tc_commit(vempty(s));
+          jp[w] = j + 2;
+          progress = true;
         }
         if (progress)
           clk.progress();
@@ -429,9 +440,8 @@ __global__ void __launch_bounds__(416, 1)
           ok = false;
       }
       if (!ok) report_timeout(abort_flag, status);
-      // every MMA this thread issued has completed once bar_drain flips
-      tc_commit(bar_drain);
-      mbar_wait(bar_drain, 0, nullptr, 200000000ull);
+      tc_commit(bar_drain + 8);
+      mbar_wait(bar_drain + 8, 0, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
