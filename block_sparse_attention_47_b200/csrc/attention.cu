@@ -31,21 +31,21 @@
 // when the row max grows by more than 8 (so every probability stays below
 // 2^8), which is still exact after the final division.
 //
-// Warp roles (448 threads):
+// Warp roles (512 threads):
 //   warps 0-3 / 4-7  softmax warpgroup 0 / 1; thread r of a group owns
 //                    query row r = TMEM lane r (warp w reaches lanes
 //                    32*(w%4)..+31); group 0 first copies Q into TMEM
 //   warp 8           stages the index lists, merges them, publishes each
-//                    step and copies box 0 (head_dim 0-63) of its K block
+//                    step, and copies box 0 (head_dim 0-63) of even steps' K
 //   warp 9           TMEM allocator; one thread issues the score bursts
-//   warps 10-12      copy K box 1, V box 0, V box 1 of each step
+//   warp 10          K box 0 of odd steps
+//   warps 11 / 12    K box 1 (head_dim 64-127) of even / odd steps
 //   warp 13          one thread issues the PV MMAs of both softmax groups
-// tcgen05.mma blocks its issuing thread while the tensor pipe is busy, so
-// score bursts and PVs come from two threads and never queue behind each
-// other.
-// Each copy stream has its own issuing warp because one thread's stream of
-// bulk tensor copies is limited to about 25 bytes per clock on this part;
-// four streams keep up with the tensor pipe.
+//   warps 14 / 15    V of even / odd steps (both halves in one copy)
+// One issuing thread completes about one bulk tensor copy per ~650 cycles
+// whatever its size, so copies are spread over six warps and V moves as a
+// single 16 KB copy; tcgen05.mma blocks its issuing thread while the tensor
+// pipe is busy, so score bursts and PVs come from two threads.
 // Tensor memory (512 columns): Q [0,64) bf16 pairs | S0 [64,128) | S1
 // [128,192) | P0 [192,224) | P1 [224,256) | O0 [256,384) | O1 [384,512).
 //
@@ -60,7 +60,7 @@ namespace {
 
 template <int D>
 struct Cfg {
-  static constexpr int kThreads = 448;
+  static constexpr int kThreads = 512;
   static constexpr int KB = D / 64;  // 64-column boxes per block (copy streams per ring)
   static constexpr int KS = 8;                    // K ring stages (even: pairs)
   static constexpr int VS = 5;                    // V ring stages
@@ -162,7 +162,7 @@ struct IdleClock {
 };
 
 template <int D, bool DENSE>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(512, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                     Geo g, const __nv_bfloat16* __restrict__ qperm,
                     const uint64_t* __restrict__ bmask, const uint8_t* __restrict__ bfull,
@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(448, 1)
   auto kempty = [&](int s) { return bar0 + 8u * uint32_t(KS + s); };
   auto vfull = [&](int s) { return bar0 + 8u * uint32_t(2 * KS + s); };
   auto vempty = [&](int s) { return bar0 + 8u * uint32_t(2 * KS + VS + s); };
+  auto ful_of = [&](bool k, int s) { return k ? kfull(s) : vfull(s); };
   const uint32_t bar_qready = bar0 + 8u * (2 * KS + 2 * VS);
   const uint32_t bar_s = bar_qready + 8;       // S of a step pair ready
   const uint32_t bar_sfree = bar_qready + 16;  // [2] group w has read its S (128 arrivals)
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(448, 1)
       mbar_init(kempty(s), 1);
     }
     for (int s = 0; s < VS; ++s) {
-      mbar_init(vfull(s), C::KB);
+      mbar_init(vfull(s), 1);
       mbar_init(vempty(s), 1);
     }
     mbar_init(bar_qready, 128);
@@ -294,13 +295,15 @@ __global__ void __launch_bounds__(448, 1)
         if (t == INT_MAX) e.tile = -1;
         __threadfence_block();
         *reinterpret_cast<volatile int32_t*>(&e.tag) = j + 1;
-        if (t == INT_MAX) {
-          mbar_arrive(kfull(s));
-          if (++ends == 2) break;
-        } else {
-          mbar_arrive_expect_tx(kfull(s), C::BOX);
-          tma_load_3d(sK + s * C::BOX, &mk, kfull(s), 0, t * 64, bh);
+        if ((j & 1) == 0) {  // K box 0 of even steps
+          if (t == INT_MAX) {
+            mbar_arrive(kfull(s));
+          } else {
+            mbar_arrive_expect_tx(kfull(s), C::BOX);
+            tma_load_3d(sK + s * C::BOX, &mk, kfull(s), 0, t * 64, bh);
+          }
         }
+        if (t == INT_MAX && ++ends == 2) break;
       }
       if (!ok) {
         report_timeout(abort_flag, status);
@@ -309,15 +312,16 @@ __global__ void __launch_bounds__(448, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 10 && warp <= 12) {
-    // ---------------------------------------------- K box 1, V boxes 0 / 1
-    const bool is_k = warp == 10;
-    const int bx = is_k ? 1 : warp - 11;
-    if (lane == 0 && bx < C::KB) {
+  } else if (warp == 10 || warp == 11 || warp == 12 || warp == 14 || warp == 15) {
+    // ---------------------------------------------- K box 0 odd, K box 1, V
+    const bool is_k = warp <= 12;
+    const int bx = warp == 10 ? 0 : 1;        // K box (unused for V)
+    const int par = (warp == 11 || warp == 14) ? 0 : 1;
+    if (lane == 0 && (!is_k || bx < C::KB)) {
       const int RS = is_k ? KS : VS;
-      int j = 0, ends = 0;
+      int j = par;
       bool ok = true;
-      for (;; ++j) {
+      for (;; j += 2) {
         // sleep on the ring first; the step is normally published by then
         const int s = j % RS;
         const uint32_t emp = is_k ? kempty(s) : vempty(s);
@@ -341,22 +345,25 @@ __global__ void __launch_bounds__(448, 1)
         }
         __threadfence_block();
         const int t = *reinterpret_cast<const volatile int32_t*>(&e.tile);
-        if (t < 0 && !is_k) break;
-        if (t < 0) {
-          mbar_arrive(ful);
-          if (++ends == 2) break;
-          continue;
+        if (t < 0) {  // each parity meets exactly one of the two end markers
+          if (is_k) mbar_arrive(ful);
+          break;
         }
-        mbar_arrive_expect_tx(ful, C::BOX);
-        if (is_k)
+        if (is_k) {
+          mbar_arrive_expect_tx(ful, C::BOX);
           tma_load_3d(sK + (bx * KS + s) * C::BOX, &mk, ful, 64 * bx, t * 64, bh);
-        else
-          tma_load_3d(sV + s * C::BLK_BYTES + bx * C::BOX, &mv, ful, 64 * bx, t * 64, bh);
+        } else {
+          mbar_arrive_expect_tx(ful, C::BLK_BYTES);
+          if constexpr (D == 128)
+            tma_load_4d(sV + s * C::BLK_BYTES, &mv, ful, 0, t * 64, 0, bh);
+          else
+            tma_load_3d(sV + s * C::BLK_BYTES, &mv, ful, 0, t * 64, bh);
+        }
       }
       if (!ok) {
         report_timeout(abort_flag, status);
-        for (int jj = j - 1; jj >= 0 && jj >= j - RS; --jj)
-          mbar_wait(is_k ? kfull(jj % RS) : vfull(jj % RS), (jj / RS) & 1, nullptr, 200000000ull);
+        for (int jj = j - 2; jj >= 0 && jj >= j - 2 * RS; jj -= 2)
+          mbar_wait(ful_of(is_k, jj % RS), (jj / RS) & 1, nullptr, 200000000ull);
       }
     }
     __syncwarp();
