@@ -154,6 +154,9 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------
 def dist_setup(want_gpus):
+    """Rank, world size and local rank from the torchrun environment; for
+    N > 1 one process group over NCCL (gloo on a host without CUDA, where
+    only the host-side plumbing and the oracle arm can run)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -161,9 +164,13 @@ def dist_setup(want_gpus):
         raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (want_gpus, world))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout,
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=timeout)
     return world, rank, local
 
 
@@ -173,11 +180,24 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest x over all ranks (every rank gets it)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank):
+    """Each rank draws its own inputs: independent calls, nothing shared."""
+    return 42002 + 1000 * rank
+
+
+def whole_job_tflops(world, flops_per_rank, ms_slowest):
+    """Weak scaling: every rank does the same work; the job's throughput is
+    all ranks' FLOPs over the slowest rank's time."""
+    return world * flops_per_rank / (ms_slowest / 1e3) / 1e12
 
 
 # ----------------------------------------------------------------------------
@@ -222,7 +242,7 @@ def measure(cfg, keep, steps, warmup, world, rank, local, do_e2e, do_dense):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     prob = bsa.Problem.make(**dict(cfg, keep_blocks=keep))
-    q, k, v = make_qkv(cfg, 42002 + 1000 * rank, pad_fill=0.0, device=dev)
+    q, k, v = make_qkv(cfg, rank_seed(rank), pad_fill=0.0, device=dev)
     attn = bsa.BlockSparseAttention(prob, device=dev)
     out = torch.empty_like(q)
     torch.cuda.synchronize()
@@ -438,7 +458,7 @@ def main():
         if rank != 0:
             return
         pk, pk_kind = peaks()
-        value = world * res["flops"] / (res["ms_step"] / 1e3) / 1e12
+        value = whole_job_tflops(world, res["flops"], res["ms_step"])
         attn_tflops = res["flops"] / (res["attn_ms"] / 1e3) / 1e12
         peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
         line = {
@@ -463,7 +483,7 @@ def main():
                              "speedup_full_call_vs_dense": res["dense_ms"] / res["ms_step"]}
         if "e2e" in res:
             e = res["e2e"]
-            line["e2e"] = {"value": world * res["flops"] / (e["ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+            line["e2e"] = {"value": whole_job_tflops(world, res["flops"], e["ms"]), "unit": "TFLOP/s",
                            "ms_per_step": e["ms"], "h2d_bytes_per_step": e["h2d"],
                            "d2h_bytes_per_step": e["d2h"]}
         if res["clocks"]:

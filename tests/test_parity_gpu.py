@@ -217,3 +217,44 @@ def test_dense_kernel_matches_oracle_and_full_keep(case):
 
 def test_status_word_untouched(case):
     assert int(case["run"].attn.status.item()) == 0
+
+
+def growing_logit_inputs(cfg, seed):
+    """Generator inputs with K scaled up frame by frame (and Q doubled), so
+    that along a CTA's walk the running row max jumps by far more than 2^8:
+    exercises the online-softmax rescale of the O accumulator."""
+    q, k, v = seeded_inputs(cfg, seed)[0]
+    geo = O.Geometry(cfg)
+    t = torch.arange(cfg["T"], device=k.device, dtype=torch.float32)
+    scale = (1.0 + 0.6 * t).repeat_interleave(cfg["H"] * cfg["W"])
+    kk = k.float()
+    kk[:, geo.P:] *= scale[None, :, None, None]
+    valid = torch.from_numpy(geo.token_valid()).to(k.device)
+    kk[:, ~valid] = 1e4
+    qq = q.float() * 2.0
+    qq[:, ~valid] = 1e4
+    return qq.to(torch.bfloat16), kk.to(torch.bfloat16), v
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_rescale_path_growing_logits(name):
+    cfg = SMALL[name]
+    q, k, v = growing_logit_inputs(cfg, 99)
+    host = [to_np64(t) for t in (q, k, v)]
+    run = GpuRun(cfg, q, k, v)
+    want, _, _, lists = O.forward(cfg, *host)
+    geo = O.Geometry(cfg)
+    idx, cnt = run.attn.idx.cpu().numpy(), run.attn.cnt.cpu().numpy()
+    lay = O.layout(cfg, host[1])
+    keep_rows = np.ones((geo.B, geo.h, geo.N), dtype=bool)
+    for b in range(geo.B):
+        perm = lay[b][0]
+        for hh in range(geo.h):
+            for i in range(geo.nbp, geo.nb):
+                if list(idx[b, hh, i, :cnt[b, hh, i]]) != list(lists[b][hh][i]):
+                    keep_rows[b, hh, perm[i * 64:(i + 1) * 64]] = False
+    assert keep_rows.mean() > 0.9
+    got = to_np64(run.out)
+    assert_close(got.transpose(0, 2, 1, 3)[keep_rows], want.transpose(0, 2, 1, 3)[keep_rows],
+                 name + " growing logits")
+    assert int(run.attn.status.item()) == 0
