@@ -31,12 +31,18 @@
 // when the row max grows by more than 8 (so every probability stays below
 // 2^8), which is still exact after the final division.
 //
+// The step sequence is fixed before the walk starts: warp 8 turns the two
+// index lists into two bitmaps over the key blocks (one bit per kept block),
+// and every role walks the union A|B with a private cursor, so no role waits
+// for another to hand it the next key block.  The walk visits 32-block words
+// in a rotated order and the set bits of a word in ascending order.
+//
 // Warp roles (512 threads):
 //   warps 0-3 / 4-7  softmax warpgroup 0 / 1; thread r of a group owns
 //                    query row r = TMEM lane r (warp w reaches lanes
 //                    32*(w%4)..+31); group 0 first copies Q into TMEM
-//   warp 8           stages the index lists, merges them, publishes each
-//                    step, and copies box 0 (head_dim 0-63) of even steps' K
+//   warp 8           builds the step bitmaps, then copies box 0 (head_dim
+//                    0-63) of even steps' K
 //   warp 9           TMEM allocator; one thread issues the score bursts
 //   warp 10          K box 0 of odd steps
 //   warps 11 / 12    K box 1 (head_dim 64-127) of even / odd steps
@@ -58,13 +64,14 @@
 namespace bsa {
 namespace {
 
+constexpr int kMaxWords = kAttnMaxBlocks / 32;  // step-bitmap words per query block
+
 template <int D>
 struct Cfg {
   static constexpr int kThreads = 512;
   static constexpr int KB = D / 64;  // 64-column boxes per block (copy streams per ring)
   static constexpr int KS = 8;                    // K ring stages (even: pairs)
   static constexpr int VS = 5;                    // V ring stages
-  static constexpr int IR = 16;                   // step-info ring entries
   static constexpr int BLK_BYTES = 64 * D * 2;    // one K (or V) block
   static constexpr int BOX = 64 * 128;            // one 64-column TMA box of a block
   static constexpr uint32_t TMEM_COLS = 512;
@@ -72,69 +79,52 @@ struct Cfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = KS * BLK_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * BLK_BYTES;
-  // kfull[KS] kempty[KS] vfull[VS] vempty[VS] qready s sfree[2] p[2] o[2] drain[2]
-  static constexpr int N_BARS = 2 * KS + 2 * VS + 11;
-  static constexpr int OFF_INFO = OFF_BAR + 8 * N_BARS;
-  static constexpr int OFF_XCH = OFF_INFO + 24 * IR;  // float m[2][128], l[2][128]
-  static constexpr int LIST_CAP = 1024;  // index-list entries cached per query block
-  static constexpr int FULL_CAP = 2560;  // blocks whose full/partial byte is cached
-  static constexpr int OFF_LIST = OFF_XCH + 4 * 4 * 128;
-  static constexpr int OFF_FULL = OFF_LIST + 2 * 4 * LIST_CAP;
-  static constexpr int OFF_MISC = OFF_FULL + FULL_CAP;
+  // kfull[KS] kempty[KS] vfull[VS] vempty[VS] qready s sfree[2] p[2] o[2] drain[2] steps
+  static constexpr int N_BARS = 2 * KS + 2 * VS + 12;
+  static constexpr int OFF_XCH = OFF_BAR + 8 * N_BARS;  // float m[2][128], l[2][128]
+  static constexpr int OFF_BM = OFF_XCH + 4 * 4 * 128;   // uint32 A, B, F [kMaxWords]
+  static constexpr int OFF_MISC = OFF_BM + 3 * 4 * kMaxWords;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(KS % 2 == 0, "step pairs must not straddle the K ring's end");
-  // A step's info entry is overwritten only after the score burst of the
-  // step KS later has run, which needs both groups past step j+KS-2.
-  static_assert(IR > KS + 2 && IR <= 32, "step-info ring size");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-struct StepInfo {
-  int32_t tag;     // j+1 once the entry describes step j (0 = none yet)
-  int32_t tile;    // key block, or -1 = no more steps
-  uint32_t flags;  // bit 0: first query block keeps it; bit 1: second one
-  uint32_t pad;
-  uint64_t vmask;  // valid-slot mask of the key block
-};
-static_assert(sizeof(StepInfo) == 24, "StepInfo layout");
-
-// Iterator over the kept key blocks of one query block, in rotated order:
-// blocks >= `start` ascending, then the blocks below `start` ascending.
-// CTAs working on the same head start at different blocks, so they do not
-// all fetch the same K/V tiles at the same moment (the online softmax does
-// not depend on the order of its steps).  p points to the shared-memory
-// copy of the list, or to global memory for very long lists; a dense row
-// walks every block.  peek() returns the rotated key (block - start) mod nb
-// of the next block, INT_MAX when done.
-struct ListIt {
-  const int32_t* p;
-  int n;       // list length (every block for a dense row)
-  bool dense;
-  int first;   // position of the first block >= start
-  int taken;   // blocks handed out so far
-  int start, nb;
-  __device__ void init(int start_, int nb_) {
-    start = start_;
-    nb = nb_;
-    taken = 0;
-    if (dense) {
-      first = start;
-      return;
+// Cursor over the step sequence: the set bits of A|B, words visited in the
+// rotated order ws, ws+1, .., nw-1, 0, .., ws-1 (CTAs working on the same
+// head start at different words, so they do not all fetch the same K/V
+// tiles at the same moment; the online softmax does not depend on the
+// order of its steps) and bits within a word in ascending order.  next()
+// returns the key block of the next step and its flags (bit 0: the first
+// query block keeps it, bit 1: the second one, bit 2: all 64 slots of the
+// key block are real tokens), or -1 past the last word.
+struct StepCursor {
+  int w;              // current word
+  uint32_t cur = 0u;  // union bits of the current word not handed out yet
+  __device__ explicit StepCursor(int ws) : w(ws - 1) {}
+  // A = first query block's bitmap; B = A + kMaxWords, F (full key blocks)
+  // = A + 2 * kMaxWords.  Reaching a word with a set bit takes at most nw
+  // word loads, so a walk past the last step ends with -1 instead of looping.
+  __device__ int next(const uint32_t* A, int nw, uint32_t& flags) {
+    for (int guard = 0; cur == 0u; ++guard) {
+      if (guard >= nw) return -1;
+      w = w + 1 == nw ? 0 : w + 1;
+      cur = A[w] | A[kMaxWords + w];
     }
-    int lo = 0, hi = n;  // lower_bound(p, p+n, start)
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (p[mid] < start) lo = mid + 1; else hi = mid;
-    }
-    first = lo;
+    const int bit = __ffs(cur) - 1;
+    cur &= cur - 1u;
+    flags = ((A[w] >> bit) & 1u) | (((A[kMaxWords + w] >> bit) & 1u) << 1) |
+            (((A[2 * kMaxWords + w] >> bit) & 1u) << 2);
+    return w * 32 + bit;
   }
-  __device__ int block_at(int i) const { return dense ? i : p[i]; }
-  __device__ int peek() const {
-    if (taken >= n) return INT_MAX;
-    int i = first + taken;
-    if (i >= n) i -= n;
-    const int v = block_at(i);
-    return v >= start ? v - start : v + nb - start;
+  __device__ int next(const uint32_t* A, int nw) {
+    for (int guard = 0; cur == 0u; ++guard) {
+      if (guard >= nw) return -1;
+      w = w + 1 == nw ? 0 : w + 1;
+      cur = A[w] | A[kMaxWords + w];
+    }
+    const int bit = __ffs(cur) - 1;
+    cur &= cur - 1u;
+    return w * 32 + bit;
   }
 };
 
@@ -169,7 +159,7 @@ __global__ void __launch_bounds__(512, 1)
                     const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
                     __nv_bfloat16* __restrict__ out, int32_t* __restrict__ status) {
   using C = Cfg<D>;
-  constexpr int KS = C::KS, VS = C::VS, IR = C::IR;
+  constexpr int KS = C::KS, VS = C::VS;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -186,10 +176,14 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t bar_p = bar_qready + 32;      // [2] P written + O corrected (128 arrivals)
   const uint32_t bar_o = bar_qready + 48;      // [2] PV of group w finished
   const uint32_t bar_drain = bar_qready + 64;  // [2] score issuer, PV issuer
-  StepInfo* info = reinterpret_cast<StepInfo*>(sm + C::OFF_INFO);
+  const uint32_t bar_steps = bar_qready + 80;  // step bitmaps built (32 arrivals)
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);  // first query block's keys
+  uint32_t* bmB = bmA + kMaxWords;                                 // second query block's keys
+  uint32_t* bmF = bmA + 2 * kMaxWords;                             // key blocks with no pad slot
   float* xch = reinterpret_cast<float*>(sm + C::OFF_XCH);  // m[2][128] then l[2][128]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
+  int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
@@ -212,10 +206,10 @@ __global__ void __launch_bounds__(512, 1)
     }
     mbar_init(bar_drain, 1);
     mbar_init(bar_drain + 8, 1);
+    mbar_init(bar_steps, 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8 && lane < IR) info[lane].tag = 0;
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
@@ -224,105 +218,81 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const int nw = (g.nb + 31) >> 5;
+  const int ws = int((uint32_t(pair) * 61u + uint32_t(bh) * 17u) % uint32_t(nw));
 
-  if (warp == 8) {
-    // ---------------------------------------------- list merge + K box 0
-    // The whole warp stages both index lists and the per-block "all slots
-    // valid" bytes in shared memory; lane 0 then merges the lists, publishes
-    // step j once K stage j%KS is free (so an info entry is never reused
-    // before every reader is past it) and copies box 0 of K_j.  After the
-    // last step it publishes two end markers (steps n and n+1).
-    int32_t* slist = reinterpret_cast<int32_t*>(sm + C::OFF_LIST);
-    uint8_t* sfull = sm + C::OFF_FULL;
-    const bool full_cached = g.nb <= C::FULL_CAP;
-    const uint8_t* gfull = bfull + int64_t(b) * g.nb;
-    if (full_cached)
-      for (int i = lane; i < g.nb; i += 32) sfull[i] = __ldg(gfull + i);
-    ListIt it[2];
-    for (int hf = 0; hf < 2; ++hf) {
-      const int qb = 2 * pair + hf;
-      it[hf].p = nullptr;
-      it[hf].n = 0;
-      it[hf].dense = false;
-      if (qb < g.nb) {
+  if (warp == 8 || warp == 10 || warp == 11 || warp == 12 || warp == 14 || warp == 15) {
+    if (warp == 8) {
+      // ------------------------------------------------------ step bitmaps
+      // Bit t of A (B) is set when the first (second) query block of the
+      // pair keeps key block t; a dense row keeps every block.  Entries
+      // outside 0..nb-1 are ignored rather than trusted.
+      for (int w = lane; w < nw; w += 32) {
+        bmA[w] = 0u;
+        bmB[w] = 0u;
+      }
+      __syncwarp();
+      for (int hf = 0; hf < 2; ++hf) {
+        const int qb = 2 * pair + hf;
+        if (qb >= g.nb) continue;
+        uint32_t* bm = hf ? bmB : bmA;
         const int c = DENSE ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
         if (c < 0) {
-          it[hf].dense = true;
-          it[hf].n = g.nb;
+          for (int w = lane; w < nw; w += 32) {
+            const int rem = g.nb - 32 * w;
+            bm[w] = rem >= 32 ? ~0u : ((1u << rem) - 1u);
+          }
         } else {
+          const int n = c < g.kcap ? c : g.kcap;
           const int32_t* src = idx + (int64_t(bh) * g.nb + qb) * g.kcap;
-          it[hf].n = c;
-          if (c <= C::LIST_CAP) {
-            for (int i = lane; i < c; i += 32) slist[hf * C::LIST_CAP + i] = __ldg(src + i);
-            it[hf].p = slist + hf * C::LIST_CAP;
-          } else {
-            it[hf].p = src;
+          for (int base = 0; base < n; base += 8 * 32) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = base + 32 * u + lane;
+              v[u] = i < n ? __ldg(src + i) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              if (v[u] >= 0 && v[u] < g.nb) atomicOr(bm + (v[u] >> 5), 1u << (v[u] & 31));
           }
         }
       }
+      // F: blocks whose 64 slots are all real tokens (no valid-slot mask needed)
+      const uint8_t* full_row = bfull + int64_t(b) * g.nb;
+      for (int w = lane; w < nw; w += 32) {
+        uint8_t by[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) by[i] = 32 * w + i < g.nb ? __ldg(full_row + 32 * w + i) : 0;
+        uint32_t f = 0u;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f |= uint32_t(by[i] != 0) << i;
+        bmF[w] = f;
+      }
+      __syncwarp();
+      int cntw = 0;
+      for (int w = lane; w < nw; w += 32) cntw += __popc(bmA[w] | bmB[w]);
+      cntw = __reduce_add_sync(0xffffffffu, cntw);
+      if (lane == 0) *n_steps_sm = cntw;
+      __syncwarp();
+      mbar_arrive(bar_steps);  // release: every lane's bitmap writes
     }
-    __syncwarp();
-    if (lane == 0) {
-      tma_prefetch_desc(&mk);
-      tma_prefetch_desc(&mv);
-      const int start = int((uint32_t(pair) * 61u + uint32_t(bh) * 17u) % uint32_t(g.nb));
-      it[0].init(start, g.nb);
-      it[1].init(start, g.nb);
-      int j = 0, ends = 0;
-      bool ok = true;
-      for (;; ++j) {
-        const int s = j % KS;
-        if (j >= KS && !mbar_wait(kempty(s), ((j / KS) - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        StepInfo& e = info[j % IR];
-        int t = INT_MAX;
-        if (ends == 0) {
-          const int ra = it[0].peek(), rb = it[1].peek();
-          const int r = ra < rb ? ra : rb;
-          if (r != INT_MAX) {
-            t = r + start < g.nb ? r + start : r + start - g.nb;
-            uint32_t flags = 0;
-            if (ra == r) { flags |= 1u; ++it[0].taken; }
-            if (rb == r) { flags |= 2u; ++it[1].taken; }
-            const bool whole = full_cached ? (sfull[t] != 0) : (__ldg(gfull + t) != 0);
-            e.tile = t;
-            e.flags = flags;
-            e.vmask = whole ? ~0ull : __ldg(bmask + int64_t(b) * g.nb + t);
-          }
-        }
-        if (t == INT_MAX) e.tile = -1;
-        __threadfence_block();
-        *reinterpret_cast<volatile int32_t*>(&e.tag) = j + 1;
-        if ((j & 1) == 0) {  // K box 0 of even steps
-          if (t == INT_MAX) {
-            mbar_arrive(kfull(s));
-          } else {
-            mbar_arrive_expect_tx(kfull(s), C::BOX);
-            tma_load_3d(sK + s * C::BOX, &mk, kfull(s), 0, t * 64, bh);
-          }
-        }
-        if (t == INT_MAX && ++ends == 2) break;
-      }
-      if (!ok) {
-        report_timeout(abort_flag, status);
-        for (int jj = j - 1; jj >= 0 && jj >= j - KS; --jj)
-          mbar_wait(kfull(jj % KS), (jj / KS) & 1, nullptr, 200000000ull);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 10 || warp == 11 || warp == 12 || warp == 14 || warp == 15) {
-    // ---------------------------------------------- K box 0 odd, K box 1, V
+    // ---------------------------------------------- K box 0 / box 1, V copies
     const bool is_k = warp <= 12;
-    const int bx = warp == 10 ? 0 : 1;        // K box (unused for V)
-    const int par = (warp == 11 || warp == 14) ? 0 : 1;
+    const int bx = (warp == 8 || warp == 10) ? 0 : 1;  // K box (unused for V)
+    const int par = (warp == 8 || warp == 11 || warp == 14) ? 0 : 1;
     if (lane == 0 && (!is_k || bx < C::KB)) {
+      if (is_k)
+        tma_prefetch_desc(&mk);
+      else
+        tma_prefetch_desc(&mv);
       const int RS = is_k ? KS : VS;
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0;
+      StepCursor sc(ws);
+      if (par == 1 && n > 0) sc.next(bmA, nw);  // step 0 belongs to the other parity
       int j = par;
-      bool ok = true;
-      for (;; j += 2) {
-        // sleep on the ring first; the step is normally published by then
+      for (; ok && j < n; j += 2) {
         const int s = j % RS;
         const uint32_t emp = is_k ? kempty(s) : vempty(s);
         const uint32_t ful = is_k ? kfull(s) : vfull(s);
@@ -330,25 +300,12 @@ __global__ void __launch_bounds__(512, 1)
           ok = false;
           break;
         }
-        const StepInfo& e = info[j % IR];
-        {
-          bool seen = false;
-          IdleClock clk;
-          for (;;) {
-            seen = *reinterpret_cast<const volatile int32_t*>(&e.tag) == j + 1;
-            if (seen || clk.expired(abort_flag)) break;
-          }
-          if (!seen) {
-            ok = false;
-            break;
-          }
-        }
-        __threadfence_block();
-        const int t = *reinterpret_cast<const volatile int32_t*>(&e.tile);
-        if (t < 0) {  // each parity meets exactly one of the two end markers
-          if (is_k) mbar_arrive(ful);
+        const int t = sc.next(bmA, nw);
+        if (t < 0) {  // the bitmaps hold fewer steps than counted: cannot happen
+          ok = false;
           break;
         }
+        if (j + 1 < n) sc.next(bmA, nw);  // skip the other parity's step
         if (is_k) {
           mbar_arrive_expect_tx(ful, C::BOX);
           tma_load_3d(sK + (bx * KS + s) * C::BOX, &mk, ful, 64 * bx, t * 64, bh);
@@ -370,30 +327,32 @@ __global__ void __launch_bounds__(512, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ score bursts
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-      bool ok = mbar_wait(bar_qready, 0, abort_flag);
+      constexpr uint32_t idesc_qk2 = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_qk1 = idesc_bf16_f32(128, 64, false);
+      bool ok = mbar_wait(bar_qready, 0, abort_flag) && mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0;
       // pair t: scores of steps 2t and 2t+1 into S0 | S1 (adjacent TMEM
       // columns); needs K of both steps and both groups done reading the
-      // previous pair's S
-      for (int t = 0; ok; ++t) {
+      // previous pair's S.  An odd last step gets an N=64 burst of its own.
+      for (int t = 0; ok && 2 * t < n; ++t) {
         const int j0 = 2 * t, s0 = j0 % KS;
+        const bool two = j0 + 1 < n;
         if (t > 0) ok = mbar_wait(bar_sfree, (t - 1) & 1, abort_flag) &&
                         mbar_wait(bar_sfree + 8, (t - 1) & 1, abort_flag);
         if (ok) ok = mbar_wait(kfull(s0), (j0 / KS) & 1, abort_flag) &&
-                     mbar_wait(kfull(s0 + 1), ((j0 + 1) / KS) & 1, abort_flag);
+                     (!two || mbar_wait(kfull(s0 + 1), ((j0 + 1) / KS) & 1, abort_flag));
         if (!ok) break;
-        if (*reinterpret_cast<volatile int32_t*>(&info[j0 % IR].tile) < 0) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t bd =
               sdesc_sw128(sK + ((kk / 4) * KS + s0) * C::BOX + (kk % 4) * 32, 16, 1024);
-          tc_mma_ts(tmem + C::COL_S, tmem + C::COL_Q + 8u * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          tc_mma_ts(tmem + C::COL_S, tmem + C::COL_Q + 8u * kk, bd, two ? idesc_qk2 : idesc_qk1,
+                    kk > 0 ? 1u : 0u);
         }
         tc_commit(bar_s);
         tc_commit(kempty(s0));
-        tc_commit(kempty(s0 + 1));
-        if (*reinterpret_cast<volatile int32_t*>(&info[(j0 + 1) % IR].tile) < 0) break;
+        if (two) tc_commit(kempty(s0 + 1));
       }
       if (!ok) report_timeout(abort_flag, status);
       // every MMA this thread issued has completed once its drain barrier flips
@@ -403,29 +362,21 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------------------------------------ PV issuer
-    // Two independent queues (one per softmax group), served in whichever
-    // order they become ready: PV_j needs P_j and V_j.  A group is done at
-    // its first end marker.
+    // Two independent queues (one per softmax group: the even and the odd
+    // steps), served in whichever order they become ready: PV_j needs P_j
+    // and V_j.
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0;
       int jp[2] = {0, 1};
-      bool done[2] = {false, false};
-      bool ok = true;
       IdleClock clk;
-      while (ok && !(done[0] && done[1])) {
+      while (ok && (jp[0] < n || jp[1] < n)) {
         bool progress = false;
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-          if (done[w]) continue;
           const int j = jp[w];
-          const StepInfo& e = info[j % IR];
-          if (*reinterpret_cast<const volatile int32_t*>(&e.tag) != j + 1) continue;
-          __threadfence_block();
-          if (*reinterpret_cast<const volatile int32_t*>(&e.tile) < 0) {
-            done[w] = true;
-            progress = true;
-            continue;
-          }
+          if (j >= n) continue;
           const int s = j % VS;
           if (!mbar_test(bar_p + 8 * w, (j >> 1) & 1) || !mbar_test(vfull(s), (j / VS) & 1))
             continue;
@@ -496,23 +447,21 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = g.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l_sum = 0.f;
     int k = 0;  // steps of this group so far
-    for (int j = wg;; j += 2, ++k) {
-      // the producer publishes step j's info (tag j+1) before its K copy
-      const StepInfo& e = info[j % IR];
-      {
-        bool seen = false;
-        IdleClock clk;
-        for (;;) {
-          seen = *reinterpret_cast<const volatile int32_t*>(&e.tag) == j + 1;
-          if (seen || clk.expired(abort_flag)) break;
-        }
-        ok = __all_sync(0xffffffffu, seen);
-        if (!ok) break;
+    // this group's steps are every other step of the cursor walk; the flags
+    // and the valid-slot mask of a step are fetched one step ahead
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const int n = ok ? *n_steps_sm : 0;
+    const uint64_t* bm_row = bmask + int64_t(b) * g.nb;
+    StepCursor sc(ws);
+    if (wg == 1 && n > 0) sc.next(bmA, nw);  // step 0 belongs to group 0
+    for (int j = wg; ok && j < n; j += 2, ++k) {
+      uint32_t flags;
+      const int tile = sc.next(bmA, nw, flags);
+      if (tile < 0) {
+        ok = false;
+        break;
       }
-      __threadfence_block();
-      if (*reinterpret_cast<const volatile int32_t*>(&e.tile) < 0) break;
-      const uint32_t flags = *reinterpret_cast<const volatile uint32_t*>(&e.flags);
-      const uint64_t vm = *reinterpret_cast<const volatile uint64_t*>(&e.vmask);
+      if (j + 1 < n) sc.next(bmA, nw);  // the other group's step
       const bool member = (flags >> half) & 1u;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s, k & 1, abort_flag));
       if (!ok) break;
@@ -525,8 +474,9 @@ __global__ void __launch_bounds__(512, 1)
         BSA_TMEM_LD64(tS, r);
         tc_fence_before();
         mbar_arrive(bar_sfree + 8 * wg);
+        const bool all_valid = (flags & 4u) != 0u;
+        const uint64_t vm = all_valid ? ~0ull : __ldg(bm_row + tile);
         const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
-        const bool all_valid = (lo & hi) == 0xFFFFFFFFu;
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (all_valid) {
 #pragma unroll

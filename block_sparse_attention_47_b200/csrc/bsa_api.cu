@@ -103,6 +103,9 @@ bsa_status make_geo(const bsa_problem* p, Geo* g) {
   g->tau = p->dyn_tau;
   g->scale = p->softmax_scale;
   if (int64_t(p->B) * p->heads > 65535) return fail(BSA_ERR_SHAPE, "B*heads must be <= 65535");
+  if (g->nb > bsa::kAttnMaxBlocks)
+    return fail(BSA_ERR_UNSUPPORTED, "%d blocks per sequence; the attention kernel walks at most %d",
+                g->nb, bsa::kAttnMaxBlocks);
   if (bsa::select_smem_bytes(*g) > kMaxSmem)
     return fail(BSA_ERR_UNSUPPORTED, "too many video blocks (%d) for on-chip selection", g->nbv);
   return BSA_OK;

@@ -13,6 +13,8 @@
 namespace bsa {
 
 constexpr int kBlock = 64;       // tokens per block
+// blocks per sequence the attention kernel walks with on-chip step bitmaps
+constexpr int kAttnMaxBlocks = 8192;
 
 // Everything a kernel needs to know about a problem (plain integers).
 struct Geo {
