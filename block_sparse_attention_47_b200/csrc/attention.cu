@@ -47,11 +47,11 @@
 //   warp 10          K box 0 of odd steps
 //   warps 11 / 12    K box 1 (head_dim 64-127) of even / odd steps
 //   warp 13          one thread issues the PV MMAs of both softmax groups
-//   warps 14 / 15    V of even / odd steps (both halves in one copy)
+//   warps 14 / 15    V of even / odd steps (both 64-column boxes)
 // One issuing thread completes about one bulk tensor copy per ~650 cycles
-// whatever its size, so copies are spread over six warps and V moves as a
-// single 16 KB copy; tcgen05.mma blocks its issuing thread while the tensor
-// pipe is busy, so score bursts and PVs come from two threads.
+// whatever its size, so copies are spread over six warps; tcgen05.mma
+// blocks its issuing thread while the tensor pipe is busy, so score bursts
+// and PVs come from two threads.
 // Tensor memory (512 columns): Q [0,64) bf16 pairs | S0 [64,128) | S1
 // [128,192) | P0 [192,224) | P1 [224,256) | O0 [256,384) | O1 [384,512).
 //
@@ -310,11 +310,11 @@ __global__ void __launch_bounds__(512, 1)
           mbar_arrive_expect_tx(ful, C::BOX);
           tma_load_3d(sK + (bx * KS + s) * C::BOX, &mk, ful, 64 * bx, t * 64, bh);
         } else {
+          // both 64-column boxes of the block, [box][row][64] in the stage
           mbar_arrive_expect_tx(ful, C::BLK_BYTES);
-          if constexpr (D == 128)
-            tma_load_4d(sV + s * C::BLK_BYTES, &mv, ful, 0, t * 64, 0, bh);
-          else
-            tma_load_3d(sV + s * C::BLK_BYTES, &mv, ful, 0, t * 64, bh);
+#pragma unroll
+          for (int hb = 0; hb < C::KB; ++hb)
+            tma_load_3d(sV + s * C::BLK_BYTES + hb * C::BOX, &mv, ful, 64 * hb, t * 64, bh);
         }
       }
       if (!ok) {

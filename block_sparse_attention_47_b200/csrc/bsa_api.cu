@@ -163,24 +163,6 @@ bsa_status make_map(CUtensorMap* m, const Geo& g, const void* ptr, int rows) {
   return BSA_OK;
 }
 
-// The same tensor viewed as [B*heads, 2 halves, N, 64]: one box of
-// 64 rows x both halves lands in shared memory as [half][row][64], i.e. the
-// two 64-column boxes of a block back to back, in a single copy.
-bsa_status make_map_halves(CUtensorMap* m, const Geo& g, const void* ptr) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint64_t dims[4] = {64, cuuint64_t(g.N), 2, cuuint64_t(g.B) * g.h};
-  cuuint64_t strides[3] = {cuuint64_t(g.d) * 2, 128, cuuint64_t(g.N) * g.d * 2};
-  cuuint32_t box[4] = {64, 64, 2, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (two-half view) failed (%d)", int(r));
-  return BSA_OK;
-}
-
 bsa_status check_device() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -322,10 +304,7 @@ static bsa_status attention_common(const bsa_problem* prob, const void* layout_b
   BSA_TRY(check_device());
   CUtensorMap maps[2];
   BSA_TRY(make_map(&maps[0], g, k_perm, 64));
-  if (g.d == 128)
-    BSA_TRY(make_map_halves(&maps[1], g, v_perm));
-  else
-    BSA_TRY(make_map(&maps[1], g, v_perm, 64));
+  BSA_TRY(make_map(&maps[1], g, v_perm, 64));
   int32_t* status = dev_status;
   if (!status) {
     cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dev_status_sink);
