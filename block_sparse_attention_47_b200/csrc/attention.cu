@@ -47,7 +47,7 @@
 //   warp 10          K box 0 of odd steps
 //   warps 11 / 12    K box 1 (head_dim 64-127) of even / odd steps
 //   warp 13          one thread issues the PV MMAs of both softmax groups
-//   warps 14 / 15    V of even / odd steps (both 64-column boxes)
+//   warps 14 / 15    V box 0 / box 1 of every step
 // One issuing thread completes about one bulk tensor copy per ~650 cycles
 // whatever its size, so copies are spread over six warps; tcgen05.mma
 // blocks its issuing thread while the tensor pipe is busy, so score bursts
@@ -137,20 +137,6 @@ __device__ __forceinline__ bool bit_of(uint32_t lo, uint32_t hi, int c) {
   return ((c < 32 ? (lo >> c) : (hi >> (c - 32))) & 1u) != 0u;
 }
 
-// Idle bookkeeping for the polling loops: expired() turns true once no
-// progress was made for 2 s or another role has aborted.
-struct IdleClock {
-  uint32_t idle = 0;
-  uint64_t since = 0;
-  __device__ void progress() { idle = 0; }
-  __device__ bool expired(volatile int* abort_flag) {
-    if ((++idle & 255) != 0) return false;
-    const uint64_t now = global_timer_ns();
-    if (idle == 256) since = now;
-    return *abort_flag || now - since > 2000000000ull;
-  }
-};
-
 template <int D, bool DENSE>
 __global__ void __launch_bounds__(512, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
@@ -194,7 +180,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(kempty(s), 1);
     }
     for (int s = 0; s < VS; ++s) {
-      mbar_init(vfull(s), 1);
+      mbar_init(vfull(s), C::KB);
       mbar_init(vempty(s), 1);
     }
     mbar_init(bar_qready, 128);
@@ -278,10 +264,16 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(bar_steps);  // release: every lane's bitmap writes
     }
     // ---------------------------------------------- K box 0 / box 1, V copies
+    // K: one warp per (box, step parity); a K stage is only ever reused by
+    // steps of one parity (KS is even), so each warp's ring waits are in
+    // order.  V: one warp per box over every step, because a V stage is
+    // reused by steps of both parities (VS is odd): a warp that skipped the
+    // other parity's uses could test a ring barrier two phases behind.
     const bool is_k = warp <= 12;
-    const int bx = (warp == 8 || warp == 10) ? 0 : 1;  // K box (unused for V)
-    const int par = (warp == 8 || warp == 11 || warp == 14) ? 0 : 1;
-    if (lane == 0 && (!is_k || bx < C::KB)) {
+    const int bx = is_k ? ((warp == 8 || warp == 10) ? 0 : 1) : warp - 14;
+    const int par = is_k ? ((warp == 8 || warp == 11) ? 0 : 1) : 0;
+    const int stride = is_k ? 2 : 1;
+    if (lane == 0 && bx < C::KB) {
       if (is_k)
         tma_prefetch_desc(&mk);
       else
@@ -292,7 +284,7 @@ __global__ void __launch_bounds__(512, 1)
       StepCursor sc(ws);
       if (par == 1 && n > 0) sc.next(bmA, nw);  // step 0 belongs to the other parity
       int j = par;
-      for (; ok && j < n; j += 2) {
+      for (; ok && j < n; j += stride) {
         const int s = j % RS;
         const uint32_t emp = is_k ? kempty(s) : vempty(s);
         const uint32_t ful = is_k ? kfull(s) : vfull(s);
@@ -305,21 +297,17 @@ __global__ void __launch_bounds__(512, 1)
           ok = false;
           break;
         }
-        if (j + 1 < n) sc.next(bmA, nw);  // skip the other parity's step
-        if (is_k) {
-          mbar_arrive_expect_tx(ful, C::BOX);
+        if (stride == 2 && j + 1 < n) sc.next(bmA, nw);  // skip the other parity's step
+        // box bx of the block: [box][row][64] in the stage
+        mbar_arrive_expect_tx(ful, C::BOX);
+        if (is_k)
           tma_load_3d(sK + (bx * KS + s) * C::BOX, &mk, ful, 64 * bx, t * 64, bh);
-        } else {
-          // both 64-column boxes of the block, [box][row][64] in the stage
-          mbar_arrive_expect_tx(ful, C::BLK_BYTES);
-#pragma unroll
-          for (int hb = 0; hb < C::KB; ++hb)
-            tma_load_3d(sV + s * C::BLK_BYTES + hb * C::BOX, &mv, ful, 64 * hb, t * 64, bh);
-        }
+        else
+          tma_load_3d(sV + s * C::BLK_BYTES + bx * C::BOX, &mv, ful, 64 * bx, t * 64, bh);
       }
       if (!ok) {
         report_timeout(abort_flag, status);
-        for (int jj = j - 2; jj >= 0 && jj >= j - 2 * RS; jj -= 2)
+        for (int jj = j - stride; jj >= 0 && jj >= j - stride * RS; jj -= stride)
           mbar_wait(ful_of(is_k, jj % RS), (jj / RS) & 1, nullptr, 200000000ull);
       }
     }
@@ -362,40 +350,28 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------------------------------------ PV issuer
-    // Two independent queues (one per softmax group: the even and the odd
-    // steps), served in whichever order they become ready: PV_j needs P_j
-    // and V_j.
+    // PVs in step order (groups alternate): PV_j needs P_j and V_j.  The
+    // order matters for the V ring: a stage is reused every VS steps by
+    // both groups, and testing its barrier for step j is unambiguous only
+    // once PV_{j-VS} has been issued.
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
       const int n = ok ? *n_steps_sm : 0;
-      int jp[2] = {0, 1};
-      IdleClock clk;
-      while (ok && (jp[0] < n || jp[1] < n)) {
-        bool progress = false;
+      for (int j = 0; ok && j < n; ++j) {
+        const int w = j & 1, s = j % VS;
+        ok = mbar_wait(bar_p + 8 * w, (j >> 1) & 1, abort_flag) &&
+             mbar_wait(vfull(s), (j / VS) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const int j = jp[w];
-          if (j >= n) continue;
-          const int s = j % VS;
-          if (!mbar_test(bar_p + 8 * w, (j >> 1) & 1) || !mbar_test(vfull(s), (j / VS) & 1))
-            continue;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = sdesc_sw128(sV + s * C::BLK_BYTES + kk * 2048, C::BOX, 1024);
-            tc_mma_ts(tmem + C::COL_O + 128u * w, tmem + C::COL_P + 32u * w + 8u * kk, bd,
-                      idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(bar_o + 8 * w);
-          tc_commit(vempty(s));
-          jp[w] = j + 2;
-          progress = true;
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = sdesc_sw128(sV + s * C::BLK_BYTES + kk * 2048, C::BOX, 1024);
+          tc_mma_ts(tmem + C::COL_O + 128u * w, tmem + C::COL_P + 32u * w + 8u * kk, bd,
+                    idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
         }
-        if (progress)
-          clk.progress();
-        else if (clk.expired(abort_flag))
-          ok = false;
+        tc_commit(bar_o + 8 * w);
+        tc_commit(vempty(s));
       }
       if (!ok) report_timeout(abort_flag, status);
       tc_commit(bar_drain + 8);
@@ -480,7 +456,9 @@ __global__ void __launch_bounds__(512, 1)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (all_valid) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
+          for (int c = 0; c < 64; c += 2)
+            mx[(c >> 1) & 3] =
+                max3f(mx[(c >> 1) & 3], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
         } else {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
@@ -496,11 +474,16 @@ __global__ void __launch_bounds__(512, 1)
         }
         float sum[4] = {0.f, 0.f, 0.f, 0.f};
         if (all_valid) {
+          // two columns per instruction for the scaling and the row sum
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, -m_used));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, -m_used));
-            sum[(c >> 1) & 3] += p0 + p1;
+            float x0, x1;
+            fma_f32x2(x0, x1, __uint_as_float(r[c]), __uint_as_float(r[c + 1]), sl2, sl2, -m_used,
+                      -m_used);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            const int a = (c >> 1) & 1;
+            add_f32x2(sum[2 * a], sum[2 * a + 1], sum[2 * a], sum[2 * a + 1], p0, p1);
             pk[c / 2] = pack_bf16x2(p0, p1);
           }
         } else {
