@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(512, 1)
   auto ful_of = [&](bool k, int s) { return k ? kfull(s) : vfull(s); };
   const uint32_t bar_qready = bar0 + 8u * (2 * KS + 2 * VS);
   const uint32_t bar_s = bar_qready + 8;       // S of a step pair ready
-  const uint32_t bar_sfree = bar_qready + 16;  // [2] group w has read its S (128 arrivals)
+  const uint32_t bar_sfree = bar_qready + 16;  // both groups have read their S (256 arrivals)
   const uint32_t bar_p = bar_qready + 32;      // [2] P written + O corrected (128 arrivals)
   const uint32_t bar_o = bar_qready + 48;      // [2] PV of group w finished
   const uint32_t bar_drain = bar_qready + 64;  // [2] score issuer, PV issuer
@@ -185,8 +185,8 @@ __global__ void __launch_bounds__(512, 1)
     }
     mbar_init(bar_qready, 128);
     mbar_init(bar_s, 1);
+    mbar_init(bar_sfree, 256);
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bar_sfree + 8 * w, 128);
       mbar_init(bar_p + 8 * w, 128);
       mbar_init(bar_o + 8 * w, 1);
     }
@@ -325,10 +325,10 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; ok && 2 * t < n; ++t) {
         const int j0 = 2 * t, s0 = j0 % KS;
         const bool two = j0 + 1 < n;
-        if (t > 0) ok = mbar_wait(bar_sfree, (t - 1) & 1, abort_flag) &&
-                        mbar_wait(bar_sfree + 8, (t - 1) & 1, abort_flag);
-        if (ok) ok = mbar_wait(kfull(s0), (j0 / KS) & 1, abort_flag) &&
-                     (!two || mbar_wait(kfull(s0 + 1), ((j0 + 1) / KS) & 1, abort_flag));
+        // K normally lands long before the groups free S: wait for it first
+        ok = mbar_wait(kfull(s0), (j0 / KS) & 1, abort_flag) &&
+             (!two || mbar_wait(kfull(s0 + 1), ((j0 + 1) / KS) & 1, abort_flag));
+        if (ok && t > 0) ok = mbar_wait(bar_sfree, (t - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -360,8 +360,8 @@ __global__ void __launch_bounds__(512, 1)
       const int n = ok ? *n_steps_sm : 0;
       for (int j = 0; ok && j < n; ++j) {
         const int w = j & 1, s = j % VS;
-        ok = mbar_wait(bar_p + 8 * w, (j >> 1) & 1, abort_flag) &&
-             mbar_wait(vfull(s), (j / VS) & 1, abort_flag);
+        ok = mbar_wait(vfull(s), (j / VS) & 1, abort_flag) &&
+             mbar_wait(bar_p + 8 * w, (j >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t r[64];
         BSA_TMEM_LD64(tS, r);
         tc_fence_before();
-        mbar_arrive(bar_sfree + 8 * wg);
+        mbar_arrive(bar_sfree);
         const bool all_valid = (flags & 4u) != 0u;
         const uint64_t vm = all_valid ? ~0ull : __ldg(bm_row + tile);
         const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(512, 1)
         l_sum = l_sum * factor + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
       } else {
         tc_fence_before();
-        mbar_arrive(bar_sfree + 8 * wg);
+        mbar_arrive(bar_sfree);
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
