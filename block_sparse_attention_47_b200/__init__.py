@@ -14,6 +14,7 @@ strings them together for one attention layer:
 
     attn = BlockSparseAttention(problem)            # allocates the buffers
     out = attn(q, k, v)                             # raster [B, N, h, d] bf16
+    out = attn.host_call(q_cpu, k_cpu, v_cpu)       # host tensors, copies overlapped
 """
 import ctypes
 import math
@@ -87,6 +88,13 @@ class Sizes(ctypes.Structure):
                 ("cnt_bytes", ctypes.c_size_t)]
 
 
+class DeviceBuffers(ctypes.Structure):
+    """Mirror of bsa_device_buffers (device pointers of one whole call)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q_raster", "k_raster", "v_raster", "o_raster", "q_perm", "k_perm", "v_perm",
+                 "o_perm", "layout_buf", "q_pool", "k_pool", "idx", "cnt")]
+
+
 _LIB = None
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -102,6 +110,8 @@ _SIGS = {
     "bsa_dense_attn_fwd": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _P]),
     "bsa_unpermute": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _I64, _I64, _I64, _P]),
     "bsa_layout_stats": (ctypes.c_int, [ctypes.POINTER(Problem), _P, ctypes.POINTER(_I64), _P]),
+    "bsa_forward_host": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P,
+                                        ctypes.POINTER(DeviceBuffers), ctypes.c_int32, _P, _P]),
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_last_error": (ctypes.c_char_p, []),
 }
@@ -195,6 +205,26 @@ def unpermute(prob, layout_buf, o_perm, o_raster, stream=None):
                                sb, sn, sh, _stream(stream)))
 
 
+def forward_host(prob, q_host, k_host, v_host, o_host, buffers, heads_per_group, dev_status=None,
+                 stream=None):
+    """The whole call on host tensors, transfers overlapped with the
+    computation by groups of heads (bsa_forward_host)."""
+    for t in (q_host, k_host, v_host, o_host):
+        if t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("host tensors are contiguous [B, N, heads, head_dim] CPU tensors")
+    _check(lib().bsa_forward_host(ctypes.byref(prob), _ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                  _ptr(o_host), ctypes.byref(buffers), int(heads_per_group),
+                                  _ptr(dev_status), _stream(stream)))
+
+
+def default_heads_per_group(heads, groups=32):
+    """The smallest divisor of `heads` that makes at most `groups` groups."""
+    for hg in range(1, heads + 1):
+        if heads % hg == 0 and heads // hg <= groups:
+            return hg
+    return heads
+
+
 def layout_stats(prob, layout_buf, stream=None):
     hist = (_I64 * 7)()
     _check(lib().bsa_layout_stats(ctypes.byref(prob), _ptr(layout_buf), hist, _stream(stream)))
@@ -246,6 +276,33 @@ class BlockSparseAttention:
         unpermute(p, self.layout_buf, self.op, out, stream)
         return out
 
+    def device_buffers(self):
+        """bsa_device_buffers over this object's buffers (raster staging
+        buffers are allocated on first use)."""
+        if not hasattr(self, "_raster"):
+            shape = (self.prob.B, self.sizes.n_tokens, self.prob.heads, self.prob.head_dim)
+            self._raster = [torch.empty(shape, dtype=torch.bfloat16, device=self.qp.device)
+                            for _ in range(4)]
+        b = DeviceBuffers()
+        for name, t in zip(("q_raster", "k_raster", "v_raster", "o_raster"), self._raster):
+            setattr(b, name, t.data_ptr())
+        for name in ("q_perm", "k_perm", "v_perm", "o_perm"):
+            setattr(b, name, getattr(self, name[0] + "p").data_ptr())
+        b.layout_buf = self.layout_buf.data_ptr()
+        b.q_pool, b.k_pool = self.q_pool.data_ptr(), self.k_pool.data_ptr()
+        b.idx, b.cnt = self.idx.data_ptr(), self.cnt.data_ptr()
+        return b
+
+    def host_call(self, q_host, k_host, v_host, out=None, heads_per_group=None, stream=None):
+        """The call on host tensors (pinned memory lets the transfers overlap
+        the computation); returns the host output."""
+        if out is None:
+            out = torch.empty(q_host.shape, dtype=q_host.dtype, pin_memory=q_host.is_pinned())
+        hg = heads_per_group or default_heads_per_group(self.prob.heads)
+        forward_host(self.prob, q_host, k_host, v_host, out, self.device_buffers(), hg,
+                     self.status, stream)
+        return out
+
     def check_status(self):
         v = int(self.status.item())
         if v:
@@ -254,4 +311,5 @@ class BlockSparseAttention:
 
 __all__ = ["Problem", "Sizes", "BSAError", "BlockSparseAttention", "lib", "keep_count",
            "query_sizes", "layout", "permute", "pool", "select_topk", "sparse_attn_fwd",
-           "dense_attn_fwd", "unpermute", "layout_stats", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]
+           "dense_attn_fwd", "unpermute", "layout_stats", "forward_host", "DeviceBuffers",
+           "default_heads_per_group", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]

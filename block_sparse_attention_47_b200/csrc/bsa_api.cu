@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "bsa_internal.cuh"
 
@@ -116,6 +117,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bsa_status check_ptr(const void* p, const char* name) {
   if (!p) return fail(BSA_ERR_INVALID_ARG, "%s is NULL", name);
   if (!aligned16(p)) return fail(BSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return BSA_OK;
+}
+
+// index lists and counts are read and written as single int32 words
+bsa_status check_ptr4(const void* p, const char* name) {
+  if (!p) return fail(BSA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) & 3u)
+    return fail(BSA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);
   return BSA_OK;
 }
 
@@ -276,8 +285,8 @@ bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const f
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(q_pool, "q_pool"));
   BSA_TRY(check_ptr(k_pool, "k_pool"));
-  BSA_TRY(check_ptr(idx, "idx"));
-  BSA_TRY(check_ptr(cnt, "cnt"));
+  BSA_TRY(check_ptr4(idx, "idx"));
+  BSA_TRY(check_ptr4(cnt, "cnt"));
   BSA_TRY(check_device());
   cudaError_t e = bsa::launch_select(g, q_pool, k_pool, idx, cnt, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_select_topk launch");
@@ -296,8 +305,8 @@ static bsa_status attention_common(const bsa_problem* prob, const void* layout_b
   BSA_TRY(check_ptr(v_perm, "v_perm"));
   BSA_TRY(check_ptr(o_perm, "o_perm"));
   if (!dense) {
-    BSA_TRY(check_ptr(idx, "idx"));
-    BSA_TRY(check_ptr(cnt, "cnt"));
+    BSA_TRY(check_ptr4(idx, "idx"));
+    BSA_TRY(check_ptr4(cnt, "cnt"));
   }
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
     return fail(BSA_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
@@ -348,6 +357,169 @@ bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const 
                                         static_cast<__nv_bfloat16*>(o_raster), stride_b,
                                         stride_n, stride_h, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_unpermute launch");
+}
+
+// ---- whole call from host memory -------------------------------------------
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_copy_mutex;
+cudaStream_t g_copy_in[kMaxDevices], g_copy_out[kMaxDevices];
+
+// the two copy streams of the current device, created on first use
+bsa_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BSA_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(g_copy_mutex);
+  if (!g_copy_in[dev]) {
+    e = cudaStreamCreateWithFlags(&g_copy_in[dev], cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&g_copy_out[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
+  }
+  *in = g_copy_in[dev];
+  *out = g_copy_out[dev];
+  return BSA_OK;
+}
+
+// events of one call, destroyed on every exit (pending work keeps them alive)
+struct EventSet {
+  std::vector<cudaEvent_t> ev;
+  ~EventSet() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+  }
+  cudaError_t make(size_t n) {
+    ev.reserve(n);
+    for (size_t i = 0; i < n; ++i) {
+      cudaEvent_t e;
+      cudaError_t r = cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+      if (r != cudaSuccess) return r;
+      ev.push_back(e);
+    }
+    return cudaSuccess;
+  }
+};
+
+}  // namespace
+
+bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const void* k_host,
+                            const void* v_host, void* o_host, const bsa_device_buffers* buf,
+                            int32_t heads_per_group, int32_t* dev_status, void* stream) {
+  g_last_error[0] = 0;
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  if (!q_host || !k_host || !v_host || !o_host)
+    return fail(BSA_ERR_INVALID_ARG, "a host tensor pointer is NULL");
+  if (!buf) return fail(BSA_ERR_INVALID_ARG, "buf is NULL");
+  const void* dev_ptrs[] = {buf->q_raster, buf->k_raster, buf->v_raster, buf->o_raster,
+                            buf->q_perm,   buf->k_perm,   buf->v_perm,   buf->o_perm,
+                            buf->layout_buf, buf->q_pool, buf->k_pool,   buf->idx,
+                            buf->cnt};
+  const char* dev_names[] = {"q_raster", "k_raster", "v_raster", "o_raster", "q_perm",
+                             "k_perm",   "v_perm",   "o_perm",   "layout_buf", "q_pool",
+                             "k_pool",   "idx",      "cnt"};
+  for (int i = 0; i < 11; ++i) BSA_TRY(check_ptr(dev_ptrs[i], dev_names[i]));
+  BSA_TRY(check_ptr4(buf->idx, "idx"));
+  BSA_TRY(check_ptr4(buf->cnt, "cnt"));
+  if (heads_per_group < 1 || heads_per_group > g.h || g.h % heads_per_group != 0)
+    return fail(BSA_ERR_INVALID_ARG, "heads_per_group %d must divide heads (%d)", heads_per_group,
+                g.h);
+  BSA_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream), s_in, s_out;
+  BSA_TRY(copy_streams(&s_in, &s_out));
+
+  const int groups = g.h / heads_per_group;
+  bsa_problem sub = *prob;
+  sub.heads = heads_per_group;
+  Geo gs;
+  BSA_TRY(make_geo(&sub, &gs));
+  // raster [B, N, heads, d]: a head group is a strided slab of every token row
+  const int64_t sn = int64_t(g.h) * g.d, sb = int64_t(g.N) * sn, sh = g.d;
+  const size_t pitch = size_t(sn) * 2, width = size_t(heads_per_group) * g.d * 2;
+  const size_t rows = size_t(g.B) * g.N;
+  const size_t perm_elems = size_t(g.B) * heads_per_group * g.N * g.d;   // per group
+  const size_t pool_elems = size_t(g.B) * heads_per_group * g.nb * g.d;
+  const size_t idx_elems = size_t(g.B) * heads_per_group * g.nb * g.kcap;
+  const size_t cnt_elems = size_t(g.B) * heads_per_group * g.nb;
+  const bool dynamic = g.mode == BSA_BLOCK_DYNAMIC_888;
+
+  EventSet es;  // start, k, in[groups], out[groups], done
+  cudaError_t e = es.make(3 + 2 * size_t(groups));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags");
+  cudaEvent_t ev_start = es.ev[0], ev_k = es.ev[1], ev_done = es.ev[2 + 2 * groups];
+  auto ev_in = [&](int i) { return es.ev[2 + i]; };
+  auto ev_out = [&](int i) { return es.ev[2 + groups + i]; };
+  auto slab = [&](const void* base, int grp) {
+    return static_cast<const char*>(base) + size_t(grp) * width;
+  };
+#define BSA_CUDA(call, what)                 \
+  do {                                       \
+    cudaError_t e_ = (call);                 \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+  // the copy streams start after the work already queued on the caller's stream
+  BSA_CUDA(cudaEventRecord(ev_start, st), "cudaEventRecord");
+  BSA_CUDA(cudaStreamWaitEvent(s_in, ev_start, 0), "cudaStreamWaitEvent");
+  BSA_CUDA(cudaStreamWaitEvent(s_out, ev_start, 0), "cudaStreamWaitEvent");
+
+  // the dynamic layout looks at every head of K: copy K whole first
+  if (dynamic) {
+    BSA_CUDA(cudaMemcpyAsync(buf->k_raster, k_host, rows * pitch, cudaMemcpyHostToDevice, s_in),
+             "cudaMemcpyAsync K");
+    BSA_CUDA(cudaEventRecord(ev_k, s_in), "cudaEventRecord");
+    BSA_CUDA(cudaStreamWaitEvent(st, ev_k, 0), "cudaStreamWaitEvent");
+  }
+  BSA_TRY(bsa_layout(prob, buf->k_raster, sb, sn, sh, buf->layout_buf, st));
+
+  // uploads: every group's slabs, in order, on the input stream
+  for (int i = 0; i < groups; ++i) {
+    const void* hosts[3] = {q_host, k_host, v_host};
+    void* devs[3] = {buf->q_raster, buf->k_raster, buf->v_raster};
+    for (int t = 0; t < 3; ++t) {
+      if (t == 1 && dynamic) continue;
+      BSA_CUDA(cudaMemcpy2DAsync(const_cast<char*>(slab(devs[t], i)), pitch, slab(hosts[t], i),
+                                 pitch, width, rows, cudaMemcpyHostToDevice, s_in),
+               "cudaMemcpy2DAsync upload");
+    }
+    BSA_CUDA(cudaEventRecord(ev_in(i), s_in), "cudaEventRecord");
+  }
+  // computation of each group once its slabs have landed
+  for (int i = 0; i < groups; ++i) {
+    BSA_CUDA(cudaStreamWaitEvent(st, ev_in(i), 0), "cudaStreamWaitEvent");
+    const int64_t h0 = int64_t(i) * heads_per_group * g.d;  // element offset of the slab
+    auto rq = static_cast<const __nv_bfloat16*>(buf->q_raster) + h0;
+    auto rk = static_cast<const __nv_bfloat16*>(buf->k_raster) + h0;
+    auto rv = static_cast<const __nv_bfloat16*>(buf->v_raster) + h0;
+    auto ro = static_cast<__nv_bfloat16*>(buf->o_raster) + h0;
+    auto pq = static_cast<__nv_bfloat16*>(buf->q_perm) + i * perm_elems;
+    auto pk = static_cast<__nv_bfloat16*>(buf->k_perm) + i * perm_elems;
+    auto pv = static_cast<__nv_bfloat16*>(buf->v_perm) + i * perm_elems;
+    auto po = static_cast<__nv_bfloat16*>(buf->o_perm) + i * perm_elems;
+    float* qpool = buf->q_pool + i * pool_elems;
+    float* kpool = buf->k_pool + i * pool_elems;
+    int32_t* idx = buf->idx + i * idx_elems;
+    int32_t* cnt = buf->cnt + i * cnt_elems;
+    BSA_TRY(bsa_permute(&sub, buf->layout_buf, rq, sb, sn, sh, pq, st));
+    BSA_TRY(bsa_permute(&sub, buf->layout_buf, rk, sb, sn, sh, pk, st));
+    BSA_TRY(bsa_permute(&sub, buf->layout_buf, rv, sb, sn, sh, pv, st));
+    BSA_TRY(bsa_pool(&sub, buf->layout_buf, pq, pk, qpool, kpool, st));
+    BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
+    BSA_TRY(bsa_sparse_attn_fwd(&sub, buf->layout_buf, pq, pk, pv, idx, cnt, po, dev_status, st));
+    BSA_TRY(bsa_unpermute(&sub, buf->layout_buf, po, ro, sb, sn, sh, st));
+    BSA_CUDA(cudaEventRecord(ev_out(i), st), "cudaEventRecord");
+  }
+  // downloads on the output stream; the caller's stream ends with the last one
+  for (int i = 0; i < groups; ++i) {
+    BSA_CUDA(cudaStreamWaitEvent(s_out, ev_out(i), 0), "cudaStreamWaitEvent");
+    BSA_CUDA(cudaMemcpy2DAsync(const_cast<char*>(slab(o_host, i)), pitch, slab(buf->o_raster, i),
+                               pitch, width, rows, cudaMemcpyDeviceToHost, s_out),
+             "cudaMemcpy2DAsync download");
+  }
+  BSA_CUDA(cudaEventRecord(ev_done, s_out), "cudaEventRecord");
+  BSA_CUDA(cudaStreamWaitEvent(st, ev_done, 0), "cudaStreamWaitEvent");
+#undef BSA_CUDA
+  return BSA_OK;
 }
 
 bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int64_t hist7[7],

@@ -27,8 +27,9 @@
  * Conventions (every entry point):
  *   - The caller owns all memory.  The library allocates no device memory;
  *     sizes of every buffer come from bsa_query_sizes.
- *   - Device pointers must be 16-byte aligned; the innermost (head_dim)
- *     dimension of every tensor is contiguous.
+ *   - Device pointers must be 16-byte aligned (index lists and counts: 4
+ *     bytes); the innermost (head_dim) dimension of every tensor is
+ *     contiguous.
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
  *     void*; NULL = legacy default stream).  Arguments are validated on the
  *     host before anything is launched: on any error nothing is launched and
@@ -185,6 +186,49 @@ bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const 
  * to the host.  Fixed mode: hist7[0] = B * n_video_blocks, no CUDA call. */
 bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int64_t hist7[7],
                             void* stream);
+
+/* Device buffers of one whole call (caller-owned, sizes from
+ * bsa_query_sizes): raster Q, K, V, O (raster_tensor_bytes each, contiguous
+ * [B, N, heads, head_dim]), permuted Q, K, V, O (perm_tensor_bytes each),
+ * the layout (layout_bytes), pooled Q and K (pool_bytes each), index lists
+ * (idx_bytes) and counts (cnt_bytes).  16-byte aligned (idx and cnt: 4). */
+typedef struct bsa_device_buffers {
+  void* q_raster;
+  void* k_raster;
+  void* v_raster;
+  void* o_raster;
+  void* q_perm;
+  void* k_perm;
+  void* v_perm;
+  void* o_perm;
+  void* layout_buf;
+  float* q_pool;
+  float* k_pool;
+  int32_t* idx;
+  int32_t* cnt;
+} bsa_device_buffers;
+
+/* The whole call (layout, permute, pool, top-k selection, sparse attention,
+ * unpermute: the sequence above) for Q, K, V and O in HOST memory, with the
+ * transfers overlapped with the computation.  Heads are processed in groups
+ * of `heads_per_group`.  Group g+1 is copied to the device while group g is
+ * computed and group g-1's output is copied back, on two library-owned
+ * copy streams tied to `stream` by events.  The dynamic layout needs every
+ * head of K, so in dynamic mode K is copied whole first.
+ *   q_host, k_host, v_host  [B, N, heads, head_dim] bf16, contiguous, host
+ *                           memory (page-locked memory lets copies overlap)
+ *   o_host                  same layout, written; pad tokens are 0
+ *   buf                     device buffers as described above
+ *   heads_per_group         1..heads, must divide heads
+ *   dev_status, stream      as in bsa_sparse_attn_fwd; the call is complete
+ *                           when the work queued on `stream` is complete.
+ * Results equal the step-by-step sequence up to the order of the attention
+ * kernel's fp32 accumulation (a group's CTAs start their key walks at
+ * different blocks).  The library creates its two copy streams per device
+ * on first use and keeps them; it allocates no memory. */
+bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const void* k_host,
+                            const void* v_host, void* o_host, const bsa_device_buffers* buf,
+                            int32_t heads_per_group, int32_t* dev_status, void* stream);
 
 /* Name of a status code. */
 const char* bsa_status_string(bsa_status status);

@@ -31,7 +31,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol():
     names = declared_functions()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(bsa.lib(), n), n
     assert set(names) == set(bsa._SIGS), "binding and header disagree"
@@ -85,6 +85,7 @@ BAD_PROBLEMS = [
     (dict(block_mode=2), 1), (dict(block_mode=1, W=12), 2), (dict(block_mode=1, H_valid=14), 2),
     (dict(block_mode=1, dyn_tau=float("nan")), 1), (dict(block_mode=1, dyn_tau=0.5), 1),
     (dict(softmax_scale=0.0), 1), (dict(softmax_scale=float("inf")), 1),
+    (dict(prefix=(8192 * 64,)), 3),  # 8,224 blocks: more than the attention kernel walks
     (dict(prefix=(0,)), 2),
 ]
 
@@ -140,3 +141,44 @@ def test_valid_call_without_gpu_reports_cuda_error():
     assert rc == 5
     with pytest.raises(bsa.BSAError):
         bsa._check(rc)
+
+
+def host_buffers(**bad):
+    b = bsa.DeviceBuffers()
+    for name, _ in bsa.DeviceBuffers._fields_:
+        setattr(b, name, 16)
+    for name, v in bad.items():
+        setattr(b, name, v)
+    return b
+
+
+def test_forward_host_validation():
+    """bsa_forward_host rejects bad arguments before touching the device."""
+    p = base()
+    L = bsa.lib()
+    P = ctypes.byref(p)
+    ok = host_buffers()
+    assert L.bsa_forward_host(P, None, 16, 16, 16, ctypes.byref(ok), 1, None, None) == 1
+    assert b"host" in L.bsa_last_error()
+    assert L.bsa_forward_host(P, 16, 16, 16, 16, None, 1, None, None) == 1
+    assert L.bsa_forward_host(P, 16, 16, 16, 16, ctypes.byref(host_buffers(v_perm=24)), 1,
+                              None, None) == 1
+    assert b"v_perm" in L.bsa_last_error()
+    assert L.bsa_forward_host(P, 16, 16, 16, 16, ctypes.byref(host_buffers(idx=18)), 1,
+                              None, None) == 1
+    assert b"idx" in L.bsa_last_error()
+    for hg in (0, -1, p.heads + 1):
+        assert L.bsa_forward_host(P, 16, 16, 16, 16, ctypes.byref(ok), hg, None, None) == 1
+    if p.heads > 1:
+        assert L.bsa_forward_host(P, 16, 16, 16, 16, ctypes.byref(ok), p.heads + 1, None,
+                                  None) == 1
+
+
+def test_forward_host_int32_lists_need_4_byte_alignment_only():
+    # idx/cnt at 4-byte (not 16-byte) boundaries pass validation; without a
+    # GPU the call then stops at the device check
+    p = base()
+    L = bsa.lib()
+    b = host_buffers(idx=20, cnt=36)
+    st = L.bsa_forward_host(ctypes.byref(p), 16, 16, 16, 16, ctypes.byref(b), 1, None, None)
+    assert st == 5, L.bsa_last_error()

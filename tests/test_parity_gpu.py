@@ -258,3 +258,38 @@ def test_rescale_path_growing_logits(name):
     assert_close(got.transpose(0, 2, 1, 3)[keep_rows], want.transpose(0, 2, 1, 3)[keep_rows],
                  name + " growing logits")
     assert int(run.attn.status.item()) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "dyn"])
+def test_host_call_pipelined_by_head_groups(name):
+    """bsa_forward_host on pinned host tensors, one head per group (so every
+    case runs several groups; the dynamic case copies K whole first): same
+    oracle bar as the device path."""
+    cfg = SMALL[name]
+    (q, k, v), (qn, kn, vn) = seeded_inputs(cfg, seed=4242)
+    run = GpuRun(cfg, q, k, v)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    out = run.attn.host_call(qh, kh, vh, heads_per_group=1)
+    torch.cuda.synchronize()
+    run.attn.check_status()
+    assert not out.is_cuda
+    geo = O.Geometry(cfg)
+    want, _, _, lists = O.forward(cfg, qn, kn, vn)
+    # one head per group: group hh's lists fill slot hh of the buffers as [B, nb, ...]
+    idx = run.attn.idx.cpu().numpy().reshape(geo.h, geo.B, geo.nb, -1)
+    cnt = run.attn.cnt.cpu().numpy().reshape(geo.h, geo.B, geo.nb)
+    lay = O.layout(cfg, kn)
+    keep_rows = np.ones((geo.B, geo.h, geo.N), dtype=bool)
+    for b in range(geo.B):
+        perm = lay[b][0]
+        for hh in range(geo.h):
+            for i in range(geo.nbp, geo.nb):
+                if list(idx[hh, b, i, :cnt[hh, b, i]]) != list(lists[b][hh][i]):
+                    keep_rows[b, hh, perm[i * 64:(i + 1) * 64]] = False
+    assert keep_rows.mean() > 0.99
+    got = to_np64(out)
+    assert_close(got.transpose(0, 2, 1, 3)[keep_rows], want.transpose(0, 2, 1, 3)[keep_rows],
+                 name + " host path")
+    assert not got[:, ~geo.token_valid()].any(), "pad tokens must come out as 0"
+    dev = to_np64(run.out)
+    assert np.abs(got - dev).max() <= 3e-2
