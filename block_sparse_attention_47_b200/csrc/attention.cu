@@ -32,10 +32,11 @@
 // 2^8), which is still exact after the final division.
 //
 // The step sequence is fixed before the walk starts: warp 8 turns the two
-// index lists into two bitmaps over the key blocks (one bit per kept block),
-// and every role walks the union A|B with a private cursor, so no role waits
-// for another to hand it the next key block.  The walk visits 32-block words
-// in a rotated order and the set bits of a word in ascending order.
+// index lists into bitmaps over the key blocks (one bit per kept block) and
+// expands their union A|B into a table of 16-bit step entries in shared
+// memory (key block and flags), 32-block words in a rotated order and bits
+// ascending within a word.  Every role reads step j straight from the table,
+// so no role waits for another to hand it the next key block.
 //
 // Warp roles (512 threads):
 //   warps 0-3 / 4-7  softmax warpgroup 0 / 1; thread r of a group owns
@@ -65,6 +66,10 @@ namespace bsa {
 namespace {
 
 constexpr int kMaxWords = kAttnMaxBlocks / 32;  // step-bitmap words per query block
+// step table entry: key block in bits 0-12, then the first query block keeps
+// it (bit 13), the second one does (bit 14), all 64 slots are real tokens (15)
+constexpr uint32_t kTileMask = 0x1FFFu, kFlagShift = 13;
+static_assert(kAttnMaxBlocks <= 8192, "13-bit key block in a step entry");
 
 template <int D>
 struct Cfg {
@@ -83,49 +88,11 @@ struct Cfg {
   static constexpr int N_BARS = 2 * KS + 2 * VS + 12;
   static constexpr int OFF_XCH = OFF_BAR + 8 * N_BARS;  // float m[2][128], l[2][128]
   static constexpr int OFF_BM = OFF_XCH + 4 * 4 * 128;   // uint32 A, B, F [kMaxWords]
-  static constexpr int OFF_MISC = OFF_BM + 3 * 4 * kMaxWords;
+  static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;  // uint16 [kAttnMaxBlocks]
+  static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(KS % 2 == 0, "step pairs must not straddle the K ring's end");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
-};
-
-// Cursor over the step sequence: the set bits of A|B, words visited in the
-// rotated order ws, ws+1, .., nw-1, 0, .., ws-1 (CTAs working on the same
-// head start at different words, so they do not all fetch the same K/V
-// tiles at the same moment; the online softmax does not depend on the
-// order of its steps) and bits within a word in ascending order.  next()
-// returns the key block of the next step and its flags (bit 0: the first
-// query block keeps it, bit 1: the second one, bit 2: all 64 slots of the
-// key block are real tokens), or -1 past the last word.
-struct StepCursor {
-  int w;              // current word
-  uint32_t cur = 0u;  // union bits of the current word not handed out yet
-  __device__ explicit StepCursor(int ws) : w(ws - 1) {}
-  // A = first query block's bitmap; B = A + kMaxWords, F (full key blocks)
-  // = A + 2 * kMaxWords.  Reaching a word with a set bit takes at most nw
-  // word loads, so a walk past the last step ends with -1 instead of looping.
-  __device__ int next(const uint32_t* A, int nw, uint32_t& flags) {
-    for (int guard = 0; cur == 0u; ++guard) {
-      if (guard >= nw) return -1;
-      w = w + 1 == nw ? 0 : w + 1;
-      cur = A[w] | A[kMaxWords + w];
-    }
-    const int bit = __ffs(cur) - 1;
-    cur &= cur - 1u;
-    flags = ((A[w] >> bit) & 1u) | (((A[kMaxWords + w] >> bit) & 1u) << 1) |
-            (((A[2 * kMaxWords + w] >> bit) & 1u) << 2);
-    return w * 32 + bit;
-  }
-  __device__ int next(const uint32_t* A, int nw) {
-    for (int guard = 0; cur == 0u; ++guard) {
-      if (guard >= nw) return -1;
-      w = w + 1 == nw ? 0 : w + 1;
-      cur = A[w] | A[kMaxWords + w];
-    }
-    const int bit = __ffs(cur) - 1;
-    cur &= cur - 1u;
-    return w * 32 + bit;
-  }
 };
 
 __device__ __forceinline__ void report_timeout(volatile int* abort_flag, int32_t* status) {
@@ -166,6 +133,7 @@ __global__ void __launch_bounds__(512, 1)
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);  // first query block's keys
   uint32_t* bmB = bmA + kMaxWords;                                 // second query block's keys
   uint32_t* bmF = bmA + 2 * kMaxWords;                             // key blocks with no pad slot
+  uint16_t* steps = reinterpret_cast<uint16_t*>(sm + C::OFF_STEPS);  // the walk, in order
   float* xch = reinterpret_cast<float*>(sm + C::OFF_XCH);  // m[2][128] then l[2][128]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
@@ -256,12 +224,36 @@ __global__ void __launch_bounds__(512, 1)
         bmF[w] = f;
       }
       __syncwarp();
-      int cntw = 0;
-      for (int w = lane; w < nw; w += 32) cntw += __popc(bmA[w] | bmB[w]);
-      cntw = __reduce_add_sync(0xffffffffu, cntw);
-      if (lane == 0) *n_steps_sm = cntw;
+      // the step table: set bits of A|B, words in the rotated order ws, ws+1,
+      // .., nw-1, 0, .., ws-1 and bits ascending within a word; lane l takes
+      // word l of each round of 32 and writes at its prefix-sum offset
+      int nsteps = 0;
+      for (int r0 = 0; r0 < nw; r0 += 32) {
+        const int pos = r0 + lane;
+        const int w = pos < nw ? (ws + pos < nw ? ws + pos : ws + pos - nw) : 0;
+        const uint32_t a = pos < nw ? bmA[w] : 0u, bb = pos < nw ? bmB[w] : 0u;
+        const uint32_t f = pos < nw ? bmF[w] : 0u;
+        uint32_t u = a | bb;
+        const int c = __popc(u);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int at = nsteps + incl - c;
+        while (u) {
+          const int bit = __ffs(u) - 1;
+          u &= u - 1u;
+          steps[at++] = uint16_t(uint32_t(32 * w + bit) | (((a >> bit) & 1u) << kFlagShift) |
+                                 (((bb >> bit) & 1u) << (kFlagShift + 1)) |
+                                 (((f >> bit) & 1u) << (kFlagShift + 2)));
+        }
+        nsteps += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) *n_steps_sm = nsteps;
       __syncwarp();
-      mbar_arrive(bar_steps);  // release: every lane's bitmap writes
+      mbar_arrive(bar_steps);  // release: every lane's table writes
     }
     // ---------------------------------------------- K box 0 / box 1, V copies
     // K: one warp per (box, step parity); a K stage is only ever reused by
@@ -281,8 +273,6 @@ __global__ void __launch_bounds__(512, 1)
       const int RS = is_k ? KS : VS;
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
       const int n = ok ? *n_steps_sm : 0;
-      StepCursor sc(ws);
-      if (par == 1 && n > 0) sc.next(bmA, nw);  // step 0 belongs to the other parity
       int j = par;
       for (; ok && j < n; j += stride) {
         const int s = j % RS;
@@ -292,12 +282,7 @@ __global__ void __launch_bounds__(512, 1)
           ok = false;
           break;
         }
-        const int t = sc.next(bmA, nw);
-        if (t < 0) {  // the bitmaps hold fewer steps than counted: cannot happen
-          ok = false;
-          break;
-        }
-        if (stride == 2 && j + 1 < n) sc.next(bmA, nw);  // skip the other parity's step
+        const int t = int(steps[j] & kTileMask);
         // box bx of the block: [box][row][64] in the stage
         mbar_arrive_expect_tx(ful, C::BOX);
         if (is_k)
@@ -423,28 +408,27 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = g.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l_sum = 0.f;
     int k = 0;  // steps of this group so far
-    // this group's steps are every other step of the cursor walk; the flags
-    // and the valid-slot mask of a step are fetched one step ahead
+    // this group's steps are every other entry of the step table.  Barrier
+    // probes are issued ahead of independent work so that their latency
+    // (~170 cycles even for a completed phase) overlaps it.
     ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
     const int n = ok ? *n_steps_sm : 0;
     const uint64_t* bm_row = bmask + int64_t(b) * g.nb;
-    StepCursor sc(ws);
-    if (wg == 1 && n > 0) sc.next(bmA, nw);  // step 0 belongs to group 0
     for (int j = wg; ok && j < n; j += 2, ++k) {
-      uint32_t flags;
-      const int tile = sc.next(bmA, nw, flags);
-      if (tile < 0) {
-        ok = false;
-        break;
-      }
-      if (j + 1 < n) sc.next(bmA, nw);  // the other group's step
+      const bool s_ready = __all_sync(0xffffffffu, mbar_test(bar_s, k & 1));
+      const uint32_t entry = steps[j];
+      const int tile = int(entry & kTileMask);
+      const uint32_t flags = entry >> kFlagShift;
       const bool member = (flags >> half) & 1u;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s, k & 1, abort_flag));
-      if (!ok) break;
+      if (!s_ready) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_s, k & 1, abort_flag));
+        if (!ok) break;
+      }
       tc_fence_after();
       uint32_t pk[32];
       float factor = 1.f;
       bool rescale = false;
+      bool o_ready = k == 0;
       if (member) {
         uint32_t r[64];
         BSA_TMEM_LD64(tS, r);
@@ -464,6 +448,9 @@ __global__ void __launch_bounds__(512, 1)
           for (int c = 0; c < 64; ++c)
             if (bit_of(lo, hi, c)) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
         }
+        // the previous PV has normally finished by now: probe it here, use
+        // the answer after the exponentials
+        o_ready = k == 0 || __all_sync(0xffffffffu, mbar_test(bar_o + 8 * wg, (k - 1) & 1));
         const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
         if (mxs > m_used + 8.f) {
           if (m_used != -INFINITY) {
@@ -506,7 +493,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
       // P and O of this group are free once its previous PV has finished
-      if (k > 0) {
+      if (!o_ready) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o + 8 * wg, (k - 1) & 1, abort_flag));
         if (!ok) break;
       }

@@ -13,8 +13,9 @@
 namespace bsa {
 
 constexpr int kBlock = 64;       // tokens per block
-// blocks per sequence the attention kernel walks with on-chip step bitmaps
-constexpr int kAttnMaxBlocks = 8192;
+// blocks per sequence the attention kernel's on-chip step table can hold
+// (16-bit entries: a 13-bit key block and 3 flags)
+constexpr int kAttnMaxBlocks = 6144;
 
 // Everything a kernel needs to know about a problem (plain integers).
 struct Geo {

@@ -64,7 +64,10 @@ typedef enum {
   BSA_OK = 0,
   BSA_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad scalar */
   BSA_ERR_SHAPE = 2,       /* grid, block or prefix geometry not allowed */
-  BSA_ERR_UNSUPPORTED = 3, /* head_dim other than 64 or 128, no sm_100 GPU */
+  BSA_ERR_UNSUPPORTED = 3, /* head_dim other than 64 or 128, more than 6,144
+                              64-token blocks per sequence (the attention
+                              kernel's on-chip step table), more video blocks
+                              than on-chip selection holds, no sm_100 GPU */
   BSA_ERR_WORKSPACE = 4,   /* a caller buffer is too small */
   BSA_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
   BSA_ERR_TIMEOUT = 6      /* device-side bounded wait ran out */
