@@ -112,6 +112,7 @@ _SIGS = {
     "bsa_layout_stats": (ctypes.c_int, [ctypes.POINTER(Problem), _P, ctypes.POINTER(_I64), _P]),
     "bsa_forward_host": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P,
                                         ctypes.POINTER(DeviceBuffers), ctypes.c_int32, _P, _P]),
+    "bsa_debug_stall_pv": (ctypes.c_int, [ctypes.c_int32]),
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_last_error": (ctypes.c_char_p, []),
 }
@@ -225,6 +226,12 @@ def default_heads_per_group(heads, groups=32):
     return heads
 
 
+def debug_stall_pv(enable):
+    """Test hook: while enabled, attention launches issue no PV, so their
+    bounded wait runs out and BSA_ERR_TIMEOUT reaches the status word."""
+    _check(lib().bsa_debug_stall_pv(1 if enable else 0))
+
+
 def layout_stats(prob, layout_buf, stream=None):
     hist = (_I64 * 7)()
     _check(lib().bsa_layout_stats(ctypes.byref(prob), _ptr(layout_buf), hist, _stream(stream)))
@@ -312,4 +319,4 @@ class BlockSparseAttention:
 __all__ = ["Problem", "Sizes", "BSAError", "BlockSparseAttention", "lib", "keep_count",
            "query_sizes", "layout", "permute", "pool", "select_topk", "sparse_attn_fwd",
            "dense_attn_fwd", "unpermute", "layout_stats", "forward_host", "DeviceBuffers",
-           "default_heads_per_group", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]
+           "default_heads_per_group", "debug_stall_pv", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]

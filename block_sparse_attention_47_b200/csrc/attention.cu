@@ -292,7 +292,9 @@ __global__ void __launch_bounds__(512, 1)
       }
       if (!ok) {
         report_timeout(abort_flag, status);
-        for (int jj = j - stride; jj >= 0 && jj >= j - stride * RS; jj -= stride)
+        // this warp's copies that may still be in flight: its last uses of
+        // the ring (RS steps back: 4 stages of one parity for K, 5 for V)
+        for (int jj = j - stride; jj >= 0 && jj >= j - RS; jj -= stride)
           mbar_wait(ful_of(is_k, jj % RS), (jj / RS) & 1, nullptr, 200000000ull);
       }
     }
@@ -342,7 +344,9 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
-      const int n = ok ? *n_steps_sm : 0;
+      // test hook: with stall_pv set no PV is issued, so the softmax's wait
+      // on the first PV runs out and the kernel takes its timeout path
+      const int n = ok && !g.stall_pv ? *n_steps_sm : 0;
       for (int j = 0; ok && j < n; ++j) {
         const int w = j & 1, s = j % VS;
         ok = mbar_wait(vfull(s), (j / VS) & 1, abort_flag) &&

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -34,6 +35,9 @@ bsa_status cuda_fail(cudaError_t e, const char* what) {
 
 // library-owned fallback status word for callers that pass dev_status = NULL
 __device__ int32_t g_dev_status_sink;
+
+// test hook (bsa_debug_stall_pv): attention launches while set issue no PV
+std::atomic<int> g_stall_pv{0};
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
@@ -103,6 +107,7 @@ bsa_status make_geo(const bsa_problem* p, Geo* g) {
   g->nreg = p->block_mode == BSA_BLOCK_DYNAMIC_888 ? (p->T / 8) * (p->H / 8) * (p->W / 8) : 0;
   g->tau = p->dyn_tau;
   g->scale = p->softmax_scale;
+  g->stall_pv = 0;
   if (int64_t(p->B) * p->heads > 65535) return fail(BSA_ERR_SHAPE, "B*heads must be <= 65535");
   if (g->nb > bsa::kAttnMaxBlocks)
     return fail(BSA_ERR_UNSUPPORTED, "%d blocks per sequence; the attention kernel walks at most %d",
@@ -319,6 +324,7 @@ static bsa_status attention_common(const bsa_problem* prob, const void* layout_b
     cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dev_status_sink);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status sink)");
   }
+  g.stall_pv = g_stall_pv.load();
   cudaError_t e = bsa::launch_attention(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
                                         maps, static_cast<const __nv_bfloat16*>(q_perm), idx,
                                         cnt, static_cast<__nv_bfloat16*>(o_perm),
@@ -519,6 +525,12 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
   BSA_CUDA(cudaEventRecord(ev_done, s_out), "cudaEventRecord");
   BSA_CUDA(cudaStreamWaitEvent(st, ev_done, 0), "cudaStreamWaitEvent");
 #undef BSA_CUDA
+  return BSA_OK;
+}
+
+bsa_status bsa_debug_stall_pv(int32_t enable) {
+  g_last_error[0] = 0;
+  g_stall_pv.store(enable ? 1 : 0);
   return BSA_OK;
 }
 

@@ -30,6 +30,7 @@ struct Geo {
   int mode;
   int nreg;   // dynamic regions per batch element (0 in fixed mode)
   float tau, scale;
+  int stall_pv;  // test hook: the attention kernel issues no PV (see bsa_debug_stall_pv)
 };
 
 // Byte offsets of the sections of the layout buffer (each 256-B aligned).

@@ -233,6 +233,14 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
                             const void* v_host, void* o_host, const bsa_device_buffers* buf,
                             int32_t heads_per_group, int32_t* dev_status, void* stream);
 
+/* Test hook for the device-side timeout path.  While enabled (nonzero),
+ * attention launches issue no PV product, so the softmax's bounded wait on
+ * the first PV runs out after 2 s.  The kernel then writes BSA_ERR_TIMEOUT
+ * to the status word, drains its copies and MMAs, frees tensor memory and
+ * returns, and the CUDA context stays usable.  Output is undefined for
+ * launches made while enabled.  Process-wide; off by default. */
+bsa_status bsa_debug_stall_pv(int32_t enable);
+
 /* Name of a status code. */
 const char* bsa_status_string(bsa_status status);
 /* Message of the last failed call on this thread ("" if none). */
