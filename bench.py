@@ -43,12 +43,12 @@ from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per sparse-attention launch from one ncu capture
-# (profiles/attn_fwd_720p_b1h4.md: 1.574 GB read + 0.125 GB written for B=1 x
+# (profiles/attn_fwd_720p_b1h4.md: 1.882 GB read + 0.125 GB written for B=1 x
 # 4 heads, scaled by the number of (batch, head) problems).  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
 # workload; null otherwise.
-ATTN_TRAFFIC = {"sha256": "df92b22af651629c19fedccd37e33732d29faeb35c8049c8e35bc21477460042",
-                "bytes_per_bh": 1.699188e9 / 4, "workload": ("720p", 0.25, 0)}
+ATTN_TRAFFIC = {"sha256": "4dcab2ba544f24533df192df6f096d1ed7264fc945c5893a47fe1e0e4ecbc7bf",
+                "bytes_per_bh": 2.006707e9 / 4, "workload": ("720p", 0.25, 0)}
 
 
 def attn_traffic(cfg, keep_ratio):
