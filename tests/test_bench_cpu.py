@@ -1,0 +1,60 @@
+"""The benchmark's accounting on the host: kept-tile counts and FLOPs for
+every workload against hand-derived totals, the weak-scaling aggregate, and
+when the stored ncu traffic figure applies."""
+import os
+import sys
+
+import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+from gen import config, derived_sizes  # noqa: E402
+import block_sparse_attention_47_b200 as bsa  # noqa: E402
+
+
+def keep_of(cfg):
+    # the library's closed form; the oracle pins cover the same function
+    return bsa.keep_count(derived_sizes(cfg)["nbv"], cfg["keep_ratio"])
+
+
+@pytest.mark.parametrize("name,over,tiles", [
+    # video query blocks x (prefix blocks + keep) + prefix query blocks x all blocks
+    ("tiny", {}, 1 * 2 * 32 * 8),                              # 512
+    ("lowres", {}, 24 * 504 * 126),                            # 1,524,096
+    ("720p", {}, 2 * 24 * 1920 * 480),                         # 44,236,800
+    ("720p", {"keep_ratio": 0.0625}, 2 * 24 * 1920 * 120),     # 11,059,200
+    ("ref_prefix", {}, 24 * (2016 * (44 + 504) + 44 * 2060)),  # 28,689,792
+    ("sweep", {"keep_ratio": 0.01}, 24 * 1440 * 15),           # 34,560 * 15
+])
+def test_kept_tiles(name, over, tiles):
+    cfg = config(name, **over)
+    assert bench.kept_tiles(cfg, keep_of(cfg)) == tiles
+
+
+def test_tile_flops_and_720p_total():
+    cfg = config("720p")
+    assert bench.tile_flops(cfg) == 4 * 64 * 64 * 128 == 2_097_152
+    total = bench.kept_tiles(cfg, keep_of(cfg)) * bench.tile_flops(cfg)
+    assert total == pytest.approx(92.77e12, rel=1e-3)
+    assert bench.dense_tiles(cfg) * bench.tile_flops(cfg) == pytest.approx(371.1e12, rel=1e-3)
+    assert bench.tile_flops(config("tiny")) == 1_048_576
+
+
+def test_whole_job_aggregate():
+    # weak scaling: N ranks' work over the slowest rank's time
+    assert bench.whole_job_tflops(1, 92.8e12, 116.0) == pytest.approx(800.0, rel=1e-3)
+    assert bench.whole_job_tflops(8, 92.8e12, 116.0) == pytest.approx(6400.0, rel=1e-3)
+
+
+def test_traffic_figure_only_for_its_workload(monkeypatch):
+    cfg = config("720p")
+    have = bench.attn_traffic(cfg, 0.25)
+    if have is not None:  # the stored capture matches today's kernel source
+        assert have == pytest.approx(bench.ATTN_TRAFFIC["bytes_per_bh"] * 2 * 24)
+    # other workloads never borrow the figure
+    assert bench.attn_traffic(config("720p"), 0.0625) is None
+    assert bench.attn_traffic(config("720p_dyn"), 0.25) is None
+    assert bench.attn_traffic(config("lowres"), 0.25) is None
+    # a changed kernel source voids it
+    monkeypatch.setitem(bench.ATTN_TRAFFIC, "sha256", "0" * 64)
+    assert bench.attn_traffic(cfg, 0.25) is None
