@@ -10,6 +10,7 @@ ms per call and the fraction of the measured bf16 tensor peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config 720p|720p_dyn|ref_prefix|lowres|sweep] [--keep-ratio r]
+                    [--block-mode 0|1]
                     [--sweep]   # keep-ratio sweep on the 1152x640 grid instead
 
 N > 1 runs under torchrun: each rank processes its own independent call
@@ -425,6 +426,8 @@ def main():
     ap.add_argument("--keep-ratio", type=float, default=None)
     ap.add_argument("--heads", type=int, default=None, help="override heads (profiling runs)")
     ap.add_argument("--batch", type=int, default=None, help="override B (profiling runs)")
+    ap.add_argument("--block-mode", type=int, default=None, choices=(0, 1),
+                    help="override the block mode (0 fixed 4x4x4, 1 dynamic 8x8x8)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -440,6 +443,8 @@ def main():
         cfg["heads"] = args.heads
     if args.batch is not None:
         cfg["B"] = args.batch
+    if args.block_mode is not None:
+        cfg["block_mode"] = args.block_mode
     import block_sparse_attention_47_b200 as bsa
     from block_sparse_attention_47_b200 import build
     build.build()
