@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 4 heads, scaled by the number of (batch, head) problems).  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
 # workload; null otherwise.
-ATTN_TRAFFIC = {"sha256": "4dcab2ba544f24533df192df6f096d1ed7264fc945c5893a47fe1e0e4ecbc7bf",
+ATTN_TRAFFIC = {"sha256": "bc92136e6dd72300f4391de9421a9a0e241c4c4a9ba3207c2f0abfed0a20d1bf",
                 "bytes_per_bh": 2.006707e9 / 4, "workload": ("720p", 0.25, 0)}
 
 

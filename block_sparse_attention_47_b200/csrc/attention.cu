@@ -6,9 +6,9 @@
 // from).
 //
 // CTA = two adjacent query blocks (128 query rows = the full tcgen05 M=128
-// datapath; M=64 would leave half of it idle).  The two blocks' sorted key
-// lists are merged on the fly into a sequence of steps, one 64-token key
-// block each.  Steps go in pairs (one per softmax warpgroup) and each pair's
+// datapath; M=64 would leave half of it idle).  The union of the two
+// blocks' key lists is the CTA's sequence of steps, one 64-token key block
+// each.  Steps go in pairs (one per softmax warpgroup) and each pair's
 // scores come from one full-width MMA burst:
 //     [S_j | S_j+1] = Q [K_j ; K_j+1]^T   M=128, N=128, K=head_dim
 //     O_w += P_j V_j                      M=128, N=head_dim, K=64
@@ -22,6 +22,13 @@
 // several steps ahead of its use and the TMA latency (far L2 partition or
 // HBM) stays hidden.  The K ring is box-major so that the K blocks of two
 // consecutive stages are contiguous (one B operand for the pair burst).
+// Ring discipline: every wait on a ring barrier must be at most one phase
+// away from the phase it tests (a parity wait cannot tell phases two apart).
+// The K ring has an even number of stages, so a stage is reused only by
+// steps of one parity and each K copy warp serves one parity in order.  A V
+// stage is reused by both parities (odd ring), so each V copy warp copies
+// one 64-column box of every step in order, and PVs are issued in step
+// order.
 //
 // Two softmax warpgroups take alternate steps, each with its own running
 // max, running sum and O accumulator (an exact split of the key set); the
@@ -58,8 +65,6 @@
 //
 // Every wait is bounded (2 s); a timeout sets the caller's status word to
 // BSA_ERR_TIMEOUT, drains in-flight copies and MMAs and frees tensor memory.
-#include <climits>
-
 #include "bsa_internal.cuh"
 
 namespace bsa {
