@@ -227,8 +227,13 @@ typedef struct bsa_device_buffers {
  *                           when the work queued on `stream` is complete.
  * Results equal the step-by-step sequence up to the order of the attention
  * kernel's fp32 accumulation (a group's CTAs start their key walks at
- * different blocks).  The library creates its two copy streams per device
- * on first use and keeps them; it allocates no memory. */
+ * different blocks).  Buffer slices: group g uses the g-th 1/groups of the
+ * permuted, pooled, idx and cnt buffers, each laid out as for a problem
+ * with heads = heads_per_group.  Every argument is validated before
+ * anything is queued; a CUDA error while queueing (rare) returns
+ * BSA_ERR_CUDA and may leave part of the work queued.  The library creates
+ * its two copy streams per device on first use and keeps them; it
+ * allocates no memory. */
 bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const void* k_host,
                             const void* v_host, void* o_host, const bsa_device_buffers* buf,
                             int32_t heads_per_group, int32_t* dev_status, void* stream);
