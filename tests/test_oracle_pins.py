@@ -380,6 +380,20 @@ def test_block_sparse_bruteforce_prefix_and_pads():
                                      prefix=(40, 64), keep_ratio=0.34, heads=2, head_dim=16))
 
 
+def test_block_sparse_bruteforce_dynamic_layout():
+    """The same brute-force pin under a dynamic layout that mixes block shapes
+    (regions coded 2, 1, 2, 0), with a padded row and a prefix segment: the
+    mask is built from the dynamic permutation, so a block that gathers the
+    wrong tokens, or a shape applied to the wrong region, fails it."""
+    prob = small_prob(T=8, H=16, W=16, T_valid=8, H_valid=15, W_valid=16, prefix=(40,),
+                      block_mode=1, blobs=6, keep_ratio=0.3, heads=2, head_dim=16)
+    q, k, v = bf16_inputs(prob, seed=5)
+    out, perms, codes, lists = O.forward(prob, q, k, v)
+    assert len(set(codes[0].tolist())) >= 3  # several shapes, not only the default
+    ref = masked_attention_bruteforce(prob, q, k, v, perms[0], lists)
+    assert np.abs(out - ref).max() < 1e-12
+
+
 def test_dynamic_vs_fixed_same_kept_tile_count():
     """The block shape changes where attention looks, not how much ([PRISM]
     section on the dynamic-block speed)."""
