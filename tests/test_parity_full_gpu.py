@@ -37,6 +37,7 @@ def built(cuda_ok):
 
 
 def bh_sample(cfg, rng, count=3):
+    count = min(count, cfg["B"] * cfg["heads"])
     pairs = {(0, 0), (cfg["B"] - 1, cfg["heads"] - 1)}
     while len(pairs) < count:
         pairs.add((int(rng.integers(0, cfg["B"])), int(rng.integers(0, cfg["heads"]))))
@@ -45,6 +46,12 @@ def bh_sample(cfg, rng, count=3):
 
 @pytest.mark.parametrize("name,over", FULL, ids=["%s%s" % (n, "-" + "-".join("%s=%s" % kv for kv in o.items()) if o else "") for n, o in FULL])
 def test_full_size_parity(name, over):
+    check_full_size(name, over)
+
+
+def check_full_size(name, over):
+    """The checks of one full-size workload (also used by the maximum-size
+    test, which runs last)."""
     cfg = config(name, **over)
     rng = np.random.default_rng(1234)
     q, k, v = make_qkv(cfg, 42000 + len(name), pad_fill=1e4, device="cuda")
