@@ -341,6 +341,24 @@ def test_sparsity0_equals_sdpa():
     check_sparsity0_is_dense(small_prob(T=4, H=8, W=8, prefix=(30, 64), heads=1, head_dim=8))
 
 
+def test_single_video_block_with_prefix_is_dense():
+    """Degenerate grid: one video block (4x4x4) behind a prefix.  Top-k has a
+    single candidate, so even the lowest keep ratio keeps every block, and
+    the call must equal dense attention (torch fp64 SDPA with a key mask)."""
+    prob = small_prob(T=4, H=4, W=4, T_valid=4, H_valid=4, W_valid=4, prefix=(20, 64),
+                      heads=2, head_dim=8, keep_ratio=0.01)
+    geo = O.Geometry(prob)
+    assert geo.nbv == 1 and geo.nbp == 2
+    assert O.keep_count(geo.nbv, prob["keep_ratio"]) == 1
+    q, k, v = bf16_inputs(prob)
+    out, _, _, lists = O.forward(prob, q, k, v)
+    assert all(list(l) == [0, 1, 2] for lb in lists for lh in lb for l in lh)
+    valid = geo.token_valid()
+    ref = sdpa_dense_raster(q, k, v, valid, 1 / math.sqrt(geo.d))
+    assert np.abs(out[:, valid] - ref[:, valid]).max() < 1e-12
+    assert not out[:, ~valid].any()
+
+
 def masked_attention_bruteforce(prob, q, k, v, perm, lists):
     """Raster-order attention under an explicit token x token mask built from
     the kept block pairs; one pass over each row with -inf outside the mask."""
