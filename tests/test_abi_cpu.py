@@ -182,3 +182,16 @@ def test_forward_host_int32_lists_need_4_byte_alignment_only():
     b = host_buffers(idx=20, cnt=36)
     st = L.bsa_forward_host(ctypes.byref(p), 16, 16, 16, 16, ctypes.byref(b), 1, None, None)
     assert st == 5, L.bsa_last_error()
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without libbsa.so every call that needs it raises."""
+    monkeypatch.setattr(bsa, "_LIB", None)
+    monkeypatch.setattr(bsa, "LIB_PATH", str(tmp_path / "libbsa.so"))
+    with pytest.raises(ImportError):
+        bsa.lib()
+    with pytest.raises(ImportError):
+        bsa.keep_count(1920, 0.25)
+    p = base()
+    with pytest.raises(ImportError):
+        bsa.BlockSparseAttention(p, device="cpu")
