@@ -95,6 +95,21 @@ def tile_flops(cfg):
     return 4 * 64 * 64 * cfg["head_dim"]
 
 
+def stage_bandwidth(cfg, stage_ms):
+    """Achieved GB/s of the memory-bound stages: algorithmic bytes (one bf16
+    [B, N, heads, d] tensor is R bytes) over each stage's time.  permute
+    reads and writes Q, K, V (6R), pool reads permuted Q and K (2R),
+    unpermute reads and writes O (2R), the dynamic layout reads K (R); the
+    pooled outputs and index lists are small and not counted."""
+    s = derived_sizes(cfg)
+    R = cfg["B"] * s["N"] * cfg["heads"] * cfg["head_dim"] * 2
+    nbytes = {"permute": 6 * R, "pool": 2 * R, "unpermute": 2 * R}
+    if cfg["block_mode"] == 1:
+        nbytes["layout"] = R
+    return {k: round(v / (stage_ms[k] * 1e-3) / 1e9, 1)
+            for k, v in nbytes.items() if stage_ms.get(k, 0) > 0}
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
@@ -479,6 +494,7 @@ def main():
                          "peak_kind": "%s bf16 sustained" % pk_kind,
                          "frac_of_burst": attn_tflops / pk["bf16_tflops"]},
             "stage_ms": res["stage_ms"],
+            "stage_gbs": stage_bandwidth(cfg, res["stage_ms"]),
             "gpu_launches": launches_per_step(cfg) * args.steps,
         }
         if "dense_ms" in res:

@@ -58,3 +58,16 @@ def test_traffic_figure_only_for_its_workload(monkeypatch):
     # a changed kernel source voids it
     monkeypatch.setitem(bench.ATTN_TRAFFIC, "sha256", "0" * 64)
     assert bench.attn_traffic(cfg, 0.25) is None
+
+
+def test_stage_bandwidth():
+    cfg = config("720p")
+    R = 2 * 122880 * 24 * 128 * 2                      # one raster tensor, 1.51 GB
+    gbs = bench.stage_bandwidth(cfg, {"permute": 1.9, "pool": 0.6, "unpermute": 0.65,
+                                      "layout": 0.009, "select": 4.7})
+    assert gbs["permute"] == pytest.approx(6 * R / 1.9e-3 / 1e9, rel=1e-3)
+    assert gbs["pool"] == pytest.approx(2 * R / 0.6e-3 / 1e9, rel=1e-3)
+    assert set(gbs) == {"permute", "pool", "unpermute"}  # fixed layout reads nothing
+    dyn = bench.stage_bandwidth(config("720p_dyn"), {"layout": 1.2, "permute": 1.9})
+    assert dyn["layout"] == pytest.approx(R / 1.2e-3 / 1e9, rel=1e-3)
+    assert bench.stage_bandwidth(cfg, {}) == {}
