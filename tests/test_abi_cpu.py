@@ -195,3 +195,31 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     p = base()
     with pytest.raises(ImportError):
         bsa.BlockSparseAttention(p, device="cpu")
+
+
+def test_last_error_is_per_thread():
+    """bsa_last_error() reports the calling thread's own failure."""
+    import threading
+    L = bsa.lib()
+    barrier = threading.Barrier(2)
+    seen = {}
+
+    def fail_with(key, **bad):
+        p = base(**bad)
+        for _ in range(200):
+            barrier.wait()
+            st = L.bsa_query_sizes(ctypes.byref(p), ctypes.byref(bsa.Sizes()))
+            barrier.wait()  # the other thread has made its own failing call too
+            seen.setdefault(key, set()).add((st, L.bsa_last_error()))
+
+    threads = [threading.Thread(target=fail_with, args=("dim",), kwargs=dict(head_dim=96)),
+               threading.Thread(target=fail_with, args=("batch",), kwargs=dict(B=0))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert len(seen["dim"]) == 1 and len(seen["batch"]) == 1
+    (st_d, msg_d), = seen["dim"]
+    (st_b, msg_b), = seen["batch"]
+    assert st_d == 3 and b"head_dim" in msg_d
+    assert st_b == 2 and b"B and heads" in msg_b
