@@ -44,8 +44,8 @@ from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per sparse-attention launch from one ncu capture
-# (profiles/attn_fwd_720p_b1h4.md: 1.882 GB read + 0.125 GB written for B=1 x
-# 4 heads, scaled by the number of (batch, head) problems).  Valid only for
+# of a B=1 x 4-head launch of the 720p grid (1.882 GB read + 0.125 GB
+# written), scaled by the number of (batch, head) problems.  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
 # workload; null otherwise.
 ATTN_TRAFFIC = {"sha256": "bc92136e6dd72300f4391de9421a9a0e241c4c4a9ba3207c2f0abfed0a20d1bf",
@@ -381,11 +381,17 @@ def cpu_baseline(cfg, keep, budget_s=15.0):
         n = int(n * min(budget_s / max(secs, 1e-3), 16))
         secs, tiles, _ = oracle_sample(cfg, keep, n, 4243, inputs)
     tflops = tiles * tile_flops(cfg) / secs / 1e12
+    full = kept_tiles(cfg, keep)
     return {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "extrapolated_full_call_s": secs * full / tiles,
             "sample": "fp64 numpy oracle, one (batch, head) of %s: layout, permute, pool, full "
                       "block scores, top-k and attention for %d seeded query blocks (%d kept "
-                      "tiles) in %.1f s; value = kept-tile FLOPs / wall time"
-                      % (cfg.get("name", "?"), n, tiles, secs)}
+                      "tiles) in %.1f s; value = kept-tile FLOPs / wall time.  The oracle "
+                      "loops over query blocks in one Python thread; only its numpy matrix "
+                      "products use the %d BLAS threads counted as cores.  "
+                      "extrapolated_full_call_s scales the sample linearly in kept tiles to "
+                      "the whole call (%d tiles)"
+                      % (cfg.get("name", "?"), n, tiles, secs, cpu_threads(), full)}
 
 
 # ----------------------------------------------------------------------------
@@ -460,16 +466,19 @@ def main():
         cfg["B"] = args.batch
     if args.block_mode is not None:
         cfg["block_mode"] = args.block_mode
-    import block_sparse_attention_47_b200 as bsa
-    from block_sparse_attention_47_b200 import build
-    build.build()
-    keep = bsa.keep_count(derived_sizes(cfg)["nbv"], cfg["keep_ratio"])
-
     world, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
-            reference_arm(args, cfg, keep, world, rank)
+            # the oracle arm shares nothing with the CUDA path: the keep count
+            # comes from the oracle and the product library is never loaded
+            from oracle import bsa_oracle as O
+            reference_arm(args, cfg, O.keep_count(derived_sizes(cfg)["nbv"], cfg["keep_ratio"]),
+                          world, rank)
             return
+        import block_sparse_attention_47_b200 as bsa
+        from block_sparse_attention_47_b200 import build
+        build.build()
+        keep = bsa.keep_count(derived_sizes(cfg)["nbv"], cfg["keep_ratio"])
         if args.sweep:
             sweep(args, world, rank, local)
             return
@@ -539,11 +548,48 @@ def sweep(args, world, rank, local):
                      "stage_ms": st})
     sched = layer_keep_schedule()
     by_ratio = {row["keep_ratio"]: row["ms_per_call"] for row in rows}
+    measured = schedule_ms(base, sched, args, world, rank, local)
     if rank == 0:
         print(json.dumps({"sweep": "1152x640 grid, 92,160 tokens, 24 heads, d=128",
                           "rows": rows,
                           "layer_schedule_40": {"keep_ratios": sched,
-                                                "ms_total": sum(by_ratio[r] for r in sched)}}))
+                                                "ms_total_measured": measured,
+                                                "ms_total_sum_of_rows":
+                                                    sum(by_ratio[r] for r in sched)}}))
+
+
+def schedule_ms(base, sched, args, world, rank, local):
+    """The 40-layer schedule timed as 40 consecutive calls on one stream (one
+    set of buffers per keep ratio, one set of seeded inputs), the median of
+    `args.steps` passes after `args.warmup` untimed ones, max over ranks."""
+    import block_sparse_attention_47_b200 as bsa
+    dev = torch.device("cuda", local)
+    nbv = derived_sizes(base)["nbv"]
+    attns = {r: bsa.BlockSparseAttention(
+        bsa.Problem.make(**dict(base, keep_blocks=bsa.keep_count(nbv, r))), device=dev)
+        for r in sorted(set(sched))}
+    q, k, v = make_qkv(base, rank_seed(rank), pad_fill=0.0, device=dev)
+    out = torch.empty_like(q)
+
+    def one_pass():
+        for r in sched:
+            run_step(bsa, attns[r], q, k, v, out, None)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        one_pass()
+        b_.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b_))
+    for attn in attns.values():
+        attn.check_status()
+    return max_over_ranks(statistics.median(times), world)
 
 
 if __name__ == "__main__":

@@ -30,7 +30,8 @@ FIXED_444 = 0
 DYNAMIC_888 = 1
 
 STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "BSA_ERR_UNSUPPORTED",
-          4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_TIMEOUT"}
+          4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_TIMEOUT",
+          7: "BSA_ERR_HOST_MEMORY"}
 
 
 class BSAError(RuntimeError):
@@ -113,6 +114,7 @@ _SIGS = {
     "bsa_forward_host": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P,
                                         ctypes.POINTER(DeviceBuffers), ctypes.c_int32, _P, _P]),
     "bsa_debug_stall_pv": (ctypes.c_int, [ctypes.c_int32]),
+    "bsa_take_default_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), _P]),
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_last_error": (ctypes.c_char_p, []),
 }
@@ -227,9 +229,19 @@ def default_heads_per_group(heads, groups=32):
 
 
 def debug_stall_pv(enable):
-    """Test hook: while enabled, attention launches issue no PV, so their
-    bounded wait runs out and BSA_ERR_TIMEOUT reaches the status word."""
+    """Test hook: while enabled, attention launches queued by the calling
+    thread issue no PV, so their bounded wait runs out and BSA_ERR_TIMEOUT
+    reaches the status word."""
     _check(lib().bsa_debug_stall_pv(1 if enable else 0))
+
+
+def take_default_status(stream=None):
+    """Read and clear the library-owned status word that receives the
+    device-side errors of calls made without a dev_status (waits for the
+    stream first)."""
+    v = ctypes.c_int32(0)
+    _check(lib().bsa_take_default_status(ctypes.byref(v), _stream(stream)))
+    return int(v.value)
 
 
 def layout_stats(prob, layout_buf, stream=None):
@@ -319,4 +331,4 @@ class BlockSparseAttention:
 __all__ = ["Problem", "Sizes", "BSAError", "BlockSparseAttention", "lib", "keep_count",
            "query_sizes", "layout", "permute", "pool", "select_topk", "sparse_attn_fwd",
            "dense_attn_fwd", "unpermute", "layout_stats", "forward_host", "DeviceBuffers",
-           "default_heads_per_group", "debug_stall_pv", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]
+           "default_heads_per_group", "debug_stall_pv", "take_default_status", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]

@@ -295,10 +295,13 @@ __global__ void __launch_bounds__(512, 1)
         else
           tma_load_3d(sV + s * C::BLK_BYTES + bx * C::BOX, &mv, ful, 64 * bx, t * 64, bh);
       }
-      if (!ok) {
-        report_timeout(abort_flag, status);
-        // this warp's copies that may still be in flight: its last uses of
-        // the ring (RS steps back: 4 stages of one parity for K, 5 for V)
+      if (!ok) report_timeout(abort_flag, status);
+      // On any abort (this warp's own wait or another role's), the consumers
+      // may have quit before reading this warp's last copies: wait, bounded,
+      // for the ones that can still be in flight, its last uses of the ring
+      // (RS steps back: 4 stages of one parity for K, 5 for V), so that no
+      // copy writes shared memory after the CTA has moved on.
+      if (!ok || *abort_flag) {
         for (int jj = j - stride; jj >= 0 && jj >= j - RS; jj -= stride)
           mbar_wait(ful_of(is_k, jj % RS), (jj / RS) & 1, nullptr, 200000000ull);
       }

@@ -5,7 +5,6 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -33,11 +32,13 @@ bsa_status cuda_fail(cudaError_t e, const char* what) {
   return fail(BSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// library-owned fallback status word for callers that pass dev_status = NULL
+// library-owned status word (one per device) for callers that pass
+// dev_status = NULL; read and cleared by bsa_take_default_status
 __device__ int32_t g_dev_status_sink;
 
-// test hook (bsa_debug_stall_pv): attention launches while set issue no PV
-std::atomic<int> g_stall_pv{0};
+// test hook (bsa_debug_stall_pv): attention launches made by this thread
+// while it is set issue no PV; other threads' launches are unaffected
+thread_local int g_stall_pv = 0;
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
@@ -324,7 +325,7 @@ static bsa_status attention_common(const bsa_problem* prob, const void* layout_b
     cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dev_status_sink);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status sink)");
   }
-  g.stall_pv = g_stall_pv.load();
+  g.stall_pv = g_stall_pv;
   cudaError_t e = bsa::launch_attention(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
                                         maps, static_cast<const __nv_bfloat16*>(q_perm), idx,
                                         cnt, static_cast<__nv_bfloat16*>(o_perm),
@@ -530,7 +531,26 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
 
 bsa_status bsa_debug_stall_pv(int32_t enable) {
   g_last_error[0] = 0;
-  g_stall_pv.store(enable ? 1 : 0);
+  g_stall_pv = enable ? 1 : 0;
+  return BSA_OK;
+}
+
+bsa_status bsa_take_default_status(int32_t* out, void* stream) {
+  g_last_error[0] = 0;
+  if (!out) return fail(BSA_ERR_INVALID_ARG, "out is NULL");
+  BSA_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  const int32_t zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_dev_status_sink, sizeof(v), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(g_dev_status_sink, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                                st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "bsa_take_default_status");
+  *out = v;
   return BSA_OK;
 }
 
@@ -549,7 +569,7 @@ bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int
   BSA_TRY(check_device());
   const size_t n = size_t(g.B) * g.nreg;
   unsigned char* host = static_cast<unsigned char*>(malloc(n));
-  if (!host) return fail(BSA_ERR_INVALID_ARG, "host allocation of %zu bytes failed", n);
+  if (!host) return fail(BSA_ERR_HOST_MEMORY, "host allocation of %zu bytes failed", n);
   const char* src = static_cast<const char*>(layout_buf) + bsa::layout_map(g).codes;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(host, src, n, cudaMemcpyDeviceToHost, st);
@@ -572,6 +592,7 @@ const char* bsa_status_string(bsa_status s) {
     case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
     case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
     case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+    case BSA_ERR_HOST_MEMORY: return "BSA_ERR_HOST_MEMORY";
   }
   return "BSA_ERR_UNKNOWN";
 }

@@ -37,7 +37,10 @@
  *     gives a message (per calling thread).
  *   - Errors found on the device (a bounded wait that ran out) are written
  *     to the optional `dev_status` int32 device word as a bsa_status value;
- *     the word is never cleared by the library.
+ *     the word is never cleared by the library.  With dev_status == NULL
+ *     they go to one library-owned word per device instead, shared by every
+ *     such call; nothing reports it unless the caller reads it with
+ *     bsa_take_default_status.
  *   - Token order "raster": prefix segment s occupies
  *     [off_s, off_s + pad64(prefix_len[s])) with its pad tokens at the end,
  *     then video token (t, y, x) sits at P + (t*H + y)*W + x, where
@@ -70,7 +73,8 @@ typedef enum {
                               than on-chip selection holds, no sm_100 GPU */
   BSA_ERR_WORKSPACE = 4,   /* a caller buffer is too small */
   BSA_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
-  BSA_ERR_TIMEOUT = 6      /* device-side bounded wait ran out */
+  BSA_ERR_TIMEOUT = 6,     /* device-side bounded wait ran out */
+  BSA_ERR_HOST_MEMORY = 7  /* a host-side allocation failed */
 } bsa_status;
 
 typedef enum {
@@ -243,8 +247,18 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
  * the first PV runs out after 2 s.  The kernel then writes BSA_ERR_TIMEOUT
  * to the status word, drains its copies and MMAs, frees tensor memory and
  * returns, and the CUDA context stays usable.  Output is undefined for
- * launches made while enabled.  Process-wide; off by default. */
+ * launches made while enabled.  The switch belongs to the calling thread:
+ * only attention launches queued by that thread are affected, never
+ * another thread's.  Off by default. */
 bsa_status bsa_debug_stall_pv(int32_t enable);
+
+/* The library-owned status word of the current device, which receives the
+ * device-side errors of every call made with dev_status == NULL: waits for
+ * the work queued on `stream` (which should include those calls), writes
+ * the word to *out (BSA_OK when nothing went wrong) and clears it.  The word
+ * is shared by all such calls on the device, so a caller that needs
+ * per-call status passes its own dev_status instead. */
+bsa_status bsa_take_default_status(int32_t* out, void* stream);
 
 /* Name of a status code. */
 const char* bsa_status_string(bsa_status status);

@@ -113,6 +113,68 @@ def check_list_row(gpu_row, scores_row, keep, nbp):
     return list(vid) == O.topk_row(scores_row, keep)
 
 
+def topk_alternatives(scores_row, keep, limit=256):
+    """Every list the oracle accepts for one query block: the `keep`-subsets
+    (ascending) that hold every block scoring above kth + band and no block
+    scoring below kth - band, where kth is the keep-th largest fp32 score
+    and band = TIE_REL * max |score| (the near-tie band).  Without a near tie
+    this is the single list O.topk_row gives."""
+    s = np.asarray(scores_row, dtype=np.float64)
+    kth = np.sort(s)[::-1][keep - 1]
+    band = TIE_REL * max(np.abs(s).max(), 1e-30)
+    sure = np.nonzero(s > kth + band)[0]
+    maybe = np.nonzero(np.abs(s - kth) <= band)[0]
+    need = keep - len(sure)
+    assert 0 < need <= len(maybe)
+    if need == len(maybe):
+        return [sorted(int(x) for x in np.concatenate([sure, maybe]))]
+    if math.comb(len(maybe), need) > limit:
+        raise AssertionError("near-tie band too wide to enumerate (%d of %d)" % (need, len(maybe)))
+    import itertools
+    return [sorted(int(x) for x in np.concatenate([sure, np.asarray(c, dtype=np.int64)]))
+            for c in itertools.combinations(maybe, need)]
+
+
+def matched_lists(geo, S, gpu_idx_bh, keep, rows=None):
+    """The oracle's list of every query block (or of `rows`) of one
+    (batch, head), chosen among its own valid alternatives
+    (topk_alternatives) as the one the GPU took.  Fails unless the GPU's
+    list is one of them.  Prefix query blocks keep every block."""
+    lists = [None] * geo.nb
+    every = np.arange(geo.nb, dtype=np.int64)
+    pre = np.arange(geo.nbp, dtype=np.int64)
+    for i in (range(geo.nb) if rows is None else rows):
+        if i < geo.nbp:
+            lists[i] = every
+            continue
+        gpu = [int(x) - geo.nbp for x in gpu_idx_bh[i, geo.nbp:geo.nbp + keep]]
+        alts = topk_alternatives(S[i - geo.nbp], keep)
+        assert gpu in alts, "query block %d: the GPU list is not a valid top-%d" % (i, keep)
+        lists[i] = np.concatenate([pre, np.asarray(alts[alts.index(gpu)], dtype=np.int64)
+                                   + geo.nbp])
+    return lists
+
+
+def oracle_forward_matched(cfg, host, gpu_idx, keep):
+    """O.forward on the host inputs with, for every (batch, head) and query
+    block, the oracle's valid selection that equals the GPU's (so every row
+    is compared, near ties included).  gpu_idx is [B, heads, nb, kcap]."""
+    geo = O.Geometry(cfg)
+    qn, kn, vn = host
+    lay = O.layout(cfg, kn)
+    all_lists = []
+    for b in range(geo.B):
+        perm = lay[b][0]
+        per = []
+        for hh in range(geo.h):
+            qp, kp, _ = oracle_bh(geo, perm, qn, kn, vn, b, hh)
+            S = O.block_scores_f32(geo, O.pool(geo, perm, qp), O.pool(geo, perm, kp))
+            per.append(matched_lists(geo, S, gpu_idx[b, hh], keep))
+        all_lists.append(per)
+    out, _, _, _ = O.forward(dict(cfg, keep_blocks=keep), qn, kn, vn, lists_override=all_lists)
+    return out
+
+
 def oracle_bh(geo, perm, q, k, v, b, hh):
     """Oracle permuted fp64 rows of one (batch, head)."""
     return (O.permute(geo, perm, q[b, :, hh]), O.permute(geo, perm, k[b, :, hh]),

@@ -31,7 +31,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol():
     names = declared_functions()
-    assert len(names) == 14, names
+    assert len(names) == 15, names
     for n in names:
         assert hasattr(bsa.lib(), n), n
     assert set(names) == set(bsa._SIGS), "binding and header disagree"
@@ -132,6 +132,13 @@ def test_null_and_misaligned_pointers_rejected():
 def test_status_strings():
     for code, name in bsa.STATUS.items():
         assert bsa.lib().bsa_status_string(code).decode() == name
+    assert bsa.lib().bsa_status_string(99).decode() == "BSA_ERR_UNKNOWN"
+
+
+def test_take_default_status_validation():
+    L = bsa.lib()
+    assert L.bsa_take_default_status(None, None) == 1
+    assert b"out" in L.bsa_last_error()
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")

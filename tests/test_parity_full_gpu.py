@@ -14,8 +14,8 @@ import torch
 
 from gen import config, make_qkv
 from oracle import bsa_oracle as O
-from parity_helpers import (GpuRun, assert_close, check_list_row, decode_map, oracle_bh,
-                            sample_blocks, scale_of, to_np64)
+from parity_helpers import (GpuRun, assert_close, decode_map, matched_lists, sample_blocks,
+                            scale_of, to_np64)
 
 pytestmark = pytest.mark.gpu
 
@@ -26,6 +26,8 @@ FULL = [
     ("ref_prefix", {}),
     ("lowres", {}),
     ("lowres", {"keep_ratio": 1.0}),
+    ("sweep", {"keep_ratio": 0.10}),
+    ("sweep", {"keep_ratio": 0.03}),
     ("sweep", {"keep_ratio": 0.01}),
 ]
 
@@ -87,7 +89,6 @@ def check_full_size(name, over):
     idx, cnt = run.attn.idx.cpu().numpy(), run.attn.cnt.cpu().numpy()
     gq_pool, gk_pool = run.attn.q_pool.cpu().numpy(), run.attn.k_pool.cpu().numpy()
     out = run.out
-    exact = total = 0
     for b, hh in bh_sample(cfg, rng):
         perm = perms[b]
         host = [to_np64(t[b, :, hh]) for t in (q, k, v)]
@@ -112,22 +113,18 @@ def check_full_size(name, over):
         np.put_along_axis(chosen, vid, True, axis=1)
         assert not np.any(~chosen & (S > (kth + band)[:, None])), "a clearly better block was dropped"
         assert not np.any(chosen & (S < (kth - band)[:, None])), "a clearly worse block was kept"
-        # attention on sampled query blocks with the oracle's own lists
+        # attention on sampled query blocks, every one compared: the oracle's
+        # list for a block is its own valid selection equal to the GPU's
         extra = []
         if cfg["H_valid"] < cfg["H"]:
             extra.append(geo.nbp + (geo.nbv - 1))
         blocks = sample_blocks(geo, 8, rng, extra)
-        lists = O.select(geo, qpool, kpool, keep, rows=blocks)
+        lists = matched_lists(geo, S, idx[b, hh], keep, rows=blocks)
         want = O.block_sparse_attention(geo, perm, *op, lists, scale_of(cfg), blocks)
         got_raster = to_np64(out[b, :, hh])
         for i in blocks:
-            total += 1
-            if i >= geo.nbp and list(idx[b, hh, i, :geo.nbp + keep]) != list(lists[i]):
-                continue  # a near tie chose differently; validity checked above
-            exact += 1
             slots = perm[i * 64:(i + 1) * 64]
             assert_close(got_raster[slots], want[i], "%s b%d h%d block %d" % (name, b, hh, i))
-    assert exact >= 0.9 * total
     pad = torch.from_numpy(~valid).to(out.device)
     assert not bool(out[:, pad].any()), "pad tokens must come out as 0"
     assert int(run.attn.status.item()) == 0
