@@ -115,6 +115,8 @@ _SIGS = {
                                         ctypes.POINTER(DeviceBuffers), ctypes.c_int32, _P, _P]),
     "bsa_debug_stall_pv": (ctypes.c_int, [ctypes.c_int32]),
     "bsa_take_default_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), _P]),
+    "bsa_forward_noalloc": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _I64, _I64, _I64,
+                                           _P, _I64, _I64, _I64, _P, _P]),
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_last_error": (ctypes.c_char_p, []),
 }
@@ -218,6 +220,21 @@ def forward_host(prob, q_host, k_host, v_host, o_host, buffers, heads_per_group,
     _check(lib().bsa_forward_host(ctypes.byref(prob), _ptr(q_host), _ptr(k_host), _ptr(v_host),
                                   _ptr(o_host), ctypes.byref(buffers), int(heads_per_group),
                                   _ptr(dev_status), _stream(stream)))
+
+
+def forward_noalloc(prob, q, k, v, out, dev_status=None, stream=None):
+    """The whole call on device raster tensors with the library's static
+    scratch instead of caller buffers (bsa_forward_noalloc), for callers that
+    cannot allocate device memory.  q, k and v must share their strides."""
+    sb, sn, sh = _raster_strides(q)
+    if _raster_strides(k) != (sb, sn, sh) or _raster_strides(v) != (sb, sn, sh):
+        raise ValueError("q, k and v must share their strides")
+    ob, on, oh = _raster_strides(out)
+    _check(lib().bsa_forward_noalloc(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), sb, sn, sh,
+                                     _ptr(out), ob, on, oh, _ptr(dev_status), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def default_heads_per_group(heads, groups=32):
@@ -331,4 +348,5 @@ class BlockSparseAttention:
 __all__ = ["Problem", "Sizes", "BSAError", "BlockSparseAttention", "lib", "keep_count",
            "query_sizes", "layout", "permute", "pool", "select_topk", "sparse_attn_fwd",
            "dense_attn_fwd", "unpermute", "layout_stats", "forward_host", "DeviceBuffers",
-           "default_heads_per_group", "debug_stall_pv", "take_default_status", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]
+           "default_heads_per_group", "debug_stall_pv", "take_default_status",
+           "forward_noalloc", "NOALLOC_SCRATCH_BYTES", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]

@@ -15,10 +15,22 @@ size_t select_smem_bytes(const Geo& g);
 }
 
 namespace {
+thread_local char g_last_error[512] = "";
+}
+
+namespace bsa {
+bsa_status set_error(bsa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+}  // namespace bsa
+
+namespace {
 
 using bsa::Geo;
-
-thread_local char g_last_error[512] = "";
 
 bsa_status fail(bsa_status st, const char* fmt, ...) {
   va_list ap;

@@ -85,6 +85,9 @@ __host__ __device__ inline void shape_sides(int code, int& st, int& sh, int& sw)
   sw = (c & 1) ? lo : hi;
 }
 
+// Record a message for bsa_last_error() on the calling thread and return st.
+bsa_status set_error(bsa_status st, const char* fmt, ...);
+
 // ---- launchers (one per translation unit) -------------------------------
 cudaError_t launch_layout(const Geo& g, const __nv_bfloat16* k, int64_t sb, int64_t sn,
                           int64_t sh, LayoutPtrs lp, cudaStream_t st);

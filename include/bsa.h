@@ -25,8 +25,9 @@
  * speed-up denominator).
  *
  * Conventions (every entry point):
- *   - The caller owns all memory.  The library allocates no device memory;
- *     sizes of every buffer come from bsa_query_sizes.
+ *   - The caller owns all memory.  The library allocates no device memory
+ *     (its one static device array, for bsa_forward_noalloc, comes with the
+ *     loaded code); sizes of every buffer come from bsa_query_sizes.
  *   - Device pointers must be 16-byte aligned (index lists and counts: 4
  *     bytes); the innermost (head_dim) dimension of every tensor is
  *     contiguous.
@@ -259,6 +260,42 @@ bsa_status bsa_debug_stall_pv(int32_t enable);
  * is shared by all such calls on the device, so a caller that needs
  * per-call status passes its own dev_status instead. */
 bsa_status bsa_take_default_status(int32_t* out, void* stream);
+
+/* Size of the library's static scratch array used by bsa_forward_noalloc
+ * (64 MiB per device that loads the library, held until the process exits). */
+#define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* The whole device-side call (layout, permute, pool, top-k selection, sparse
+ * attention, unpermute) without any caller-provided intermediate buffer and
+ * without allocating device memory.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate, such as a plugin or
+ * FFI binding that receives only the tensors it is handed and cannot reach
+ * its host application's allocator, a runtime whose device memory is fixed
+ * at start-up, or a latency-bound loop that must not call cudaMalloc (which
+ * can synchronise the device).
+ *   q_raster, k_raster, v_raster  [B, N, heads, head_dim] bf16 on the device,
+ *                                 sharing the element strides (stride_b,
+ *                                 stride_n, stride_h)
+ *   o_raster                      output, same layout with strides
+ *                                 (o_stride_b, o_stride_n, o_stride_h); pad
+ *                                 tokens are written as 0
+ *   dev_status, stream            as in bsa_sparse_attn_fwd
+ * The intermediates (layout, permuted Q/K/V/O, pooled means, index lists)
+ * live in one static device array of BSA_NOALLOC_SCRATCH_BYTES owned by the
+ * library.  A problem that needs more returns BSA_ERR_WORKSPACE with the
+ * byte counts in bsa_last_error(), before anything is launched.  The first
+ * call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents
+ * behind; no part of it needs to start at zero, because each step writes
+ * what later steps read.  Calls whose work overlaps on the GPU (other
+ * streams, other threads) race on the array: serialise them.  The library
+ * calls no cudaMalloc, cudaFree or allocating routine here. */
+bsa_status bsa_forward_noalloc(const bsa_problem* prob, const void* q_raster,
+                               const void* k_raster, const void* v_raster, int64_t stride_b,
+                               int64_t stride_n, int64_t stride_h, void* o_raster,
+                               int64_t o_stride_b, int64_t o_stride_n, int64_t o_stride_h,
+                               int32_t* dev_status, void* stream);
 
 /* Name of a status code. */
 const char* bsa_status_string(bsa_status status);
