@@ -44,12 +44,12 @@ from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per sparse-attention launch from one ncu capture
-# of a B=1 x 4-head launch of the 720p grid (1.882 GB read + 0.125 GB
+# of a B=1 x 4-head launch of the 720p grid (1.555 GB read + 0.126 GB
 # written), scaled by the number of (batch, head) problems.  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
-# workload; null otherwise.
-ATTN_TRAFFIC = {"sha256": "bc92136e6dd72300f4391de9421a9a0e241c4c4a9ba3207c2f0abfed0a20d1bf",
-                "bytes_per_bh": 2.006707e9 / 4, "workload": ("720p", 0.25, 0)}
+# workload on the permuted path; null otherwise.
+ATTN_TRAFFIC = {"sha256": "c20bdf7196b5db994bfb8b1aecc059712513c15137fecd1905ad5ee04af3cbf0",
+                "bytes_per_bh": 1.680738e9 / 4, "workload": ("720p", 0.25, 0)}
 
 
 def attn_traffic(cfg, keep_ratio):
@@ -62,6 +62,8 @@ def attn_traffic(cfg, keep_ratio):
     if digest != ATTN_TRAFFIC["sha256"]:
         return None
     if (cfg.get("name"), keep_ratio, cfg["block_mode"]) != ATTN_TRAFFIC["workload"]:
+        return None
+    if PATH["path"] != "perm" or PATH.get("windows") is not None:
         return None
     return ATTN_TRAFFIC["bytes_per_bh"] * cfg["B"] * cfg["heads"]
 METRIC = "ms/call & effective TFLOP/s (kept tiles) at 122,880 tok, s=0.75; % BF16 peak"
@@ -221,35 +223,97 @@ def whole_job_tflops(world, flops_per_rank, ms_slowest):
 STAGES = ("layout", "permute", "pool", "select", "attention", "unpermute")
 
 
+# "perm" (permuted copies) or "raster" (permute-free); the learned-gate
+# matrices (select_topk_gated) and the window heads (window attention) when
+# those modes are timed
+PATH = {"path": "perm", "row_pad": 0, "gate": None, "windows": None}
+
+# window-head patterns for --windows (w_t, w_y, w_x), negative = unbounded: a
+# spatial head sees +-1 latent frame, a temporal head +-2 latent pixels
+WINDOW_PATTERNS = {"spatial": [(1, -1, -1)], "temporal": [(-1, 2, 2)],
+                   "mixed": [(1, -1, -1), (-1, 2, 2)]}
+
+
 def run_step(bsa, attn, q, k, v, out, ev):
-    """One call; ev (list of 7 events or None) brackets the six stages."""
+    """One call; ev (list of 7 events or None) brackets the six stages.  The
+    permute-free path has no permute and unpermute stages (0 ms); window
+    heads have no pool and select stages either."""
     p, L = attn.prob, attn.layout_buf
+    raster = PATH["path"] == "raster"
+    windows = PATH["windows"]
     if ev:
         ev[0].record()
     bsa.layout(p, k, L)
     if ev:
         ev[1].record()
-    bsa.permute(p, L, q, attn.qp)
-    bsa.permute(p, L, k, attn.kp)
-    bsa.permute(p, L, v, attn.vp)
+    if not raster:
+        bsa.permute(p, L, q, attn.qp)
+        bsa.permute(p, L, k, attn.kp)
+        bsa.permute(p, L, v, attn.vp)
     if ev:
         ev[2].record()
-    bsa.pool(p, L, attn.qp, attn.kp, attn.q_pool, attn.k_pool)
+    if windows is None:
+        if raster:
+            bsa.pool_raster(p, L, q, k, attn.q_pool, attn.k_pool)
+        else:
+            bsa.pool(p, L, attn.qp, attn.kp, attn.q_pool, attn.k_pool)
     if ev:
         ev[3].record()
-    bsa.select_topk(p, attn.q_pool, attn.k_pool, attn.idx, attn.cnt)
+    if windows is not None:
+        pass
+    elif PATH["gate"] is not None:
+        bsa.select_topk_gated(p, attn.q_pool, attn.k_pool, PATH["gate"], attn.idx, attn.cnt)
+    else:
+        bsa.select_topk(p, attn.q_pool, attn.k_pool, attn.idx, attn.cnt)
     if ev:
         ev[4].record()
-    bsa.sparse_attn_fwd(p, L, attn.qp, attn.kp, attn.vp, attn.idx, attn.cnt, attn.op, attn.status)
+    if windows is not None:
+        bsa.window_attn_fwd_raster(p, L, q, k, v, windows, out, attn.status)
+    elif raster:
+        bsa.sparse_attn_fwd_raster(p, L, q, k, v, attn.idx, attn.cnt, out, attn.status)
+    else:
+        bsa.sparse_attn_fwd(p, L, attn.qp, attn.kp, attn.vp, attn.idx, attn.cnt, attn.op,
+                            attn.status)
     if ev:
         ev[5].record()
-    bsa.unpermute(p, L, attn.op, out)
+    if not raster:
+        bsa.unpermute(p, L, attn.op, out)
     if ev:
         ev[6].record()
 
 
 def launches_per_step(cfg):
-    return (2 if cfg["block_mode"] == 1 else 1) + 3 + 1 + 1 + 1 + 1
+    layout = 2 if cfg["block_mode"] == 1 else 1
+    if PATH["windows"] is not None:
+        return layout + 1
+    if PATH["path"] == "raster":
+        return layout + 1 + 1 + 1
+    return layout + 3 + 1 + 1 + 1 + 1
+
+
+def window_heads(cfg, pattern):
+    """Per-head windows of a pattern, cycling over the heads."""
+    pat = WINDOW_PATTERNS[pattern]
+    return [pat[h % len(pat)] for h in range(cfg["heads"])]
+
+
+def window_tiles(cfg, wins):
+    """64x64 tiles the window heads visit on the fixed 4x4x4 layout: every
+    prefix row and column, plus the video block pairs whose boxes come within
+    the window on every axis (two blocks d apart along an axis have a gap of
+    4|d| - 3 tokens).  The axes are independent, so the video count of a head
+    is the product of the per-axis counts."""
+    s = derived_sizes(cfg)
+    n = {"t": cfg["T"] // 4, "y": cfg["H"] // 4, "x": cfg["W"] // 4}
+    per_b = 0
+    for w3 in wins:
+        video = 1
+        for w, ax in zip(w3, ("t", "y", "x")):
+            a = np.arange(n[ax])
+            gap = np.maximum(0, 4 * np.abs(a[:, None] - a[None, :]) - 3)
+            video *= int(((gap <= w) | (w < 0)).sum())
+        per_b += video + s["nbp"] * s["nb"] + s["nbv"] * s["nbp"]
+    return cfg["B"] * per_b
 
 
 def measure(cfg, keep, steps, warmup, world, rank, local, do_e2e, do_dense):
@@ -260,11 +324,27 @@ def measure(cfg, keep, steps, warmup, world, rank, local, do_e2e, do_dense):
     torch.cuda.set_device(dev)
     prob = bsa.Problem.make(**dict(cfg, keep_blocks=keep))
     q, k, v = make_qkv(cfg, rank_seed(rank), pad_fill=0.0, device=dev)
+    if PATH.get("row_pad"):
+        # the same tensors in rows of heads*d + row_pad elements (a wider token
+        # stride, as in a fused projection's output buffer)
+        def padded(x):
+            B, N, h, d = x.shape
+            buf = torch.zeros((B, N, h * d + PATH["row_pad"]), dtype=x.dtype, device=x.device)
+            buf[..., :h * d] = x.reshape(B, N, h * d)
+            return buf[..., :h * d].view(B, N, h, d)
+        q, k, v = padded(q), padded(k), padded(v)
     attn = bsa.BlockSparseAttention(prob, device=dev)
     out = torch.empty_like(q)
+    wins = None
+    if PATH.get("window_pattern"):
+        wins = window_heads(cfg, PATH["window_pattern"])
+        PATH["windows"] = torch.tensor(wins, dtype=torch.int32, device=dev)
+    if PATH.get("gate_seed") is not None:
+        from gen import make_gate
+        PATH["gate"] = make_gate(cfg["heads"], cfg["head_dim"], PATH["gate_seed"], device=dev)
     torch.cuda.synchronize()
 
-    flops = kept_tiles(cfg, keep) * tile_flops(cfg)
+    flops = (window_tiles(cfg, wins) if wins else kept_tiles(cfg, keep)) * tile_flops(cfg)
     for _ in range(warmup):
         run_step(bsa, attn, q, k, v, out, None)
     torch.cuda.synchronize()
@@ -307,6 +387,42 @@ def measure(cfg, keep, steps, warmup, world, rank, local, do_e2e, do_dense):
         res["dense_flops"] = dense_tiles(cfg) * tile_flops(cfg)
         del o
 
+    if PATH.get("backward") and PATH["path"] == "perm":
+        # the training step's attention: forward with row statistics, then
+        # the backward (dQ, dK, dV) over the same kept tiles
+        n_tok = attn.sizes.n_tokens
+        lse = torch.empty((cfg["B"], cfg["heads"], n_tok), dtype=torch.float32, device=dev)
+        o = torch.empty_like(attn.op)
+        dout = torch.randn(attn.op.shape, device=dev).to(torch.bfloat16)
+        grads = [torch.empty_like(attn.op) for _ in range(3)]
+        ws = torch.empty(bsa.bwd_workspace_bytes(prob), dtype=torch.uint8, device=dev)
+
+        def fwd():
+            bsa.sparse_attn_fwd_lse(prob, attn.layout_buf, attn.qp, attn.kp, attn.vp, attn.idx,
+                                    attn.cnt, o, lse, attn.status)
+
+        def bwd():
+            bsa.sparse_attn_bwd(prob, attn.layout_buf, attn.qp, attn.kp, attn.vp, o, dout, lse,
+                                attn.idx, attn.cnt, *grads, ws, attn.status)
+        for _ in range(warmup):
+            fwd()
+            bwd()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        fms, bms = [], []
+        for _ in range(steps):
+            ev[0].record()
+            fwd()
+            ev[1].record()
+            bwd()
+            ev[2].record()
+            torch.cuda.synchronize()
+            fms.append(ev[0].elapsed_time(ev[1]))
+            bms.append(ev[1].elapsed_time(ev[2]))
+        attn.check_status()
+        res["backward"] = dict(fwd_lse_ms=statistics.median(fms), bwd_ms=statistics.median(bms))
+        del lse, o, dout, grads, ws
+
     if do_e2e:
         # the call a user with host tensors makes: bsa_forward_host moves
         # every input to the device and the output back, overlapped with the
@@ -316,7 +432,8 @@ def measure(cfg, keep, steps, warmup, world, rank, local, do_e2e, do_dense):
         hg = bsa.default_heads_per_group(cfg["heads"])
 
         def e2e_step():
-            attn.host_call(hq, hk, hv, out=hout, heads_per_group=hg)
+            attn.host_call(hq, hk, hv, out=hout, heads_per_group=hg,
+                           raster=PATH["path"] == "raster")
 
         for _ in range(max(1, min(warmup, 2))):
             e2e_step()
@@ -433,6 +550,12 @@ def workload_config(cfg, keep, args):
                                          "dynamic 8x8x8" if cfg["block_mode"] else "fixed 4x4x4"),
             "global_batch": cfg["B"] * args.gpus, "seq_len": s["N"], "keep_blocks": keep,
             "keep_ratio": cfg["keep_ratio"], "parallelism": "independent calls per GPU (dp%d)" % args.gpus,
+            "path": PATH["path"],
+            "selection": ("window heads (%s: %s)" % (PATH["window_pattern"],
+                                                     WINDOW_PATTERNS[PATH["window_pattern"]])
+                          if PATH.get("window_pattern") else
+                          "learned gate (synthetic seeded matrices)" if PATH.get("gate_seed")
+                          else "pooled-mean top-k"),
             "l2": "inputs larger than L2 (Q, K, V %.2f GB each); no flush" %
                   (cfg["B"] * s["N"] * cfg["heads"] * cfg["head_dim"] * 2 / 1e9)}
 
@@ -449,6 +572,19 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B (profiling runs)")
     ap.add_argument("--block-mode", type=int, default=None, choices=(0, 1),
                     help="override the block mode (0 fixed 4x4x4, 1 dynamic 8x8x8)")
+    ap.add_argument("--path", default="perm", choices=("raster", "perm"),
+                    help="perm: permute -> attention -> unpermute; raster: tiles read straight "
+                         "from the raster tensors (no permuted copies)")
+    ap.add_argument("--row-pad", type=int, default=0,
+                    help="extra elements per raster token row (a wider token stride)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the training step's attention: forward with row "
+                         "statistics and the backward (permuted path)")
+    ap.add_argument("--gate", action="store_true",
+                    help="learned-gate selection with seeded synthetic gate matrices")
+    ap.add_argument("--windows", default=None, choices=sorted(WINDOW_PATTERNS),
+                    help="window heads instead of top-k selection (raster path, fixed blocks); "
+                         "the metric counts the tiles the windows visit")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -456,6 +592,13 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    PATH["path"] = args.path
+    PATH["row_pad"] = args.row_pad
+    PATH["gate_seed"] = 42010 if args.gate else None
+    PATH["window_pattern"] = args.windows
+    PATH["backward"] = args.backward
+    if args.windows:
+        PATH["path"] = "raster"
 
     cfg = config(args.config)
     if args.keep_ratio is not None:
@@ -499,7 +642,9 @@ def main():
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": attn_tflops / peak,
                          "traffic": attn_traffic(cfg, cfg["keep_ratio"]),
-                         "kernel": "attn_fwd_kernel<128,false> (sparse attention)",
+                         "kernel": "attn_fwd_kernel<128,false,%s> (sparse attention, %s)" % (
+                             "true" if PATH["path"] == "raster" else "false",
+                             "raster tensors" if PATH["path"] == "raster" else "permuted tensors"),
                          "peak_kind": "%s bf16 sustained" % pk_kind,
                          "frac_of_burst": attn_tflops / pk["bf16_tflops"]},
             "stage_ms": res["stage_ms"],
@@ -511,6 +656,15 @@ def main():
                              "tflops": res["dense_flops"] / (res["dense_ms"] / 1e3) / 1e12,
                              "speedup_sparse_attention_vs_dense": res["dense_ms"] / res["attn_ms"],
                              "speedup_full_call_vs_dense": res["dense_ms"] / res["ms_step"]}
+        if "backward" in res:
+            bw = res["backward"]
+            # standard count: the backward's five products (S recomputed,
+            # dP, dV, dQ, dK) are 2.5x the forward's two per kept tile
+            line["backward"] = {
+                "fwd_lse_ms": bw["fwd_lse_ms"], "bwd_ms": bw["bwd_ms"],
+                "bwd_tflops": 2.5 * res["flops"] / (bw["bwd_ms"] / 1e3) / 1e12,
+                "flop_count": "2.5 x the forward's kept-tile FLOPs (the kernels compute S and "
+                              "dP in both passes, 3.5 x)"}
         if "e2e" in res:
             e = res["e2e"]
             line["e2e"] = {"value": whole_job_tflops(world, res["flops"], e["ms"]), "unit": "TFLOP/s",

@@ -115,6 +115,20 @@ _SIGS = {
                                         ctypes.POINTER(DeviceBuffers), ctypes.c_int32, _P, _P]),
     "bsa_debug_stall_pv": (ctypes.c_int, [ctypes.c_int32]),
     "bsa_take_default_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), _P]),
+    "bsa_pool_raster": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _I64, _I64, _I64,
+                                       _P, _P, _P]),
+    "bsa_sparse_attn_fwd_raster": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _I64,
+                                                  _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P,
+                                                  _P]),
+    "bsa_sparse_attn_fwd_lse": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P,
+                                               _P, _P, _P, _P]),
+    "bsa_query_bwd_workspace": (ctypes.c_int, [ctypes.POINTER(Problem),
+                                               ctypes.POINTER(ctypes.c_size_t)]),
+    "bsa_sparse_attn_bwd": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _P,
+                                           _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "bsa_select_topk_gated": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P]),
+    "bsa_window_attn_fwd_raster": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _I64,
+                                                  _I64, _I64, _P, _P, _I64, _I64, _I64, _P, _P]),
     "bsa_forward_noalloc": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _I64, _I64, _I64,
                                            _P, _I64, _I64, _I64, _P, _P]),
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -208,6 +222,86 @@ def unpermute(prob, layout_buf, o_perm, o_raster, stream=None):
     sb, sn, sh = _raster_strides(o_raster)
     _check(lib().bsa_unpermute(ctypes.byref(prob), _ptr(layout_buf), _ptr(o_perm), _ptr(o_raster),
                                sb, sn, sh, _stream(stream)))
+
+
+def _shared_strides(*ts):
+    st = _raster_strides(ts[0])
+    if any(_raster_strides(t) != st for t in ts[1:]):
+        raise ValueError("these raster tensors must share their strides")
+    return st
+
+
+def pool_raster(prob, layout_buf, q_raster, k_raster, q_pool, k_pool, stream=None):
+    """Block means straight from raster Q and K (bsa_pool_raster)."""
+    sb, sn, sh = _shared_strides(q_raster, k_raster)
+    _check(lib().bsa_pool_raster(ctypes.byref(prob), _ptr(layout_buf), _ptr(q_raster),
+                                 _ptr(k_raster), sb, sn, sh, _ptr(q_pool), _ptr(k_pool),
+                                 _stream(stream)))
+
+
+def sparse_attn_fwd_raster(prob, layout_buf, q, k, v, idx, cnt, out, dev_status=None,
+                           stream=None):
+    """Block-sparse attention on raster tensors, no permuted copies
+    (bsa_sparse_attn_fwd_raster)."""
+    sb, sn, sh = _shared_strides(q, k, v)
+    ob, on, oh = _raster_strides(out)
+    _check(lib().bsa_sparse_attn_fwd_raster(ctypes.byref(prob), _ptr(layout_buf), _ptr(q),
+                                            _ptr(k), _ptr(v), sb, sn, sh, _ptr(idx), _ptr(cnt),
+                                            _ptr(out), ob, on, oh, _ptr(dev_status),
+                                            _stream(stream)))
+
+
+def sparse_attn_fwd_lse(prob, layout_buf, q_perm, k_perm, v_perm, idx, cnt, o_perm, lse,
+                        dev_status=None, stream=None):
+    """Forward that also writes each row's log-sum-exp (exp2 domain) into the
+    fp32 [B, heads, N] tensor lse, for the backward."""
+    _check(lib().bsa_sparse_attn_fwd_lse(ctypes.byref(prob), _ptr(layout_buf), _ptr(q_perm),
+                                         _ptr(k_perm), _ptr(v_perm), _ptr(idx), _ptr(cnt),
+                                         _ptr(o_perm), _ptr(lse), _ptr(dev_status),
+                                         _stream(stream)))
+
+
+def bwd_workspace_bytes(prob):
+    n = ctypes.c_size_t(0)
+    _check(lib().bsa_query_bwd_workspace(ctypes.byref(prob), ctypes.byref(n)))
+    return int(n.value)
+
+
+def sparse_attn_bwd(prob, layout_buf, q_perm, k_perm, v_perm, o_perm, do_perm, lse, idx, cnt,
+                    dq_perm, dk_perm, dv_perm, workspace, dev_status=None, stream=None):
+    """Gradients dQ, dK, dV (block order) over the forward's kept tiles."""
+    _check(lib().bsa_sparse_attn_bwd(ctypes.byref(prob), _ptr(layout_buf), _ptr(q_perm),
+                                     _ptr(k_perm), _ptr(v_perm), _ptr(o_perm), _ptr(do_perm),
+                                     _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(dq_perm), _ptr(dk_perm),
+                                     _ptr(dv_perm), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _ptr(dev_status), _stream(stream)))
+
+
+def select_topk_gated(prob, q_pool, k_pool, gate, idx, cnt, stream=None):
+    """Top-k selection with a learned-gate score (bsa_select_topk_gated): gate
+    is a device fp32 [heads, head_dim, head_dim] tensor."""
+    if gate.dtype != torch.float32 or tuple(gate.shape) != (prob.heads, prob.head_dim,
+                                                           prob.head_dim) or \
+            not gate.is_contiguous():
+        raise ValueError("gate must be a contiguous float32 [heads, head_dim, head_dim] tensor")
+    _check(lib().bsa_select_topk_gated(ctypes.byref(prob), _ptr(q_pool), _ptr(k_pool), _ptr(gate),
+                                       _ptr(idx), _ptr(cnt), _stream(stream)))
+
+
+def window_attn_fwd_raster(prob, layout_buf, q, k, v, windows, out, dev_status=None,
+                           stream=None):
+    """Attention of window heads on raster tensors (bsa_window_attn_fwd_raster):
+    windows is a device int32 [heads, 3] tensor of (w_t, w_y, w_x), negative =
+    unbounded."""
+    if windows.dtype != torch.int32 or tuple(windows.shape) != (prob.heads, 3) or \
+            not windows.is_contiguous():
+        raise ValueError("windows must be a contiguous int32 [heads, 3] tensor")
+    sb, sn, sh = _shared_strides(q, k, v)
+    ob, on, oh = _raster_strides(out)
+    _check(lib().bsa_window_attn_fwd_raster(ctypes.byref(prob), _ptr(layout_buf), _ptr(q), _ptr(k),
+                                            _ptr(v), sb, sn, sh, _ptr(windows), _ptr(out), ob, on,
+                                            oh, _ptr(dev_status), _stream(stream)))
 
 
 def forward_host(prob, q_host, k_host, v_host, o_host, buffers, heads_per_group, dev_status=None,
@@ -312,9 +406,24 @@ class BlockSparseAttention:
         unpermute(p, self.layout_buf, self.op, out, stream)
         return out
 
-    def device_buffers(self):
+    def raster_call(self, q, k, v, out=None, stream=None):
+        """The same call without permuted copies: layout -> pool_raster ->
+        select -> sparse_attn_fwd_raster (q, k, v share strides, heads
+        contiguous in a token row)."""
+        p = self.prob
+        if out is None:
+            out = torch.empty_like(q)
+        layout(p, k, self.layout_buf, stream)
+        pool_raster(p, self.layout_buf, q, k, self.q_pool, self.k_pool, stream)
+        select_topk(p, self.q_pool, self.k_pool, self.idx, self.cnt, stream)
+        sparse_attn_fwd_raster(p, self.layout_buf, q, k, v, self.idx, self.cnt, out, self.status,
+                               stream)
+        return out
+
+    def device_buffers(self, raster=False):
         """bsa_device_buffers over this object's buffers (raster staging
-        buffers are allocated on first use)."""
+        buffers are allocated on first use).  raster=True leaves the
+        permuted buffers out (NULL): the permute-free sequence runs."""
         if not hasattr(self, "_raster"):
             shape = (self.prob.B, self.sizes.n_tokens, self.prob.heads, self.prob.head_dim)
             self._raster = [torch.empty(shape, dtype=torch.bfloat16, device=self.qp.device)
@@ -323,19 +432,21 @@ class BlockSparseAttention:
         for name, t in zip(("q_raster", "k_raster", "v_raster", "o_raster"), self._raster):
             setattr(b, name, t.data_ptr())
         for name in ("q_perm", "k_perm", "v_perm", "o_perm"):
-            setattr(b, name, getattr(self, name[0] + "p").data_ptr())
+            setattr(b, name, None if raster else getattr(self, name[0] + "p").data_ptr())
         b.layout_buf = self.layout_buf.data_ptr()
         b.q_pool, b.k_pool = self.q_pool.data_ptr(), self.k_pool.data_ptr()
         b.idx, b.cnt = self.idx.data_ptr(), self.cnt.data_ptr()
         return b
 
-    def host_call(self, q_host, k_host, v_host, out=None, heads_per_group=None, stream=None):
+    def host_call(self, q_host, k_host, v_host, out=None, heads_per_group=None, stream=None,
+                  raster=False):
         """The call on host tensors (pinned memory lets the transfers overlap
-        the computation); returns the host output."""
+        the computation); returns the host output.  raster=True runs the
+        permute-free sequence."""
         if out is None:
             out = torch.empty(q_host.shape, dtype=q_host.dtype, pin_memory=q_host.is_pinned())
         hg = heads_per_group or default_heads_per_group(self.prob.heads)
-        forward_host(self.prob, q_host, k_host, v_host, out, self.device_buffers(), hg,
+        forward_host(self.prob, q_host, k_host, v_host, out, self.device_buffers(raster), hg,
                      self.status, stream)
         return out
 
@@ -349,4 +460,7 @@ __all__ = ["Problem", "Sizes", "BSAError", "BlockSparseAttention", "lib", "keep_
            "query_sizes", "layout", "permute", "pool", "select_topk", "sparse_attn_fwd",
            "dense_attn_fwd", "unpermute", "layout_stats", "forward_host", "DeviceBuffers",
            "default_heads_per_group", "debug_stall_pv", "take_default_status",
-           "forward_noalloc", "NOALLOC_SCRATCH_BYTES", "FIXED_444", "DYNAMIC_888", "LIB_PATH"]
+           "forward_noalloc", "NOALLOC_SCRATCH_BYTES", "pool_raster", "sparse_attn_fwd_raster",
+           "window_attn_fwd_raster", "select_topk_gated", "sparse_attn_fwd_lse",
+           "bwd_workspace_bytes", "sparse_attn_bwd",
+           "FIXED_444", "DYNAMIC_888", "LIB_PATH"]

@@ -109,14 +109,122 @@ __device__ __forceinline__ bool bit_of(uint32_t lo, uint32_t hi, int c) {
   return ((c < 32 ? (lo >> c) : (hi >> (c - 32))) & 1u) != 0u;
 }
 
-template <int D, bool DENSE>
+// The box of video block t (t >= nbp) of batch element b: origin
+// (t0, y0, x0) on the grid and sides (st, sh, sw); returns its shape code
+// (0 = 4x4x4).  Its 64 slots hold the box's tokens in (t, y, x) order.
+struct Box {
+  int t0, y0, x0, st, sh, sw;
+};
+
+__device__ __forceinline__ int video_block_box(const Geo& g, const uint8_t* __restrict__ codes,
+                                               int b, int t, Box& bx) {
+  const int jv = t - g.nbp;
+  if (g.mode == BSA_BLOCK_FIXED_444) {
+    const int nbh = g.H >> 2, nbw = g.W >> 2;
+    const int bt = jv / (nbh * nbw), rem = jv - bt * (nbh * nbw);
+    const int bhh = rem / nbw;
+    bx = {4 * bt, 4 * bhh, 4 * (rem - bhh * nbw), 4, 4, 4};
+    return 0;
+  }
+  const int r = jv >> 3, sub = jv & 7;
+  const int nrh = g.H >> 3, nrw = g.W >> 3;
+  const int rt = r / (nrh * nrw), rem = r - rt * (nrh * nrw);
+  const int rh = rem / nrw, rw = rem - rh * nrw;
+  int code = __ldg(codes + int64_t(b) * g.nreg + r);
+  code = code > 6 ? 0 : code;
+  int st, sh, sw;
+  shape_sides(code, st, sh, sw);
+  const int gh = 8 / sh, gw = 8 / sw;
+  const int bt = sub / (gh * gw), bhh = (sub / gw) % gh, bw = sub % gw;
+  bx = {8 * rt + st * bt, 8 * rh + sh * bhh, 8 * rw + sw * bw, st, sh, sw};
+  return code;
+}
+
+// One K (or V) copy: box bx (64 head_dim columns) of key block t of
+// (batch, head) bh into shared memory at dst.  Block order: one 3-D box of
+// the permuted tensor.  Raster order: a prefix block is 64 consecutive
+// tokens (3-D map over [B, N, heads*d]); a video block is one 5-D box
+// {64 columns, sw, sh, st, 1} of the [B, T, H, W, heads*d] grid whose rows
+// land in shared memory in (t, y, x) order, i.e. in slot order, so the
+// shared-memory tile is the same as the permuted one.
+template <int D, bool RASTER>
+__device__ __forceinline__ void kv_copy(uint32_t dst, const KVMaps<RASTER>& maps, bool is_k,
+                                        uint32_t bar, int bx, int t, int bh, const Geo& g,
+                                        const uint8_t* __restrict__ codes) {
+  if constexpr (!RASTER) {
+    tma_load_3d(dst, is_k ? &maps.k : &maps.v, bar, 64 * bx, t * 64, bh);
+  } else {
+    const int b = bh / g.h, c0 = (bh - b * g.h) * D + 64 * bx;
+    const CUtensorMap* m = is_k ? maps.k : maps.v;
+    if (t < g.nbp) {
+      tma_load_3d(dst, m, bar, c0, t * 64, b);
+      return;
+    }
+    Box box;
+    const int code = video_block_box(g, codes, b, t, box);
+    tma_load_5d(dst, m + 1 + code, bar, c0, box.x0, box.y0, box.t0, b);
+  }
+}
+
+// ---- window heads ------------------------------------------------------------
+// A window head (Sparse VideoGen on TPU, aibase.it, section "Sparse
+// VideoGen의 핵심 아이디어": spatial heads look within nearby frames,
+// temporal heads at the same place across frames) lets query token
+// (t, y, x) see video key (t', y', x') when |t' - t| <= w_t, |y' - y| <= w_y
+// and |x' - x| <= w_x, a negative w leaving that axis free; prefix keys and
+// prefix queries stay dense.  A tile is empty when, on some axis, the two
+// blocks' extents are farther apart than the window (skipped: not in the
+// walk), full when every pair is inside, boundary otherwise (an element mask
+// per query row, built from the key block's box).
+
+// 1 when some pair of the extents [a0, a0+la) and [b0, b0+lb) is within w
+__device__ __forceinline__ bool axis_reach(int a0, int la, int b0, int lb, int w) {
+  if (w < 0) return true;
+  const int gap = max(0, max(b0 - (a0 + la - 1), a0 - (b0 + lb - 1)));
+  return gap <= w;
+}
+
+// bits [lo, hi) of a 64-bit word (0 when lo >= hi)
+__device__ __forceinline__ uint64_t bit_range(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 64);
+  if (lo >= hi) return 0ull;
+  const uint64_t up = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
+  return up & ~((1ull << lo) - 1ull);
+}
+
+// slots s of a key block whose coordinate along one axis, k0 + (s / inner)
+// % side, lies in [q - w, q + w]: a run of `inner`-wide groups repeated with
+// period inner*side (a divisor of 64)
+__device__ __forceinline__ uint64_t axis_bits(int q, int w, int k0, int side, int inner) {
+  if (w < 0) return ~0ull;
+  const int lo = max(q - w - k0, 0), hi = min(q + w - k0, side - 1);
+  if (lo > hi) return 0ull;
+  const int period = inner * side;
+  const uint64_t one = bit_range(lo * inner, (hi + 1) * inner);
+  const uint64_t comb = period >= 64 ? 1ull : (~0ull / ((1ull << period) - 1ull));
+  return one * comb;
+}
+
+// element mask of one query row (video token at tq, yq, xq) for a video key block
+__device__ __forceinline__ uint64_t window_bits(const Box& k, int tq, int yq, int xq, int wt,
+                                                int wy, int wx) {
+  return axis_bits(tq, wt, k.t0, k.st, k.sh * k.sw) & axis_bits(yq, wy, k.y0, k.sh, k.sw) &
+         axis_bits(xq, wx, k.x0, k.sw, 1);
+}
+
+// what decides a CTA's walk: index lists, every block, or per-head windows
+enum { kModeLists = 0, kModeDense = 1, kModeWindow = 2 };
+
+template <int D, int MODE, bool RASTER>
 __global__ void __launch_bounds__(512, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-                    Geo g, const __nv_bfloat16* __restrict__ qperm,
-                    const uint64_t* __restrict__ bmask, const uint8_t* __restrict__ bfull,
-                    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
-                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ status) {
+    attn_fwd_kernel(const __grid_constant__ KVMaps<RASTER> maps, Geo g, const AttnIO io) {
   using C = Cfg<D>;
+  const uint64_t* __restrict__ bmask = io.bmask;
+  const uint8_t* __restrict__ bfull = io.bfull;
+  const int32_t* __restrict__ idx = io.idx;
+  const int32_t* __restrict__ cnt = io.cnt;
+  int32_t* __restrict__ status = io.status;
   constexpr int KS = C::KS, VS = C::VS;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -195,7 +303,31 @@ __global__ void __launch_bounds__(512, 1)
         const int qb = 2 * pair + hf;
         if (qb >= g.nb) continue;
         uint32_t* bm = hf ? bmB : bmA;
-        const int c = DENSE ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
+        if constexpr (MODE == kModeWindow) {
+          // a video query block walks the prefix and every video key block
+          // its box can reach through the window (non-empty tiles)
+          if (qb >= g.nbp) {
+            const int32_t* win = io.windows + 3 * (bh - b * g.h);
+            const int wt = __ldg(win), wy = __ldg(win + 1), wx = __ldg(win + 2);
+            Box qx;
+            video_block_box(g, io.codes, b, qb, qx);
+            for (int w = 0; w < nw; ++w) {
+              const int j = 32 * w + lane;
+              bool on = j < g.nbp;
+              if (j >= g.nbp && j < g.nb) {
+                Box kx;
+                video_block_box(g, io.codes, b, j, kx);
+                on = axis_reach(qx.t0, qx.st, kx.t0, kx.st, wt) &&
+                     axis_reach(qx.y0, qx.sh, kx.y0, kx.sh, wy) &&
+                     axis_reach(qx.x0, qx.sw, kx.x0, kx.sw, wx);
+              }
+              const uint32_t word = __ballot_sync(0xffffffffu, on);
+              if (lane == 0) bm[w] = word;
+            }
+            continue;
+          }
+        }
+        const int c = MODE != kModeLists ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
         if (c < 0) {
           for (int w = lane; w < nw; w += 32) {
             const int rem = g.nb - 32 * w;
@@ -271,10 +403,7 @@ __global__ void __launch_bounds__(512, 1)
     const int par = is_k ? ((warp == 8 || warp == 11) ? 0 : 1) : 0;
     const int stride = is_k ? 2 : 1;
     if (lane == 0 && bx < C::KB) {
-      if (is_k)
-        tma_prefetch_desc(&mk);
-      else
-        tma_prefetch_desc(&mv);
+      if constexpr (!RASTER) tma_prefetch_desc(is_k ? &maps.k : &maps.v);
       const int RS = is_k ? KS : VS;
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
       const int n = ok ? *n_steps_sm : 0;
@@ -290,10 +419,8 @@ __global__ void __launch_bounds__(512, 1)
         const int t = int(steps[j] & kTileMask);
         // box bx of the block: [box][row][64] in the stage
         mbar_arrive_expect_tx(ful, C::BOX);
-        if (is_k)
-          tma_load_3d(sK + (bx * KS + s) * C::BOX, &mk, ful, 64 * bx, t * 64, bh);
-        else
-          tma_load_3d(sV + s * C::BLK_BYTES + bx * C::BOX, &mv, ful, 64 * bx, t * 64, bh);
+        kv_copy<D, RASTER>(is_k ? sK + (bx * KS + s) * C::BOX : sV + s * C::BLK_BYTES + bx * C::BOX,
+                           maps, is_k, ful, bx, t, bh, g, io.codes);
       }
       if (!ok) report_timeout(abort_flag, status);
       // On any abort (this warp's own wait or another role's), the consumers
@@ -391,8 +518,20 @@ __global__ void __launch_bounds__(512, 1)
       // Q rows into tensor memory (A operand of S = Q K^T), bf16 pairs per column
       uint32_t qr[D / 2];
       const int64_t qrow = int64_t(pair) * 128 + row;
+      const __nv_bfloat16* qsrc = nullptr;
       if (qrow < g.N) {
-        const uint4* src = reinterpret_cast<const uint4*>(qperm + (int64_t(bh) * g.N + qrow) * D);
+        if constexpr (RASTER) {
+          // the slot's raster token; pad slots read nothing (their rows are
+          // zero and their outputs are written as 0)
+          const uint32_t pr = uint32_t(__ldg(io.perm + int64_t(b) * g.N + qrow));
+          if (!(pr & 0x80000000u))
+            qsrc = io.q + int64_t(b) * io.qsb + int64_t(pr) * io.qsn + int64_t(bh - b * g.h) * io.qsh;
+        } else {
+          qsrc = io.q + (int64_t(bh) * g.N + qrow) * D;
+        }
+      }
+      if (qsrc) {
+        const uint4* src = reinterpret_cast<const uint4*>(qsrc);
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) {
           const uint4 u = __ldg(src + i);
@@ -423,6 +562,26 @@ __global__ void __launch_bounds__(512, 1)
     // this group's steps are every other entry of the step table.  Barrier
     // probes are issued ahead of independent work so that their latency
     // (~170 cycles even for a completed phase) overlaps it.
+    // window heads: this row's grid coordinates and its head's window
+    struct {
+      bool video;
+      int tq, yq, xq, wt, wy, wx;
+    } win = {false, 0, 0, 0, -1, -1, -1};
+    if constexpr (MODE == kModeWindow) {
+      if (q_exists && qb >= g.nbp) {
+        const int v = int(uint32_t(__ldg(io.perm + int64_t(b) * g.N + int64_t(qb) * 64 +
+                                         (row & 63))) & 0x7FFFFFFFu) - g.P;
+        const int hw = g.H * g.W;
+        win.video = true;
+        win.tq = v / hw;
+        win.yq = (v - win.tq * hw) / g.W;
+        win.xq = v - win.tq * hw - win.yq * g.W;
+        const int32_t* w3 = io.windows + 3 * (bh - b * g.h);
+        win.wt = __ldg(w3);
+        win.wy = __ldg(w3 + 1);
+        win.wx = __ldg(w3 + 2);
+      }
+    }
     ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
     const int n = ok ? *n_steps_sm : 0;
     const uint64_t* bm_row = bmask + int64_t(b) * g.nb;
@@ -446,8 +605,18 @@ __global__ void __launch_bounds__(512, 1)
         BSA_TMEM_LD64(tS, r);
         tc_fence_before();
         mbar_arrive(bar_sfree);
-        const bool all_valid = (flags & 4u) != 0u;
-        const uint64_t vm = all_valid ? ~0ull : __ldg(bm_row + tile);
+        bool all_valid = (flags & 4u) != 0u;
+        uint64_t vm = all_valid ? ~0ull : __ldg(bm_row + tile);
+        if constexpr (MODE == kModeWindow) {
+          // the row's element mask for this key block (boundary tiles);
+          // prefix rows and prefix keys are dense
+          if (win.video && tile >= g.nbp) {
+            Box kx;
+            video_block_box(g, io.codes, b, tile, kx);
+            vm &= window_bits(kx, win.tq, win.yq, win.xq, win.wt, win.wy, win.wx);
+          }
+          all_valid = __all_sync(0xffffffffu, vm == ~0ull);
+        }
         const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (all_valid) {
@@ -542,7 +711,19 @@ __global__ void __launch_bounds__(512, 1)
       const float l = l0 * a0 + l1 * a1;
       const float inv = (row_valid && l > 0.f) ? 1.f / l : 0.f;
       const float f0 = a0 * inv, f1 = a1 * inv;
-      __nv_bfloat16* orow = out + (int64_t(bh) * g.N + int64_t(qb) * 64 + (row & 63)) * D;
+      // the row's log-sum-exp in the exp2 domain, for the backward
+      // (P = exp2(s * scale * log2(e) - lse2)); +inf for pad rows
+      if (io.lse && wg == 0)
+        io.lse[int64_t(bh) * g.N + int64_t(qb) * 64 + (row & 63)] =
+            (row_valid && l > 0.f) ? m + __log2f(l) : INFINITY;
+      __nv_bfloat16* orow;
+      if constexpr (RASTER) {
+        const int64_t slot = int64_t(qb) * 64 + (row & 63);
+        const int64_t pr = int64_t(uint32_t(__ldg(io.perm + int64_t(b) * g.N + slot)) & 0x7FFFFFFFu);
+        orow = io.o + int64_t(b) * io.osb + pr * io.osn + int64_t(bh - b * g.h) * io.osh;
+      } else {
+        orow = io.o + (int64_t(bh) * g.N + int64_t(qb) * 64 + (row & 63)) * D;
+      }
       // group wg writes columns [wg*D/2, (wg+1)*D/2)
 #pragma unroll
       for (int ch = 0; ch < D / 64; ++ch) {
@@ -575,30 +756,36 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
-template <int D, bool DENSE>
-cudaError_t launch_t(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps,
-                     const __nv_bfloat16* qp, const int32_t* idx, const int32_t* cnt,
-                     __nv_bfloat16* o, int32_t* status, cudaStream_t st) {
+template <int D, int MODE, bool RASTER>
+cudaError_t launch_t(const Geo& g, const KVMaps<RASTER>& maps, const AttnIO& io, cudaStream_t st) {
   using C = Cfg<D>;
-  auto kern = attn_fwd_kernel<D, DENSE>;
+  auto kern = attn_fwd_kernel<D, MODE, RASTER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((g.nb + 1) / 2, g.B * g.h);
-  kern<<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], g, qp, lp.bmask, lp.bfull, idx, cnt, o,
-                                           status);
+  kern<<<grid, C::kThreads, C::SMEM, st>>>(maps, g, io);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attention(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps,
-                             const __nv_bfloat16* qp, const int32_t* idx, const int32_t* cnt,
-                             __nv_bfloat16* o, int32_t* dev_status, bool dense, cudaStream_t st) {
+cudaError_t launch_attention(const Geo& g, const KVMaps<false>& maps, const AttnIO& io,
+                             bool dense, cudaStream_t st) {
   if (g.d == 128)
-    return dense ? launch_t<128, true>(g, lp, maps, qp, idx, cnt, o, dev_status, st)
-                 : launch_t<128, false>(g, lp, maps, qp, idx, cnt, o, dev_status, st);
-  return dense ? launch_t<64, true>(g, lp, maps, qp, idx, cnt, o, dev_status, st)
-               : launch_t<64, false>(g, lp, maps, qp, idx, cnt, o, dev_status, st);
+    return dense ? launch_t<128, kModeDense, false>(g, maps, io, st)
+                 : launch_t<128, kModeLists, false>(g, maps, io, st);
+  return dense ? launch_t<64, kModeDense, false>(g, maps, io, st)
+               : launch_t<64, kModeLists, false>(g, maps, io, st);
+}
+
+cudaError_t launch_attention_raster(const Geo& g, const KVMaps<true>& maps, const AttnIO& io,
+                                    cudaStream_t st) {
+  if (io.windows) {
+    if (g.d == 128) return launch_t<128, kModeWindow, true>(g, maps, io, st);
+    return launch_t<64, kModeWindow, true>(g, maps, io, st);
+  }
+  if (g.d == 128) return launch_t<128, kModeLists, true>(g, maps, io, st);
+  return launch_t<64, kModeLists, true>(g, maps, io, st);
 }
 
 }  // namespace bsa

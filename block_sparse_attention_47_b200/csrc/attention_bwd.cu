@@ -1,0 +1,672 @@
+// Backward of the block-sparse attention on sm_100a: gradients dQ, dK, dV
+// over the same kept 64x64 tiles as the forward (Prism / Kandinsky 6 speed
+// ablation, oh-my-gpu.com, section "같은 계산량 안에서 볼 곳을 고르는 Prism":
+// the sparse attention also trains, a 2K step going from 26.5 to 10.6
+// minutes).  With P = exp2(S * scale * log2(e) - lse2) recomputed from the
+// forward's per-row log-sum-exp (exp2 domain) and D = rowsum(dO * O):
+//     dP = dO V^T,  dS = P * (dP - D),
+//     dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
+//
+// Two kernels, both tcgen05 with the accumulators in tensor memory and the
+// tiles in 128-byte-swizzled shared memory:
+//   dQ   CTA = two adjacent query blocks (128 rows, as the forward), walking
+//        the union of their key lists; per step S and dP (two SS MMAs,
+//        M=128 N=64), dS from them in registers, then dQ += dS K (A = dS in
+//        tensor memory, B = the same K tile read N-major).
+//   dKdV CTA = two adjacent key blocks (128 key rows), walking the union of
+//        the query blocks that kept them (transposed lists, built as
+//        bitmaps); per step S^T = K Q^T and dP^T = V dO^T (M=128 N=64), P^T
+//        and dS^T in registers, then dV += P^T dO and dK += dS^T Q.
+// One thread issues the copies and MMAs in step order; the 128 row threads
+// turn each step's S/dP into P/dS.  K/V (dQ) or Q/dO (dKdV) tiles are
+// double-buffered so the next step's copies run under the current step.
+// Every wait is bounded (2 s) and reports BSA_ERR_TIMEOUT as the forward.
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kMaxWords = kAttnMaxBlocks / 32;
+constexpr uint32_t kTileMask = 0x1FFFu, kFlagShift = 13;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kThreads = 256;             // warps 0-3 rows, 4 issuer, 5-7 idle
+  static constexpr int KB = D / 64;                // 64-column boxes
+  static constexpr int TILE64 = 64 * D * 2;        // one 64-row tile
+  static constexpr int TILE128 = 128 * D * 2;      // the CTA's own 128-row tile
+  static constexpr int BOX64 = 64 * 128, BOX128 = 128 * 128;
+  // dQ: own = Q | dO (128 rows each); stages = K | V (64 rows) x 2
+  // dKdV: own = K | V; stages = Q | dO x 2, plus lse2 | delta (64 floats) x 2
+  static constexpr int OFF_OWN_A = 0;
+  static constexpr int OFF_OWN_B = TILE128;
+  static constexpr int OFF_STG = 2 * TILE128;             // [stage][a | b] 64-row tiles
+  static constexpr int OFF_VEC = OFF_STG + 4 * TILE64;    // [stage][lse2 | delta][64] fp32
+  static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * 64 * 4;
+  // full[2] empty[2] mma1 ready own steps done drain
+  static constexpr int N_BARS = 10;
+  static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;     // uint32 A, B, F [kMaxWords]
+  static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
+  static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // tensor memory: S [0,64) | dP [64,128) | P or dS [128,160) | dS [160,192)
+  // | accumulators from 256 (dQ; or dV then dK)
+  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_X = 128, COL_Y = 160, COL_ACC = 256;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+__device__ __forceinline__ void report_timeout(volatile int* abort_flag, int32_t* status) {
+  *abort_flag = 1;
+  atomicCAS(status, 0, int32_t(BSA_ERR_TIMEOUT));
+}
+
+__device__ __forceinline__ bool bit_of(uint32_t lo, uint32_t hi, int c) {
+  return ((c < 32 ? (lo >> c) : (hi >> (c - 32))) & 1u) != 0u;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// The step table of one CTA (run by one warp): bitmaps A and B over the
+// walked blocks, their union expanded in ascending order into 16-bit
+// entries (block index, bit 13: A has it, bit 14: B has it, bit 15: the
+// block is full).  Returns the number of steps (all lanes).
+__device__ __forceinline__ int build_steps(const uint32_t* bmA, const uint32_t* bmB,
+                                           const uint32_t* bmF, int nw, uint16_t* steps,
+                                           int lane) {
+  int nsteps = 0;
+  for (int r0 = 0; r0 < nw; r0 += 32) {
+    const int w = r0 + lane;
+    const uint32_t a = w < nw ? bmA[w] : 0u, bb = w < nw ? bmB[w] : 0u;
+    const uint32_t f = w < nw ? bmF[w] : 0u;
+    uint32_t u = a | bb;
+    const int c = __popc(u);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int at = nsteps + incl - c;
+    while (u) {
+      const int bit = __ffs(u) - 1;
+      u &= u - 1u;
+      steps[at++] = uint16_t(uint32_t(32 * w + bit) | (((a >> bit) & 1u) << kFlagShift) |
+                             (((bb >> bit) & 1u) << (kFlagShift + 1)) |
+                             (((f >> bit) & 1u) << (kFlagShift + 2)));
+    }
+    nsteps += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return nsteps;
+}
+
+// rows r of a [rows x D] bf16 tile into 128-byte-swizzled 64-column boxes
+__device__ __forceinline__ void store_row_swizzled(uint32_t tile, int box_bytes, int r,
+                                                   const __nv_bfloat16* src, int D) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  for (int i = 0; i < D / 8; ++i) {
+    const uint4 u = src ? __ldg(s + i) : make_uint4(0u, 0u, 0u, 0u);
+    st_shared_v4(tile + (i >> 3) * box_bytes + r * 128 + (((i & 7) ^ (r & 7)) << 4), u);
+  }
+}
+
+// ============================================================================
+// dQ: CTA = query pair, walk = union of the two key lists
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                       Geo g, const BwdIO io) {
+  using C = BwdCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sm = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::OFF_OWN_A, sdO = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
+  const uint32_t bar0 = base + C::OFF_BAR;
+  const uint32_t bar_full = bar0, bar_empty = bar0 + 16, bar_mma1 = bar0 + 32;
+  const uint32_t bar_ready = bar0 + 40, bar_own = bar0 + 48, bar_steps = bar0 + 56;
+  const uint32_t bar_done = bar0 + 64, bar_drain = bar0 + 72;
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
+  uint32_t* bmB = bmA + kMaxWords;
+  uint32_t* bmF = bmA + 2 * kMaxWords;
+  uint16_t* steps = reinterpret_cast<uint16_t*>(sm + C::OFF_STEPS);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
+  int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
+  auto stage_a = [&](int s) { return sStg + s * 2 * C::TILE64; };  // K
+  auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // V
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_mma1, 1);
+    mbar_init(bar_ready, 128);
+    mbar_init(bar_own, 128);
+    mbar_init(bar_steps, 32);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nw = (g.nb + 31) >> 5;
+
+  if (warp == 5) {
+    // ---- the walk: union of the two query blocks' key lists (a dense row
+    // keeps every block); bmF marks key blocks without pad slots
+    for (int w = lane; w < nw; w += 32) bmA[w] = bmB[w] = 0u;
+    __syncwarp();
+    for (int hf = 0; hf < 2; ++hf) {
+      const int qb = 2 * pair + hf;
+      if (qb >= g.nb) continue;
+      uint32_t* bm = hf ? bmB : bmA;
+      const int c = __ldg(io.cnt + int64_t(bh) * g.nb + qb);
+      if (c < 0) {
+        for (int w = lane; w < nw; w += 32) {
+          const int rem = g.nb - 32 * w;
+          bm[w] = rem >= 32 ? ~0u : ((1u << rem) - 1u);
+        }
+      } else {
+        const int n = c < g.kcap ? c : g.kcap;
+        const int32_t* src = io.idx + (int64_t(bh) * g.nb + qb) * g.kcap;
+        for (int i = lane; i < n; i += 32) {
+          const int v = __ldg(src + i);
+          if (v >= 0 && v < g.nb) atomicOr(bm + (v >> 5), 1u << (v & 31));
+        }
+      }
+    }
+    for (int w = lane; w < nw; w += 32) {
+      uint32_t f = 0u;
+      for (int i = 0; i < 32; ++i)
+        if (32 * w + i < g.nb && __ldg(io.bfull + int64_t(b) * g.nb + 32 * w + i)) f |= 1u << i;
+      bmF[w] = f;
+    }
+    __syncwarp();
+    const int n = build_steps(bmA, bmB, bmF, nw, steps, lane);
+    if (lane == 0) *n_steps_sm = n;
+    __syncwarp();
+    mbar_arrive(bar_steps);
+  } else if (warp == 4) {
+    // ---- the issuer: copies and MMAs in step order
+    if (lane == 0) {
+      constexpr uint32_t idesc_sn = idesc_bf16_f32(128, 64, false);  // S, dP: B K-major
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);   // dQ: B N-major
+      tma_prefetch_desc(&mk);
+      tma_prefetch_desc(&mv);
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0;
+      auto load = [&](int j) {
+        const int s = j & 1, t = int(steps[j] & kTileMask);
+        mbar_arrive_expect_tx(bar_full + 8 * s, 2 * C::TILE64);
+        for (int bx = 0; bx < C::KB; ++bx) {
+          tma_load_3d(stage_a(s) + bx * C::BOX64, &mk, bar_full + 8 * s, 64 * bx, t * 64, bh);
+          tma_load_3d(stage_b(s) + bx * C::BOX64, &mv, bar_full + 8 * s, 64 * bx, t * 64, bh);
+        }
+      };
+      for (int j = 0; j < n && j < 2; ++j) load(j);
+      ok = ok && mbar_wait(bar_own, 0, abort_flag);
+      int j = 0;
+      for (; ok && j < n; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(bar_full + 8 * s, (j >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
+          const uint32_t offo = (kk / 4) * C::BOX128 + (kk % 4) * 32;
+          tc_mma_ss(tmem + C::COL_S, sdesc_sw128(sQ + offo, 16, 1024),
+                    sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
+          tc_mma_ss(tmem + C::COL_DP, sdesc_sw128(sdO + offo, 16, 1024),
+                    sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
+        }
+        tc_commit(bar_mma1);
+        if (!mbar_wait(bar_ready, j & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dQ += dS K: A = dS (tensor memory), B = K as [keys x D] read N-major
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_X + 8u * kk,
+                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar_empty + 8 * s);
+        if (j + 2 < n) {
+          if (!mbar_wait(bar_empty + 8 * s, (j >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          load(j + 2);
+        }
+      }
+      if (!ok) {
+        report_timeout(abort_flag, io.status);
+        // copies that may still be in flight: the steps loaded but not used
+        for (int jj = j; jj < n && jj < j + 2; ++jj)
+          mbar_wait(bar_full + 8 * (jj & 1), (jj >> 1) & 1, nullptr, 200000000ull);
+      }
+      tc_commit(bar_done);
+      tc_commit(bar_drain);
+      mbar_wait(bar_drain, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---- row threads: row r of the pair = TMEM lane r
+    const int row = threadIdx.x, half = row >> 6, qb = 2 * pair + half;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const bool q_exists = qb < g.nb;
+    const int64_t slot = int64_t(pair) * 128 + row;
+    const bool row_valid =
+        q_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + qb) >> (row & 63)) & 1ull);
+    const int64_t prow = int64_t(bh) * g.N + slot;
+    // Q and dO rows into shared memory (A operands of S and dP)
+    store_row_swizzled(sQ, C::BOX128, row, q_exists ? io.q + prow * D : nullptr, D);
+    store_row_swizzled(sdO, C::BOX128, row, row_valid ? io.dout + prow * D : nullptr, D);
+    fence_proxy_async_smem();
+    mbar_arrive(bar_own);
+    const float lse2 = row_valid ? __ldg(io.lse + prow) : INFINITY;
+    const float dlt = row_valid ? __ldg(io.delta + prow) : 0.f;
+    const float sl2 = g.scale * 1.4426950408889634f;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const int n = ok ? *n_steps_sm : 0;
+    for (int j = 0; ok && j < n; ++j) {
+      const uint32_t entry = steps[j];
+      const int tile = int(entry & kTileMask);
+      const uint32_t flags = entry >> kFlagShift;
+      const bool member = row_valid && ((flags >> half) & 1u);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_mma1, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64], dp[64], pk[32];
+      BSA_TMEM_LD64(tmem + C::COL_S + lane_base, sv);
+      BSA_TMEM_LD64(tmem + C::COL_DP + lane_base, dp);
+      const uint64_t vm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
+      const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float d0 = 0.f, d1 = 0.f;
+        if (member) {
+          const float p0 =
+              bit_of(lo, hi, c) ? ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2)) : 0.f;
+          const float p1 = bit_of(lo, hi, c + 1)
+                               ? ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2))
+                               : 0.f;
+          d0 = p0 * (__uint_as_float(dp[c]) - dlt);
+          d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt);
+        }
+        pk[c / 2] = pack_bf16x2(d0, d1);
+      }
+      BSA_TMEM_ST32(tmem + C::COL_X + lane_base, pk);
+      tc_fence_before();
+      mbar_arrive(bar_ready);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag));
+    if (!ok) {
+      if (lane == 0) report_timeout(abort_flag, io.status);
+    } else if (q_exists) {
+      tc_fence_after();
+      __nv_bfloat16* dst = io.dq + prow * D;
+      const bool live = row_valid && n > 0;  // no steps: the accumulator was never written
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t a[32];
+        BSA_TMEM_LD32(tmem + C::COL_ACC + 32u * ch + lane_base, a);
+        uint32_t w16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w16[i] = pack_bf16x2(live ? __uint_as_float(a[2 * i]) * g.scale : 0.f,
+                               live ? __uint_as_float(a[2 * i + 1]) * g.scale : 0.f);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          d4[i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// dK, dV: CTA = key pair, walk = union of the query blocks that kept them
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq,
+                         const __grid_constant__ CUtensorMap mdo, Geo g, const BwdIO io) {
+  using C = BwdCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sm = smem_raw + (base - raw);
+  const uint32_t sK = base + C::OFF_OWN_A, sV = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
+  const uint32_t sVec = base + C::OFF_VEC;
+  const float* vec = reinterpret_cast<const float*>(sm + C::OFF_VEC);
+  const uint32_t bar0 = base + C::OFF_BAR;
+  const uint32_t bar_full = bar0, bar_empty = bar0 + 16, bar_mma1 = bar0 + 32;
+  const uint32_t bar_ready = bar0 + 40, bar_own = bar0 + 48, bar_steps = bar0 + 56;
+  const uint32_t bar_done = bar0 + 64, bar_drain = bar0 + 72;
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
+  uint32_t* bmB = bmA + kMaxWords;
+  uint32_t* bmF = bmA + 2 * kMaxWords;
+  uint16_t* steps = reinterpret_cast<uint16_t*>(sm + C::OFF_STEPS);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
+  int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
+  auto stage_a = [&](int s) { return sStg + s * 2 * C::TILE64; };  // Q
+  auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // dO
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_mma1, 1);
+    mbar_init(bar_ready, 128);
+    mbar_init(bar_own, 128);
+    mbar_init(bar_steps, 32);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nw = (g.nb + 31) >> 5;
+
+  if (warp == 5) {
+    // ---- the walk: query blocks that kept key block 2*pair (A) or
+    // 2*pair + 1 (B), from the transposed bitmaps; bmF marks query blocks
+    // without pad slots
+    const uint32_t* kt = io.kmask + (int64_t(bh) * g.nb) * nw;
+    for (int w = lane; w < nw; w += 32) {
+      bmA[w] = 2 * pair < g.nb ? __ldg(kt + int64_t(2 * pair) * nw + w) : 0u;
+      bmB[w] = 2 * pair + 1 < g.nb ? __ldg(kt + int64_t(2 * pair + 1) * nw + w) : 0u;
+      uint32_t f = 0u;
+      for (int i = 0; i < 32; ++i)
+        if (32 * w + i < g.nb && __ldg(io.bfull + int64_t(b) * g.nb + 32 * w + i)) f |= 1u << i;
+      bmF[w] = f;
+    }
+    __syncwarp();
+    const int n = build_steps(bmA, bmB, bmF, nw, steps, lane);
+    if (lane == 0) *n_steps_sm = n;
+    __syncwarp();
+    mbar_arrive(bar_steps);
+  } else if (warp == 4) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_sn = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
+      tma_prefetch_desc(&mq);
+      tma_prefetch_desc(&mdo);
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0;
+      auto load = [&](int j) {
+        const int s = j & 1, t = int(steps[j] & kTileMask);
+        const int64_t r0 = int64_t(bh) * g.N + int64_t(t) * 64;
+        mbar_arrive_expect_tx(bar_full + 8 * s, 2 * C::TILE64 + 2 * 256);
+        for (int bx = 0; bx < C::KB; ++bx) {
+          tma_load_3d(stage_a(s) + bx * C::BOX64, &mq, bar_full + 8 * s, 64 * bx, t * 64, bh);
+          tma_load_3d(stage_b(s) + bx * C::BOX64, &mdo, bar_full + 8 * s, 64 * bx, t * 64, bh);
+        }
+        bulk_load(sVec + s * 512, io.lse + r0, 256, bar_full + 8 * s);
+        bulk_load(sVec + s * 512 + 256, io.delta + r0, 256, bar_full + 8 * s);
+      };
+      for (int j = 0; j < n && j < 2; ++j) load(j);
+      ok = ok && mbar_wait(bar_own, 0, abort_flag);
+      int j = 0;
+      for (; ok && j < n; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(bar_full + 8 * s, (j >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
+          const uint32_t offo = (kk / 4) * C::BOX128 + (kk % 4) * 32;
+          tc_mma_ss(tmem + C::COL_S, sdesc_sw128(sK + offo, 16, 1024),
+                    sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
+          tc_mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offo, 16, 1024),
+                    sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
+        }
+        tc_commit(bar_mma1);
+        if (!mbar_wait(bar_ready, j & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dV += P^T dO and dK += dS^T Q (A from tensor memory, B N-major)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_X + 8u * kk,
+                    sdesc_sw128(stage_b(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + C::COL_ACC + D, tmem + C::COL_Y + 8u * kk,
+                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar_empty + 8 * s);
+        if (j + 2 < n) {
+          if (!mbar_wait(bar_empty + 8 * s, (j >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          load(j + 2);
+        }
+      }
+      if (!ok) {
+        report_timeout(abort_flag, io.status);
+        for (int jj = j; jj < n && jj < j + 2; ++jj)
+          mbar_wait(bar_full + 8 * (jj & 1), (jj >> 1) & 1, nullptr, 200000000ull);
+      }
+      tc_commit(bar_done);
+      tc_commit(bar_drain);
+      mbar_wait(bar_drain, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---- row threads: key row r of the pair = TMEM lane r
+    const int row = threadIdx.x, half = row >> 6, kb = 2 * pair + half;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const bool k_exists = kb < g.nb;
+    const int64_t prow = int64_t(bh) * g.N + int64_t(pair) * 128 + row;
+    const bool key_valid =
+        k_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + kb) >> (row & 63)) & 1ull);
+    store_row_swizzled(sK, C::BOX128, row, k_exists ? io.k + prow * D : nullptr, D);
+    store_row_swizzled(sV, C::BOX128, row, k_exists ? io.v + prow * D : nullptr, D);
+    fence_proxy_async_smem();
+    mbar_arrive(bar_own);
+    const float sl2 = g.scale * 1.4426950408889634f;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const int n = ok ? *n_steps_sm : 0;
+    for (int j = 0; ok && j < n; ++j) {
+      const uint32_t entry = steps[j];
+      const int tile = int(entry & kTileMask);
+      const uint32_t flags = entry >> kFlagShift;
+      const bool member = key_valid && ((flags >> half) & 1u);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_mma1, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64], dp[64], pk[32], dk[32];
+      BSA_TMEM_LD64(tmem + C::COL_S + lane_base, sv);
+      BSA_TMEM_LD64(tmem + C::COL_DP + lane_base, dp);
+      // query slots of block `tile`: real tokens only (pad queries have no output)
+      const uint64_t qm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
+      const uint32_t lo = uint32_t(qm), hi = uint32_t(qm >> 32);
+      const float* lse = vec + (j & 1) * 128;
+      const float* dlt = lse + 64;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+        if (member) {
+          if (bit_of(lo, hi, c)) {
+            p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse[c]));
+            d0 = p0 * (__uint_as_float(dp[c]) - dlt[c]);
+          }
+          if (bit_of(lo, hi, c + 1)) {
+            p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse[c + 1]));
+            d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt[c + 1]);
+          }
+        }
+        pk[c / 2] = pack_bf16x2(p0, p1);
+        dk[c / 2] = pack_bf16x2(d0, d1);
+      }
+      BSA_TMEM_ST32(tmem + C::COL_X + lane_base, pk);
+      BSA_TMEM_ST32(tmem + C::COL_Y + lane_base, dk);
+      tc_fence_before();
+      mbar_arrive(bar_ready);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag));
+    if (!ok) {
+      if (lane == 0) report_timeout(abort_flag, io.status);
+    } else if (k_exists) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
+        __nv_bfloat16* dst = (which ? io.dk : io.dv) + prow * D;
+        const float f = which ? g.scale : 1.f;
+        // a key block no query kept has no steps and zero gradients (its
+        // accumulators were never written)
+        const bool live = key_valid && n > 0;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t a[32];
+          BSA_TMEM_LD32(tmem + C::COL_ACC + uint32_t(which * D) + 32u * ch + lane_base, a);
+          uint32_t w16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w16[i] = pack_bf16x2(live ? __uint_as_float(a[2 * i]) * f : 0.f,
+                                 live ? __uint_as_float(a[2 * i + 1]) * f : 0.f);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// D = rowsum(dO * O) and the transposed (key block -> query blocks) bitmaps
+// ============================================================================
+__global__ void __launch_bounds__(256) bwd_delta_kernel(Geo g, const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ dout,
+                                                        float* __restrict__ delta) {
+  // 8 threads per row, each 16 bytes at a time
+  const int64_t rows = int64_t(g.B) * g.h * g.N;
+  const int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
+  const int sub = threadIdx.x & 7;
+  float acc = 0.f;
+  if (r < rows) {
+    const uint4* po = reinterpret_cast<const uint4*>(o + r * g.d);
+    const uint4* pd = reinterpret_cast<const uint4*>(dout + r * g.d);
+    for (int i = sub; i < g.d / 8; i += 8) {
+      const uint4 a = __ldg(po + i), c = __ldg(pd + i);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 x = __bfloat1622float2(a2[k]), y = __bfloat1622float2(c2[k]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (r < rows && sub == 0) delta[r] = acc;
+}
+
+// kmask[bh][key block j] bit i: query block i keeps j (a dense row keeps all)
+__global__ void __launch_bounds__(256) bwd_transpose_kernel(Geo g, const int32_t* __restrict__ idx,
+                                                            const int32_t* __restrict__ cnt,
+                                                            uint32_t* __restrict__ kmask) {
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int nw = (g.nb + 31) >> 5;
+  uint32_t* km = kmask + int64_t(bh) * g.nb * nw;
+  const uint32_t bit = 1u << (i & 31);
+  const int c = cnt[int64_t(bh) * g.nb + i];
+  if (c < 0) {
+    for (int j = threadIdx.x; j < g.nb; j += blockDim.x) atomicOr(km + int64_t(j) * nw + (i >> 5), bit);
+  } else {
+    const int n = c < g.kcap ? c : g.kcap;
+    const int32_t* src = idx + (int64_t(bh) * g.nb + i) * g.kcap;
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+      const int j = src[e];
+      if (j >= 0 && j < g.nb) atomicOr(km + int64_t(j) * nw + (i >> 5), bit);
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_t(const Geo& g, const CUtensorMap* maps, const BwdIO& io, cudaStream_t st) {
+  using C = BwdCfg<D>;
+  const int nw = (g.nb + 31) >> 5;
+  cudaError_t e = cudaMemsetAsync(io.kmask, 0, sizeof(uint32_t) * size_t(g.B) * g.h * g.nb * nw, st);
+  if (e != cudaSuccess) return e;
+  bwd_transpose_kernel<<<dim3(g.nb, g.B * g.h), 256, 0, st>>>(g, io.idx, io.cnt, io.kmask);
+  const int64_t rows = int64_t(g.B) * g.h * g.N;
+  bwd_delta_kernel<<<unsigned((rows * 8 + 255) / 256), 256, 0, st>>>(g, io.o, io.dout, io.delta);
+  e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((g.nb + 1) / 2, g.B * g.h);
+  attn_bwd_dq_kernel<D><<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], g, io);
+  attn_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::SMEM, st>>>(maps[2], maps[3], g, io);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention_bwd(const Geo& g, const CUtensorMap* maps, const BwdIO& io,
+                                 cudaStream_t st) {
+  return g.d == 128 ? launch_bwd_t<128>(g, maps, io, st) : launch_bwd_t<64>(g, maps, io, st);
+}
+
+}  // namespace bsa

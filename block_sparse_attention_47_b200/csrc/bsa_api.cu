@@ -8,6 +8,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -16,6 +18,16 @@ size_t select_smem_bytes(const Geo& g);
 
 namespace {
 thread_local char g_last_error[512] = "";
+
+// one NVTX range per entry point call (free unless a profiler is attached),
+// so that a timeline shows which library call queued which kernels
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
+#define BSA_RANGE() NvtxRange bsa_nvtx_range_(__func__)
+namespace {
 }
 
 namespace bsa {
@@ -190,6 +202,46 @@ bsa_status make_map(CUtensorMap* m, const Geo& g, const void* ptr, int rows) {
   return BSA_OK;
 }
 
+// Raster K or V [B, N, heads, d] with heads contiguous in a token row
+// (stride_h == d): maps[0] covers the prefix as 64-token boxes of
+// [B, N, heads*d]; maps[1 + code] covers the video grid [B, T, H, W, heads*d]
+// (starting at token P) with one box per block of shape code.
+bsa_status make_raster_maps(CUtensorMap* maps, const Geo& g, const void* ptr, int64_t sb,
+                            int64_t sn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t row = cuuint64_t(g.h) * g.d;  // elements of one token row
+  {
+    cuuint64_t dims[3] = {row, cuuint64_t(g.N), cuuint64_t(g.B)};
+    cuuint64_t strides[2] = {cuuint64_t(sn) * 2, cuuint64_t(sb) * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (raster prefix) failed (%d)", int(r));
+  }
+  void* video = static_cast<char*>(const_cast<void*>(ptr)) + int64_t(g.P) * sn * 2;
+  for (int code = 0; code < 7; ++code) {
+    int st, sh, sw;
+    bsa::shape_sides(code, st, sh, sw);
+    cuuint64_t dims[5] = {row, cuuint64_t(g.W), cuuint64_t(g.H), cuuint64_t(g.T), cuuint64_t(g.B)};
+    cuuint64_t strides[4] = {cuuint64_t(sn) * 2, cuuint64_t(sn) * g.W * 2,
+                             cuuint64_t(sn) * g.W * g.H * 2, cuuint64_t(sb) * 2};
+    cuuint32_t box[5] = {64, cuuint32_t(sw), cuuint32_t(sh), cuuint32_t(st), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(&maps[1 + code], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, video, dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled (raster block shape %d) failed (%d)", code,
+                  int(r));
+    if (g.mode == BSA_BLOCK_FIXED_444) break;  // only the cube is used
+  }
+  return BSA_OK;
+}
+
 bsa_status check_device() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -209,6 +261,23 @@ bsa_status check_device() {
     if (_s != BSA_OK) return _s;   \
   } while (0)
 
+// the caller's status word, or the library's own word of this device
+bsa_status status_word(int32_t** status) {
+  if (*status) return BSA_OK;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(status), g_dev_status_sink);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "cudaGetSymbolAddress(status sink)");
+}
+
+// raster K/V read by TMA boxes: heads contiguous within a token row
+bsa_status check_raster_kv(const Geo& g, int64_t sh, const char* name) {
+  if (sh != g.d)
+    return fail(BSA_ERR_UNSUPPORTED,
+                "%s: the raster attention path reads K and V as boxes of whole token rows and "
+                "needs stride_h == head_dim (got %lld)",
+                name, (long long)sh);
+  return BSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -224,6 +293,7 @@ int32_t bsa_keep_count(int32_t n_blocks, double keep_ratio) {
 
 bsa_status bsa_query_sizes(const bsa_problem* prob, bsa_sizes* out) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   if (!out) return fail(BSA_ERR_INVALID_ARG, "out is NULL");
   Geo g;
   BSA_TRY(make_geo(prob, &g));
@@ -246,6 +316,7 @@ bsa_status bsa_query_sizes(const bsa_problem* prob, bsa_sizes* out) {
 bsa_status bsa_layout(const bsa_problem* prob, const void* k_raster, int64_t stride_b,
                       int64_t stride_n, int64_t stride_h, void* layout_buf, void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(layout_buf, "layout_buf"));
@@ -264,6 +335,7 @@ bsa_status bsa_permute(const bsa_problem* prob, const void* layout_buf, const vo
                        int64_t stride_b, int64_t stride_n, int64_t stride_h, void* x_perm,
                        void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(layout_buf, "layout_buf"));
@@ -281,6 +353,7 @@ bsa_status bsa_permute(const bsa_problem* prob, const void* layout_buf, const vo
 bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void* q_perm,
                     const void* k_perm, float* q_pool, float* k_pool, void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(layout_buf, "layout_buf"));
@@ -296,9 +369,25 @@ bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void*
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_pool launch");
 }
 
+// 2-D map over the pooled keys [B*heads*nb rows, d] fp32 for the TMA-fed
+// score tiles (32 channels x 256 rows per box, 128-byte swizzle); false when
+// the driver offers no encoder (the select kernel then loads the tiles itself)
+static bool make_pool_map(CUtensorMap* m, const Geo& g, const float* k_pool) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(g.d), cuuint64_t(g.B) * g.h * g.nb};
+  cuuint64_t strides[1] = {cuuint64_t(g.d) * 4};
+  cuuint32_t box[2] = {32, 256};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(k_pool), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const float* k_pool,
                            int32_t* idx, int32_t* cnt, void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(q_pool, "q_pool"));
@@ -306,15 +395,40 @@ bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const f
   BSA_TRY(check_ptr4(idx, "idx"));
   BSA_TRY(check_ptr4(cnt, "cnt"));
   BSA_TRY(check_device());
-  cudaError_t e = bsa::launch_select(g, q_pool, k_pool, idx, cnt, static_cast<cudaStream_t>(stream));
+  CUtensorMap kmap;
+  const bool tma = make_pool_map(&kmap, g, k_pool);
+  cudaError_t e = bsa::launch_select(g, q_pool, k_pool, nullptr, tma ? &kmap : nullptr, idx, cnt,
+                                     static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_select_topk launch");
+}
+
+bsa_status bsa_select_topk_gated(const bsa_problem* prob, const float* q_pool,
+                                 const float* k_pool, const float* gate, int32_t* idx,
+                                 int32_t* cnt, void* stream) {
+  g_last_error[0] = 0;
+  BSA_RANGE();
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(q_pool, "q_pool"));
+  BSA_TRY(check_ptr(k_pool, "k_pool"));
+  BSA_TRY(check_ptr(gate, "gate"));
+  BSA_TRY(check_ptr4(idx, "idx"));
+  BSA_TRY(check_ptr4(cnt, "cnt"));
+  BSA_TRY(check_device());
+  CUtensorMap kmap;
+  const bool tma = make_pool_map(&kmap, g, k_pool);
+  cudaError_t e = bsa::launch_select(g, q_pool, k_pool, gate, tma ? &kmap : nullptr, idx, cnt,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_select_topk_gated launch");
 }
 
 static bsa_status attention_common(const bsa_problem* prob, const void* layout_buf,
                                    const void* q_perm, const void* k_perm, const void* v_perm,
                                    const int32_t* idx, const int32_t* cnt, void* o_perm,
-                                   int32_t* dev_status, bool dense, void* stream) {
+                                   int32_t* dev_status, bool dense, void* stream,
+                                   float* lse = nullptr) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(layout_buf, "layout_buf"));
@@ -326,22 +440,29 @@ static bsa_status attention_common(const bsa_problem* prob, const void* layout_b
     BSA_TRY(check_ptr4(idx, "idx"));
     BSA_TRY(check_ptr4(cnt, "cnt"));
   }
+  if (lse) BSA_TRY(check_ptr4(lse, "lse"));
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
     return fail(BSA_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
   BSA_TRY(check_device());
-  CUtensorMap maps[2];
-  BSA_TRY(make_map(&maps[0], g, k_perm, 64));
-  BSA_TRY(make_map(&maps[1], g, v_perm, 64));
+  bsa::KVMaps<false> maps;
+  BSA_TRY(make_map(&maps.k, g, k_perm, 64));
+  BSA_TRY(make_map(&maps.v, g, v_perm, 64));
   int32_t* status = dev_status;
-  if (!status) {
-    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dev_status_sink);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status sink)");
-  }
+  BSA_TRY(status_word(&status));
   g.stall_pv = g_stall_pv;
-  cudaError_t e = bsa::launch_attention(g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
-                                        maps, static_cast<const __nv_bfloat16*>(q_perm), idx,
-                                        cnt, static_cast<__nv_bfloat16*>(o_perm),
-                                        status, dense, static_cast<cudaStream_t>(stream));
+  const bsa::LayoutPtrs lp = bsa::layout_ptrs(g, const_cast<void*>(layout_buf));
+  bsa::AttnIO io{};
+  io.q = static_cast<const __nv_bfloat16*>(q_perm);
+  io.o = static_cast<__nv_bfloat16*>(o_perm);
+  io.perm = lp.perm;
+  io.codes = lp.codes;
+  io.bmask = lp.bmask;
+  io.bfull = lp.bfull;
+  io.idx = idx;
+  io.cnt = cnt;
+  io.status = status;
+  io.lse = lse;
+  cudaError_t e = bsa::launch_attention(g, maps, io, dense, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "attention launch");
 }
 
@@ -351,6 +472,87 @@ bsa_status bsa_sparse_attn_fwd(const bsa_problem* prob, const void* layout_buf,
                                int32_t* dev_status, void* stream) {
   return attention_common(prob, layout_buf, q_perm, k_perm, v_perm, idx, cnt, o_perm, dev_status,
                           false, stream);
+}
+
+bsa_status bsa_sparse_attn_fwd_lse(const bsa_problem* prob, const void* layout_buf,
+                                   const void* q_perm, const void* k_perm, const void* v_perm,
+                                   const int32_t* idx, const int32_t* cnt, void* o_perm,
+                                   float* lse, int32_t* dev_status, void* stream) {
+  if (!lse) {
+    g_last_error[0] = 0;
+  BSA_RANGE();
+    return fail(BSA_ERR_INVALID_ARG, "lse is NULL");
+  }
+  return attention_common(prob, layout_buf, q_perm, k_perm, v_perm, idx, cnt, o_perm, dev_status,
+                          false, stream, lse);
+}
+
+bsa_status bsa_query_bwd_workspace(const bsa_problem* prob, size_t* bytes) {
+  g_last_error[0] = 0;
+  BSA_RANGE();
+  if (!bytes) return fail(BSA_ERR_INVALID_ARG, "bytes is NULL");
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  const size_t nw = size_t(g.nb + 31) / 32;
+  *bytes = bsa::align256(sizeof(float) * size_t(g.B) * g.h * g.N) +
+           bsa::align256(sizeof(uint32_t) * size_t(g.B) * g.h * g.nb * nw);
+  return BSA_OK;
+}
+
+bsa_status bsa_sparse_attn_bwd(const bsa_problem* prob, const void* layout_buf,
+                               const void* q_perm, const void* k_perm, const void* v_perm,
+                               const void* o_perm, const void* do_perm, const float* lse,
+                               const int32_t* idx, const int32_t* cnt, void* dq_perm,
+                               void* dk_perm, void* dv_perm, void* workspace, size_t ws_bytes,
+                               int32_t* dev_status, void* stream) {
+  g_last_error[0] = 0;
+  BSA_RANGE();
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  const void* p16[] = {layout_buf, q_perm, k_perm, v_perm, o_perm, do_perm, dq_perm, dk_perm,
+                       dv_perm, workspace};
+  const char* n16[] = {"layout_buf", "q_perm", "k_perm", "v_perm", "o_perm", "do_perm",
+                       "dq_perm", "dk_perm", "dv_perm", "workspace"};
+  for (int i = 0; i < 10; ++i) BSA_TRY(check_ptr(p16[i], n16[i]));
+  BSA_TRY(check_ptr(lse, "lse"));
+  BSA_TRY(check_ptr4(idx, "idx"));
+  BSA_TRY(check_ptr4(cnt, "cnt"));
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+    return fail(BSA_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  size_t need = 0;
+  BSA_TRY(bsa_query_bwd_workspace(prob, &need));
+  if (ws_bytes < need)
+    return fail(BSA_ERR_WORKSPACE, "workspace of %zu bytes; the backward needs %zu", ws_bytes,
+                need);
+  BSA_TRY(check_device());
+  CUtensorMap maps[4];
+  BSA_TRY(make_map(&maps[0], g, k_perm, 64));
+  BSA_TRY(make_map(&maps[1], g, v_perm, 64));
+  BSA_TRY(make_map(&maps[2], g, q_perm, 64));
+  BSA_TRY(make_map(&maps[3], g, do_perm, 64));
+  int32_t* status = dev_status;
+  BSA_TRY(status_word(&status));
+  const bsa::LayoutPtrs lp = bsa::layout_ptrs(g, const_cast<void*>(layout_buf));
+  bsa::BwdIO io{};
+  io.q = static_cast<const __nv_bfloat16*>(q_perm);
+  io.k = static_cast<const __nv_bfloat16*>(k_perm);
+  io.v = static_cast<const __nv_bfloat16*>(v_perm);
+  io.o = static_cast<const __nv_bfloat16*>(o_perm);
+  io.dout = static_cast<const __nv_bfloat16*>(do_perm);
+  io.lse = lse;
+  io.delta = static_cast<float*>(workspace);
+  io.kmask = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) +
+                                         bsa::align256(sizeof(float) * size_t(g.B) * g.h * g.N));
+  io.idx = idx;
+  io.cnt = cnt;
+  io.bmask = lp.bmask;
+  io.bfull = lp.bfull;
+  io.dq = static_cast<__nv_bfloat16*>(dq_perm);
+  io.dk = static_cast<__nv_bfloat16*>(dk_perm);
+  io.dv = static_cast<__nv_bfloat16*>(dv_perm);
+  io.status = status;
+  cudaError_t e = bsa::launch_attention_bwd(g, maps, io, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "backward launch");
 }
 
 bsa_status bsa_dense_attn_fwd(const bsa_problem* prob, const void* layout_buf,
@@ -364,6 +566,7 @@ bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const 
                          void* o_raster, int64_t stride_b, int64_t stride_n, int64_t stride_h,
                          void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(layout_buf, "layout_buf"));
@@ -376,6 +579,111 @@ bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const 
                                         static_cast<__nv_bfloat16*>(o_raster), stride_b,
                                         stride_n, stride_h, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_unpermute launch");
+}
+
+// ---- raster order: no permuted copies ---------------------------------------
+bsa_status bsa_pool_raster(const bsa_problem* prob, const void* layout_buf, const void* q_raster,
+                           const void* k_raster, int64_t stride_b, int64_t stride_n,
+                           int64_t stride_h, float* q_pool, float* k_pool, void* stream) {
+  g_last_error[0] = 0;
+  BSA_RANGE();
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(q_raster, "q_raster"));
+  BSA_TRY(check_ptr(k_raster, "k_raster"));
+  BSA_TRY(check_ptr(q_pool, "q_pool"));
+  BSA_TRY(check_ptr(k_pool, "k_pool"));
+  BSA_TRY(check_strides(g, stride_b, stride_n, stride_h, "q_raster/k_raster"));
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_pool_raster(
+      g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
+      static_cast<const __nv_bfloat16*>(q_raster), static_cast<const __nv_bfloat16*>(k_raster),
+      stride_b, stride_n, stride_h, q_pool, k_pool, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_pool_raster launch");
+}
+
+static bsa_status raster_attention(const bsa_problem* prob, const void* layout_buf,
+                                   const void* q_raster, const void* k_raster,
+                                   const void* v_raster, int64_t stride_b, int64_t stride_n,
+                                   int64_t stride_h, const int32_t* idx, const int32_t* cnt,
+                                   const int32_t* windows, void* o_raster, int64_t o_stride_b,
+                                   int64_t o_stride_n, int64_t o_stride_h, int32_t* dev_status,
+                                   void* stream) {
+  g_last_error[0] = 0;
+  BSA_RANGE();
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(q_raster, "q_raster"));
+  BSA_TRY(check_ptr(k_raster, "k_raster"));
+  BSA_TRY(check_ptr(v_raster, "v_raster"));
+  BSA_TRY(check_ptr(o_raster, "o_raster"));
+  if (windows) {
+    BSA_TRY(check_ptr4(windows, "windows"));
+  } else {
+    BSA_TRY(check_ptr4(idx, "idx"));
+    BSA_TRY(check_ptr4(cnt, "cnt"));
+  }
+  BSA_TRY(check_strides(g, stride_b, stride_n, stride_h, "q_raster/k_raster/v_raster"));
+  BSA_TRY(check_strides(g, o_stride_b, o_stride_n, o_stride_h, "o_raster"));
+  BSA_TRY(check_raster_kv(g, stride_h, "k_raster/v_raster"));
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+    return fail(BSA_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  BSA_TRY(check_device());
+  bsa::KVMaps<true> maps{};
+  BSA_TRY(make_raster_maps(maps.k, g, k_raster, stride_b, stride_n));
+  BSA_TRY(make_raster_maps(maps.v, g, v_raster, stride_b, stride_n));
+  int32_t* status = dev_status;
+  BSA_TRY(status_word(&status));
+  g.stall_pv = g_stall_pv;
+  const bsa::LayoutPtrs lp = bsa::layout_ptrs(g, const_cast<void*>(layout_buf));
+  bsa::AttnIO io{};
+  io.q = static_cast<const __nv_bfloat16*>(q_raster);
+  io.qsb = stride_b;
+  io.qsn = stride_n;
+  io.qsh = stride_h;
+  io.o = static_cast<__nv_bfloat16*>(o_raster);
+  io.osb = o_stride_b;
+  io.osn = o_stride_n;
+  io.osh = o_stride_h;
+  io.perm = lp.perm;
+  io.codes = lp.codes;
+  io.bmask = lp.bmask;
+  io.bfull = lp.bfull;
+  io.idx = idx;
+  io.cnt = cnt;
+  io.status = status;
+  io.windows = windows;
+  cudaError_t e = bsa::launch_attention_raster(g, maps, io, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "raster attention launch");
+}
+
+bsa_status bsa_sparse_attn_fwd_raster(const bsa_problem* prob, const void* layout_buf,
+                                      const void* q_raster, const void* k_raster,
+                                      const void* v_raster, int64_t stride_b, int64_t stride_n,
+                                      int64_t stride_h, const int32_t* idx, const int32_t* cnt,
+                                      void* o_raster, int64_t o_stride_b, int64_t o_stride_n,
+                                      int64_t o_stride_h, int32_t* dev_status, void* stream) {
+  return raster_attention(prob, layout_buf, q_raster, k_raster, v_raster, stride_b, stride_n,
+                          stride_h, idx, cnt, nullptr, o_raster, o_stride_b, o_stride_n,
+                          o_stride_h, dev_status, stream);
+}
+
+bsa_status bsa_window_attn_fwd_raster(const bsa_problem* prob, const void* layout_buf,
+                                      const void* q_raster, const void* k_raster,
+                                      const void* v_raster, int64_t stride_b, int64_t stride_n,
+                                      int64_t stride_h, const int32_t* windows, void* o_raster,
+                                      int64_t o_stride_b, int64_t o_stride_n, int64_t o_stride_h,
+                                      int32_t* dev_status, void* stream) {
+  if (!windows) {
+    g_last_error[0] = 0;
+  BSA_RANGE();
+    return fail(BSA_ERR_INVALID_ARG, "windows is NULL");
+  }
+  return raster_attention(prob, layout_buf, q_raster, k_raster, v_raster, stride_b, stride_n,
+                          stride_h, nullptr, nullptr, windows, o_raster, o_stride_b, o_stride_n,
+                          o_stride_h, dev_status, stream);
 }
 
 // ---- whole call from host memory -------------------------------------------
@@ -426,6 +734,7 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
                             const void* v_host, void* o_host, const bsa_device_buffers* buf,
                             int32_t heads_per_group, int32_t* dev_status, void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   if (!q_host || !k_host || !v_host || !o_host)
@@ -438,7 +747,11 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
   const char* dev_names[] = {"q_raster", "k_raster", "v_raster", "o_raster", "q_perm",
                              "k_perm",   "v_perm",   "o_perm",   "layout_buf", "q_pool",
                              "k_pool",   "idx",      "cnt"};
-  for (int i = 0; i < 11; ++i) BSA_TRY(check_ptr(dev_ptrs[i], dev_names[i]));
+  // no permuted buffers at all: the permute-free path reads the tiles
+  // straight from the raster buffers
+  const bool raster = !buf->q_perm && !buf->k_perm && !buf->v_perm && !buf->o_perm;
+  for (int i = 0; i < 11; ++i)
+    if (!(raster && i >= 4 && i < 8)) BSA_TRY(check_ptr(dev_ptrs[i], dev_names[i]));
   BSA_TRY(check_ptr4(buf->idx, "idx"));
   BSA_TRY(check_ptr4(buf->cnt, "cnt"));
   if (heads_per_group < 1 || heads_per_group > g.h || g.h % heads_per_group != 0)
@@ -519,13 +832,21 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
     float* kpool = buf->k_pool + i * pool_elems;
     int32_t* idx = buf->idx + i * idx_elems;
     int32_t* cnt = buf->cnt + i * cnt_elems;
-    BSA_TRY(bsa_permute(&sub, buf->layout_buf, rq, sb, sn, sh, pq, st));
-    BSA_TRY(bsa_permute(&sub, buf->layout_buf, rk, sb, sn, sh, pk, st));
-    BSA_TRY(bsa_permute(&sub, buf->layout_buf, rv, sb, sn, sh, pv, st));
-    BSA_TRY(bsa_pool(&sub, buf->layout_buf, pq, pk, qpool, kpool, st));
-    BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
-    BSA_TRY(bsa_sparse_attn_fwd(&sub, buf->layout_buf, pq, pk, pv, idx, cnt, po, dev_status, st));
-    BSA_TRY(bsa_unpermute(&sub, buf->layout_buf, po, ro, sb, sn, sh, st));
+    if (raster) {
+      BSA_TRY(bsa_pool_raster(&sub, buf->layout_buf, rq, rk, sb, sn, sh, qpool, kpool, st));
+      BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
+      BSA_TRY(bsa_sparse_attn_fwd_raster(&sub, buf->layout_buf, rq, rk, rv, sb, sn, sh, idx, cnt,
+                                         ro, sb, sn, sh, dev_status, st));
+    } else {
+      BSA_TRY(bsa_permute(&sub, buf->layout_buf, rq, sb, sn, sh, pq, st));
+      BSA_TRY(bsa_permute(&sub, buf->layout_buf, rk, sb, sn, sh, pk, st));
+      BSA_TRY(bsa_permute(&sub, buf->layout_buf, rv, sb, sn, sh, pv, st));
+      BSA_TRY(bsa_pool(&sub, buf->layout_buf, pq, pk, qpool, kpool, st));
+      BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
+      BSA_TRY(bsa_sparse_attn_fwd(&sub, buf->layout_buf, pq, pk, pv, idx, cnt, po, dev_status,
+                                  st));
+      BSA_TRY(bsa_unpermute(&sub, buf->layout_buf, po, ro, sb, sn, sh, st));
+    }
     BSA_CUDA(cudaEventRecord(ev_out(i), st), "cudaEventRecord");
   }
   // downloads on the output stream; the caller's stream ends with the last one
@@ -543,12 +864,14 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
 
 bsa_status bsa_debug_stall_pv(int32_t enable) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   g_stall_pv = enable ? 1 : 0;
   return BSA_OK;
 }
 
 bsa_status bsa_take_default_status(int32_t* out, void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   if (!out) return fail(BSA_ERR_INVALID_ARG, "out is NULL");
   BSA_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -569,6 +892,7 @@ bsa_status bsa_take_default_status(int32_t* out, void* stream) {
 bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int64_t hist7[7],
                             void* stream) {
   g_last_error[0] = 0;
+  BSA_RANGE();
   Geo g;
   BSA_TRY(make_geo(prob, &g));
   BSA_TRY(check_ptr(layout_buf, "layout_buf"));

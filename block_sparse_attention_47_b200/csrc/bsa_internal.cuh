@@ -98,11 +98,73 @@ cudaError_t launch_unpermute(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* o
                              cudaStream_t st);
 cudaError_t launch_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* qp,
                         const __nv_bfloat16* kp, float* qpool, float* kpool, cudaStream_t st);
-cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, int32_t* idx,
-                          int32_t* cnt, cudaStream_t st);
-cudaError_t launch_attention(const Geo& g, LayoutPtrs lp, const CUtensorMap* maps,
-                             const __nv_bfloat16* qp, const int32_t* idx, const int32_t* cnt,
-                             __nv_bfloat16* o, int32_t* dev_status, bool dense, cudaStream_t st);
+// kmap (optional): 2-D map over the pooled keys [B*heads*nb rows, d] fp32,
+// 32 x 256 boxes, 128-byte swizzle (the TMA-fed score tiles)
+cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, const float* gate,
+                          const CUtensorMap* kmap, int32_t* idx, int32_t* cnt, cudaStream_t st);
+cudaError_t launch_pool_raster(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* q,
+                               const __nv_bfloat16* k, int64_t sb, int64_t sn, int64_t sh,
+                               float* qpool, float* kpool, cudaStream_t st);
+
+// Pointers and strides of one attention launch.  Block order: q and o are
+// permuted [B, heads, N, d] tensors (strides unused).  Raster order: q and o
+// are raster [B, N, heads, d] tensors with element strides, addressed
+// through the slot -> raster map `perm`.
+struct AttnIO {
+  const __nv_bfloat16* q;
+  int64_t qsb, qsn, qsh;
+  __nv_bfloat16* o;
+  int64_t osb, osn, osh;
+  const int32_t* perm;
+  const uint8_t* codes;
+  const uint64_t* bmask;
+  const uint8_t* bfull;
+  const int32_t* idx;
+  const int32_t* cnt;
+  int32_t* status;
+  // window heads instead of index lists: int32 [heads][3] (w_t, w_y, w_x),
+  // negative = unbounded; null for the list-driven walk
+  const int32_t* windows;
+  // optional output: per-row log-sum-exp (exp2 domain) [B, heads, N], block order
+  float* lse;
+};
+
+// Pointers of one backward (block-order tensors [B, heads, N, d]).
+struct BwdIO {
+  const __nv_bfloat16 *q, *k, *v, *o, *dout;
+  const float* lse;       // [B, heads, N] from the forward
+  float* delta;           // workspace [B, heads, N]: rowsum(dO * O)
+  uint32_t* kmask;        // workspace [B, heads, nb, ceil(nb/32)]: transposed lists
+  const int32_t *idx, *cnt;
+  const uint64_t* bmask;
+  const uint8_t* bfull;
+  __nv_bfloat16 *dq, *dk, *dv;
+  int32_t* status;
+};
+
+// maps: K, V, Q, dO (3-D maps over the permuted tensors, 64-row boxes)
+cudaError_t launch_attention_bwd(const Geo& g, const CUtensorMap* maps, const BwdIO& io,
+                                 cudaStream_t st);
+
+// TMA maps of K and V.  Block order: one 3-D map each over [B*heads, N, d].
+// Raster order: [0] a 3-D map over [B, N, heads*d] for the prefix blocks
+// (64 consecutive tokens), [1 + code] a 5-D map over [B, T, H, W, heads*d]
+// whose box is one video block of shape code (0 = 4x4x4).
+template <bool RASTER>
+struct KVMaps;
+template <>
+struct KVMaps<false> {
+  CUtensorMap k, v;
+};
+template <>
+struct KVMaps<true> {
+  CUtensorMap k[8], v[8];
+};
+
+cudaError_t launch_attention(const Geo& g, const KVMaps<false>& maps, const AttnIO& io,
+                             bool dense, cudaStream_t st);
+cudaError_t launch_attention_raster(const Geo& g, const KVMaps<true>& maps, const AttnIO& io,
+                                    cudaStream_t st);
 
 // ---- device helpers -----------------------------------------------------
 #if defined(__CUDACC__)
@@ -121,6 +183,11 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 }
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -179,6 +246,31 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(c4)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -59,6 +59,55 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
   }
 }
 
+// The same block means read straight from raster Q and K through the
+// layout's slot -> raster map (no permuted copies).  Rows are summed in the
+// same order as pool_kernel (pad slots, zero there, are skipped here), so
+// the two give bit-identical means.
+__global__ void __launch_bounds__(kPoolThreads) pool_raster_kernel(
+    Geo g, const int32_t* __restrict__ perm, const int32_t* __restrict__ bcount,
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int64_t sb,
+    int64_t sn, int64_t sh, float* __restrict__ qpool, float* __restrict__ kpool) {
+  const int j = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int vec = g.d / 8;
+  const int groups = kPoolThreads / vec;
+  const int v = threadIdx.x % vec, rg = threadIdx.x / vec;
+  __shared__ float red[2][kPoolThreads / 8][129];
+  __shared__ int64_t src[kBlock];  // element offset of each slot's row, -1 for pad
+  if (threadIdx.x < kBlock) {
+    const uint32_t pr = uint32_t(perm[int64_t(b) * g.N + int64_t(j) * kBlock + threadIdx.x]);
+    src[threadIdx.x] =
+        (pr & 0x80000000u) ? -1 : int64_t(b) * sb + int64_t(pr) * sn + int64_t(hh) * sh;
+  }
+  __syncthreads();
+  for (int which = 0; which < 2; ++which) {
+    const __nv_bfloat16* x = which ? k : q;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int r = rg; r < kBlock; r += groups) {
+      const int64_t off = src[r];
+      if (off < 0) continue;
+      const uint4 u = *reinterpret_cast<const uint4*>(x + off + v * 8);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[which][rg][v * 8 + i] = acc[i];
+  }
+  __syncthreads();
+  const float inv = 1.0f / float(bcount[int64_t(b) * g.nb + j]);
+  const int64_t out0 = ((int64_t(b) * g.h + hh) * g.nb + j) * g.d;
+  for (int c = threadIdx.x; c < 2 * g.d; c += kPoolThreads) {
+    const int which = c / g.d, ch = c % g.d;
+    float s = 0.f;
+    for (int r = 0; r < groups; ++r) s += red[which][r][ch];
+    (which ? kpool : qpool)[out0 + ch] = s * inv;
+  }
+}
+
 // ---- selection --------------------------------------------------------------
 constexpr int kSelThreads = 256;
 constexpr int kSelRows = 8;  // query blocks per CTA, one per warp in the top-k phase
@@ -68,16 +117,43 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// dynamic smem: q rows [kSelRows][d] fp32, keys [kSelRows][nbv] u32,
-// histograms [8 warps][256] u32
-__global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, const float* __restrict__ qpool,
-                                                             const float* __restrict__ kpool,
-                                                             int32_t* __restrict__ idx,
-                                                             int32_t* __restrict__ cnt) {
+// Score tiles: KPT key blocks per thread, so kSelThreads * KPT pooled key
+// rows per pass, staged through shared memory 32 channels at a time with
+// coalesced 16-byte loads (row stride 36 floats: the 16-byte reads of 8
+// consecutive rows hit 8 distinct bank quads).
+constexpr int kSelChunk = 32;
+constexpr int kSelStride = kSelChunk + 4;
+
+template <int KPT>
+constexpr size_t select_tile_floats() {
+  return size_t(kSelThreads) * KPT * kSelStride;
+}
+
+// dynamic smem: q rows [kSelRows][d] fp32, keys [kSelRows][nbv] u32, then
+// the key tile (KPT > 0), whose space the histograms [8 warps][256] u32 of
+// the top-k phase reuse.
+//
+// KPT > 0: every score is one fmaf chain over the channels in ascending
+// order, as in the KPT == 0 form (one key block per thread read straight
+// from global memory, for sequences whose scores leave no room for a tile),
+// so both give bit-identical lists.
+//
+// gate (optional, fp32 [heads][d][d]): the learned-gate score of the VSA
+// description (Ref2VA VSA, pulmap.app, section "토큰 75%를 건너뛰는 VSA": a
+// trained predictor, to_gate_compress, decides which tiles matter): each
+// pooled query row is first mapped through its head's gate matrix,
+// q~_c = sum_e G[c][e] q_e (one fmaf chain in e order), and the key blocks
+// are scored against q~.  G = identity gives the ungated scores bit for bit.
+template <int KPT, bool TMA>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(
+    const __grid_constant__ CUtensorMap kmap, Geo g, const float* __restrict__ qpool,
+    const float* __restrict__ kpool, const float* __restrict__ gate, int32_t* __restrict__ idx,
+    int32_t* __restrict__ cnt) {
   extern __shared__ __align__(16) unsigned char smem[];
   float* sq = reinterpret_cast<float*>(smem);
   uint32_t* skey = reinterpret_cast<uint32_t*>(sq + kSelRows * g.d);
-  uint32_t* shist = skey + kSelRows * g.nbv;
+  float* stile = reinterpret_cast<float*>(skey + ((kSelRows * g.nbv + 3) & ~3));
+  uint32_t* shist = KPT > 0 ? reinterpret_cast<uint32_t*>(stile) : skey + kSelRows * g.nbv;
 
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * kSelRows;  // first video query block of this CTA
@@ -94,7 +170,153 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(Geo g, const float*
     sq[e] = r < rows ? qpool[pool0 + int64_t(g.nbp + i0 + r) * g.d + c] : 0.f;
   }
   __syncthreads();
+  if (gate) {
+    // 8 rows x d outputs, at most 4 per thread (d <= 128)
+    const float* G = gate + int64_t(bh % g.h) * g.d * g.d;
+    float gq[(kSelRows * 128) / kSelThreads];
+    int n_out = 0;
+    for (int e = threadIdx.x; e < kSelRows * g.d; e += kSelThreads, ++n_out) {
+      const int r = e / g.d, c = e % g.d;
+      const float4* gr = reinterpret_cast<const float4*>(G + int64_t(c) * g.d);
+      const float4* qr = reinterpret_cast<const float4*>(sq + r * g.d);
+      float acc = 0.f;
+      for (int e4 = 0; e4 < g.d / 4; ++e4) {
+        const float4 gv = __ldg(gr + e4), qv = qr[e4];
+        acc = fmaf(gv.x, qv.x, acc);
+        acc = fmaf(gv.y, qv.y, acc);
+        acc = fmaf(gv.z, qv.z, acc);
+        acc = fmaf(gv.w, qv.w, acc);
+      }
+      gq[n_out] = acc;
+    }
+    __syncthreads();
+    n_out = 0;
+    for (int e = threadIdx.x; e < kSelRows * g.d; e += kSelThreads, ++n_out) sq[e] = gq[n_out];
+    __syncthreads();
+  }
 
+  if constexpr (TMA) {
+    // scores, register-tiled as below, with the pooled-key chunks (KT rows x
+    // 32 channels) brought in by TMA into two 128-byte-swizzled buffers: the
+    // next chunk's copy runs while this one is multiplied
+    constexpr int KT = kSelThreads * KPT;
+    constexpr int TILE = KT * 128;
+    const uint32_t tiles = (smem_u32(stile) + 1023u) & ~1023u;
+    const uint32_t bar = tiles + 2 * TILE;
+    const int ncpp = g.d / kSelChunk;                     // chunks per pass
+    const int total = ((g.nbv + KT - 1) / KT) * ncpp;
+    const int row0 = bh * g.nb + g.nbp;                   // this (b, h)'s first video key row
+    if (threadIdx.x == 0) {
+      mbar_init(bar, 1);
+      mbar_init(bar + 8, 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int c) {
+      const int kb = (c / ncpp) * KT, cc = (c % ncpp) * kSelChunk;
+      const uint32_t b8 = bar + 8u * uint32_t(c & 1);
+      mbar_arrive_expect_tx(b8, TILE);
+#pragma unroll
+      for (int part = 0; part < KT / 256; ++part)
+        tma_load_2d(tiles + (c & 1) * TILE + part * 256 * 128, &kmap, b8, cc,
+                    row0 + kb + part * 256);
+    };
+    if (threadIdx.x == 0) issue(0);
+    float acc[kSelRows][KPT];
+    for (int c = 0; c < total; ++c) {
+      // buffer (c+1)&1 was last read in chunk c-1, which ended in a barrier
+      if (threadIdx.x == 0 && c + 1 < total) issue(c + 1);
+      const int kb = (c / ncpp) * KT, cc = (c % ncpp) * kSelChunk;
+      if (cc == 0) {
+#pragma unroll
+        for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) acc[r][u] = 0.f;
+      }
+      mbar_wait(bar + 8u * uint32_t(c & 1), (c >> 1) & 1, nullptr);
+      const uint32_t buf = tiles + (c & 1) * TILE;
+#pragma unroll
+      for (int c4 = 0; c4 < kSelChunk / 4; ++c4) {
+        float4 kv[KPT];
+#pragma unroll
+        for (int u = 0; u < KPT; ++u) {
+          const int rr = threadIdx.x + kSelThreads * u;
+          kv[u] = ld_shared_f4(buf + rr * 128 + ((c4 ^ (rr & 7)) << 4));
+        }
+#pragma unroll
+        for (int r = 0; r < kSelRows; ++r) {
+          const float4 qv = *reinterpret_cast<const float4*>(sq + r * g.d + cc + 4 * c4);
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) {
+            acc[r][u] = fmaf(qv.x, kv[u].x, acc[r][u]);
+            acc[r][u] = fmaf(qv.y, kv[u].y, acc[r][u]);
+            acc[r][u] = fmaf(qv.z, kv[u].z, acc[r][u]);
+            acc[r][u] = fmaf(qv.w, kv[u].w, acc[r][u]);
+          }
+        }
+      }
+      if (cc + kSelChunk == g.d) {
+#pragma unroll
+        for (int u = 0; u < KPT; ++u) {
+          const int jv = kb + threadIdx.x + kSelThreads * u;
+          if (jv < g.nbv)
+#pragma unroll
+            for (int r = 0; r < kSelRows; ++r) skey[r * g.nbv + jv] = order_key(acc[r][u]);
+        }
+      }
+      __syncthreads();
+    }
+  } else if constexpr (KPT > 0) {
+    // scores, register-tiled: thread t owns key blocks kb + t + 256*u
+    // (u < KPT) for all 8 rows
+    constexpr int KT = kSelThreads * KPT;
+    const float* kbase = kpool + pool0 + int64_t(g.nbp) * g.d;
+    for (int kb = 0; kb < g.nbv; kb += KT) {
+      float acc[kSelRows][KPT];
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+        for (int u = 0; u < KPT; ++u) acc[r][u] = 0.f;
+      for (int cc = 0; cc < g.d; cc += kSelChunk) {
+        __syncthreads();  // the previous chunk has been read
+        // rows kb..kb+KT-1, channels cc..cc+31: 8 float4 per row, coalesced
+        for (int e = threadIdx.x; e < KT * (kSelChunk / 4); e += kSelThreads) {
+          const int kr = e >> 3, c4 = e & 7;
+          float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (kb + kr < g.nbv)
+            val = __ldg(reinterpret_cast<const float4*>(kbase + int64_t(kb + kr) * g.d + cc) + c4);
+          *reinterpret_cast<float4*>(stile + kr * kSelStride + 4 * c4) = val;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c4 = 0; c4 < kSelChunk / 4; ++c4) {
+          float4 kv[KPT];
+#pragma unroll
+          for (int u = 0; u < KPT; ++u)
+            kv[u] = *reinterpret_cast<const float4*>(stile + (threadIdx.x + kSelThreads * u) *
+                                                                 kSelStride + 4 * c4);
+#pragma unroll
+          for (int r = 0; r < kSelRows; ++r) {
+            const float4 qv = *reinterpret_cast<const float4*>(sq + r * g.d + cc + 4 * c4);
+#pragma unroll
+            for (int u = 0; u < KPT; ++u) {
+              acc[r][u] = fmaf(qv.x, kv[u].x, acc[r][u]);
+              acc[r][u] = fmaf(qv.y, kv[u].y, acc[r][u]);
+              acc[r][u] = fmaf(qv.z, kv[u].z, acc[r][u]);
+              acc[r][u] = fmaf(qv.w, kv[u].w, acc[r][u]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < KPT; ++u) {
+        const int jv = kb + threadIdx.x + kSelThreads * u;
+        if (jv < g.nbv)
+#pragma unroll
+          for (int r = 0; r < kSelRows; ++r) skey[r * g.nbv + jv] = order_key(acc[r][u]);
+      }
+    }
+  } else
   // scores: thread per key block, all rows of the CTA at once
   for (int jv = threadIdx.x; jv < g.nbv; jv += kSelThreads) {
     const float4* kr = reinterpret_cast<const float4*>(kpool + pool0 + int64_t(g.nbp + jv) * g.d);
@@ -200,20 +422,70 @@ cudaError_t launch_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* qp,
   return cudaGetLastError();
 }
 
+cudaError_t launch_pool_raster(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* q,
+                               const __nv_bfloat16* k, int64_t sb, int64_t sn, int64_t sh,
+                               float* qpool, float* kpool, cudaStream_t st) {
+  pool_raster_kernel<<<dim3(g.nb, g.h, g.B), kPoolThreads, 0, st>>>(g, lp.perm, lp.bcount, q, k,
+                                                                    sb, sn, sh, qpool, kpool);
+  return cudaGetLastError();
+}
+
+// shared memory of the untiled form (the limit a problem is validated against)
 size_t select_smem_bytes(const Geo& g) {
   return sizeof(float) * kSelRows * g.d + sizeof(uint32_t) * kSelRows * g.nbv +
          sizeof(uint32_t) * (kSelThreads / 32) * 256;
 }
 
-cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, int32_t* idx,
-                          int32_t* cnt, cudaStream_t st) {
-  const size_t smem = select_smem_bytes(g);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+namespace {
+template <int KPT>
+size_t select_tiled_smem_bytes(const Geo& g) {
+  return sizeof(float) * kSelRows * g.d + sizeof(uint32_t) * ((kSelRows * g.nbv + 3) & ~3) +
+         sizeof(float) * select_tile_floats<KPT>();
+}
+
+// the TMA form: two 128-byte-swizzled chunk buffers (1024-byte aligned) and
+// their two barriers after the row scores
+template <int KPT>
+size_t select_tma_smem_bytes(const Geo& g) {
+  return sizeof(float) * kSelRows * g.d + sizeof(uint32_t) * ((kSelRows * g.nbv + 3) & ~3) +
+         1024 + 2 * size_t(kSelThreads) * KPT * 128 + 16;
+}
+
+template <int KPT, bool TMA>
+cudaError_t launch_select_t(const Geo& g, size_t smem, const CUtensorMap* kmap,
+                            const float* qpool, const float* kpool, const float* gate,
+                            int32_t* idx, int32_t* cnt, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT, TMA>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
+  CUtensorMap none{};
   const int ctas = (g.nbv + kSelRows - 1) / kSelRows;
-  select_kernel<<<dim3(ctas, g.B * g.h), kSelThreads, smem, st>>>(g, qpool, kpool, idx, cnt);
+  select_kernel<KPT, TMA><<<dim3(ctas, g.B * g.h), kSelThreads, smem, st>>>(
+      kmap ? *kmap : none, g, qpool, kpool, gate, idx, cnt);
   return cudaGetLastError();
+}
+}  // namespace
+
+// The TMA-fed form when a pooled-key map is given and its two buffers fit
+// next to the row scores; else the widest register tile that fits; else one
+// key block per thread.
+cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, const float* gate,
+                          const CUtensorMap* kmap, int32_t* idx, int32_t* cnt, cudaStream_t st) {
+  constexpr size_t kMax = 227 * 1024;
+  if (kmap && select_tma_smem_bytes<2>(g) <= kMax)
+    return launch_select_t<2, true>(g, select_tma_smem_bytes<2>(g), kmap, qpool, kpool, gate, idx,
+                                    cnt, st);
+  if (select_tiled_smem_bytes<4>(g) <= kMax)
+    return launch_select_t<4, false>(g, select_tiled_smem_bytes<4>(g), nullptr, qpool, kpool, gate,
+                                     idx, cnt, st);
+  if (select_tiled_smem_bytes<2>(g) <= kMax)
+    return launch_select_t<2, false>(g, select_tiled_smem_bytes<2>(g), nullptr, qpool, kpool, gate,
+                                     idx, cnt, st);
+  if (select_tiled_smem_bytes<1>(g) <= kMax)
+    return launch_select_t<1, false>(g, select_tiled_smem_bytes<1>(g), nullptr, qpool, kpool, gate,
+                                     idx, cnt, st);
+  return launch_select_t<0, false>(g, select_smem_bytes(g), nullptr, qpool, kpool, gate, idx, cnt,
+                                   st);
 }
 
 }  // namespace bsa

@@ -114,6 +114,17 @@ def make_qkv(cfg, seed, pad_fill=1e4, device="cpu"):
     return tuple(make_tensor(cfg, seed, i, pad_fill, device) for i in range(3))
 
 
+def make_gate(heads, head_dim, seed, spread=0.5, device="cpu"):
+    """Synthetic gate matrices fp32 [heads, d, d] standing in for trained
+    to_gate_compress weights (none are available): identity plus seeded
+    Gaussian entries of standard deviation spread/sqrt(d), so the gated
+    selection differs from the plain pooled score but keeps its structure."""
+    g = _gen(seed, 50, device)
+    eye = torch.eye(head_dim, device=device).expand(heads, head_dim, head_dim)
+    noise = torch.randn((heads, head_dim, head_dim), generator=g, device=device)
+    return (eye + noise * (spread / math.sqrt(head_dim))).float().contiguous()
+
+
 def layer_keep_schedule(n_layers=40, seed=42004, choices=(0.01, 0.03, 0.05, 0.10)):
     """Per-layer keep ratios drawn by seed from the 1/3/5/10 % menu that the
     "倍速で回した一晩" digest's layer controller chose from."""

@@ -165,6 +165,18 @@ bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void*
 bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const float* k_pool,
                            int32_t* idx, int32_t* cnt, void* stream);
 
+/* bsa_select_topk with a learned-gate score (Ref2VA VSA, pulmap.app, section
+ * "토큰 75%를 건너뛰는 VSA": a trained predictor, to_gate_compress, picks the
+ * tiles that matter instead of a fixed rule).  Each pooled query row is
+ * mapped through its head's gate matrix before scoring:
+ *   S[i, j] = sum_c (sum_e G[h][c][e] q_pool[i][e]) k_pool[j][c]   (fp32)
+ * gate: device fp32 [heads][head_dim][head_dim], row-major, caller-owned.
+ * G = identity gives exactly the bsa_select_topk lists.  Everything else
+ * (prefix handling, ties, output format) as bsa_select_topk. */
+bsa_status bsa_select_topk_gated(const bsa_problem* prob, const float* q_pool,
+                                 const float* k_pool, const float* gate, int32_t* idx,
+                                 int32_t* cnt, void* stream);
+
 /* Block-sparse attention over the kept tiles: for each query block i and
  * each key block j in idx row i (all blocks when cnt[i] == -1), logits
  * softmax_scale * q.k over the valid keys of j, online softmax, O = P V,
@@ -174,6 +186,42 @@ bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const f
 bsa_status bsa_sparse_attn_fwd(const bsa_problem* prob, const void* layout_buf,
                                const void* q_perm, const void* k_perm, const void* v_perm,
                                const int32_t* idx, const int32_t* cnt, void* o_perm,
+                               int32_t* dev_status, void* stream);
+
+/* ---- training: the same sparse attention, forward with statistics and
+ * backward (Prism / Kandinsky 6 speed ablation, section "같은 계산량 안에서
+ * 볼 곳을 고르는 Prism": the sparse attention also trains, a 2K training step
+ * from 26.5 to 10.6 minutes). */
+
+/* bsa_sparse_attn_fwd that also writes each query row's log-sum-exp in the
+ * exp2 domain, lse[b, h, slot] = m + log2(l) with P = exp2(s * softmax_scale
+ * * log2(e) - lse) (fp32 [B, heads, N], block order, 16-byte aligned; +inf
+ * for pad rows), which the backward reuses. */
+bsa_status bsa_sparse_attn_fwd_lse(const bsa_problem* prob, const void* layout_buf,
+                                   const void* q_perm, const void* k_perm, const void* v_perm,
+                                   const int32_t* idx, const int32_t* cnt, void* o_perm,
+                                   float* lse, int32_t* dev_status, void* stream);
+
+/* Bytes of the backward's workspace (rowsum(dO * O) per row and the
+ * transposed key-block -> query-block bitmaps).  Host only. */
+bsa_status bsa_query_bwd_workspace(const bsa_problem* prob, size_t* bytes);
+
+/* Gradients of the block-sparse attention over the same kept tiles, all in
+ * block order [B, heads, N, head_dim] bf16 (use bsa_permute on dO and
+ * bsa_unpermute on the gradients for raster order):
+ *   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),
+ *   dQ = softmax_scale * dS K,  dK = softmax_scale * dS^T Q,
+ * with P recomputed from lse (bsa_sparse_attn_fwd_lse) over the kept tiles
+ * of idx/cnt (the forward's lists).  Pad tokens get zero gradients.
+ * workspace: caller-owned, ws_bytes >= bsa_query_bwd_workspace (16-byte
+ * aligned), else BSA_ERR_WORKSPACE.  Accumulation is fp32 in tensor memory;
+ * each gradient element is written once (no atomics), so results are
+ * deterministic. */
+bsa_status bsa_sparse_attn_bwd(const bsa_problem* prob, const void* layout_buf,
+                               const void* q_perm, const void* k_perm, const void* v_perm,
+                               const void* o_perm, const void* do_perm, const float* lse,
+                               const int32_t* idx, const int32_t* cnt, void* dq_perm,
+                               void* dk_perm, void* dv_perm, void* workspace, size_t ws_bytes,
                                int32_t* dev_status, void* stream);
 
 /* The same attention over every tile (pad keys masked): the dense comparator. */
@@ -187,6 +235,72 @@ bsa_status bsa_unpermute(const bsa_problem* prob, const void* layout_buf, const 
                          void* o_raster, int64_t stride_b, int64_t stride_n, int64_t stride_h,
                          void* stream);
 
+/* ---- raster order: the same call without permuted copies -----------------
+ * The permutation exists only so that every kept block is one contiguous
+ * tile (Sparse VideoGen on TPU, section "실무에서 배울 최적화 기준": token
+ * order decides whether a sparse pattern pays).  With these two calls the
+ * kernels read the tiles straight out of the raster tensors instead, so
+ * bsa_permute and bsa_unpermute, and the four permuted buffers, drop out:
+ *   bsa_layout -> bsa_pool_raster -> bsa_select_topk
+ *   -> bsa_sparse_attn_fwd_raster
+ * Results equal the permuted sequence's (pooled means bit for bit; the
+ * attention output up to the order of fp32 accumulation, which is the same). */
+
+/* Block means of raster Q and K (the bsa_pool definition), read through the
+ * layout's slot -> raster map.  q_raster and k_raster share the element
+ * strides (stride_b, stride_n, stride_h). */
+bsa_status bsa_pool_raster(const bsa_problem* prob, const void* layout_buf, const void* q_raster,
+                           const void* k_raster, int64_t stride_b, int64_t stride_n,
+                           int64_t stride_h, float* q_pool, float* k_pool, void* stream);
+
+/* bsa_sparse_attn_fwd on raster tensors.  Each kept K or V block is loaded
+ * as one TMA box of the [B, T, H, W, heads*head_dim] grid (video blocks;
+ * one box shape per block shape) or as 64 consecutive tokens (prefix
+ * blocks); query rows are read and output rows written through the
+ * layout's slot -> raster map.
+ *   q_raster, k_raster, v_raster  [B, N, heads, head_dim] bf16 sharing the
+ *                                 strides (stride_b, stride_n, stride_h);
+ *                                 stride_h must equal head_dim (heads
+ *                                 contiguous in a token row, as a fused QKV
+ *                                 projection leaves them), else
+ *                                 BSA_ERR_UNSUPPORTED
+ *   o_raster                      output [B, N, heads, head_dim] with its own
+ *                                 strides; pad tokens are written as 0
+ * Pad tokens of the raster K and V are read (and masked out of the
+ * softmax), so they must hold finite values; a pad row of V multiplies a
+ * probability of exactly 0. */
+bsa_status bsa_sparse_attn_fwd_raster(const bsa_problem* prob, const void* layout_buf,
+                                      const void* q_raster, const void* k_raster,
+                                      const void* v_raster, int64_t stride_b, int64_t stride_n,
+                                      int64_t stride_h, const int32_t* idx, const int32_t* cnt,
+                                      void* o_raster, int64_t o_stride_b, int64_t o_stride_n,
+                                      int64_t o_stride_h, int32_t* dev_status, void* stream);
+
+/* Window heads: attention under a per-head spatio-temporal window instead of
+ * top-k lists, with tiles classed full / boundary / empty (Sparse VideoGen on
+ * TPU, sections "Sparse VideoGen의 핵심 아이디어": spatial heads look within
+ * nearby frames, temporal heads at the same place across frames; and
+ * "이론적 sparsity와 물리적 sparsity의 차이": empty tiles are skipped, only
+ * boundary tiles need an element mask).
+ *   windows  device int32 [heads][3] = (w_t, w_y, w_x); a negative entry
+ *            leaves that axis unbounded.  Query token (t, y, x) attends to
+ *            video key (t', y', x') when |t'-t| <= w_t, |y'-y| <= w_y and
+ *            |x'-x| <= w_x; every query attends to every prefix key and
+ *            prefix queries attend to every key; pad keys are excluded and
+ *            pad query rows are 0.  A spatial head is (w, -1, -1), a
+ *            temporal head (-1, r, r).
+ * A query block walks only the key blocks whose box its box can reach
+ * through the window (non-empty tiles); inside a tile each query row masks
+ * the keys outside its window (boundary tiles), while full tiles need no
+ * mask.  Other arguments as in bsa_sparse_attn_fwd_raster (prob.keep_blocks
+ * is validated but unused). */
+bsa_status bsa_window_attn_fwd_raster(const bsa_problem* prob, const void* layout_buf,
+                                      const void* q_raster, const void* k_raster,
+                                      const void* v_raster, int64_t stride_b, int64_t stride_n,
+                                      int64_t stride_h, const int32_t* windows, void* o_raster,
+                                      int64_t o_stride_b, int64_t o_stride_n, int64_t o_stride_h,
+                                      int32_t* dev_status, void* stream);
+
 /* Histogram of video blocks by shape code over the whole batch (hist7[0]
  * counts 4x4x4 blocks; each dynamic region adds 8 blocks of its code), the
  * block-shape log of the Prism speed ablation (section "동적 블록을 켜도
@@ -199,7 +313,10 @@ bsa_status bsa_layout_stats(const bsa_problem* prob, const void* layout_buf, int
  * bsa_query_sizes): raster Q, K, V, O (raster_tensor_bytes each, contiguous
  * [B, N, heads, head_dim]), permuted Q, K, V, O (perm_tensor_bytes each),
  * the layout (layout_bytes), pooled Q and K (pool_bytes each), index lists
- * (idx_bytes) and counts (cnt_bytes).  16-byte aligned (idx and cnt: 4). */
+ * (idx_bytes) and counts (cnt_bytes).  16-byte aligned (idx and cnt: 4).
+ * The four permuted buffers may all be NULL: bsa_forward_host then runs the
+ * permute-free sequence (bsa_pool_raster, bsa_sparse_attn_fwd_raster) on the
+ * raster buffers and needs no permuted copies. */
 typedef struct bsa_device_buffers {
   void* q_raster;
   void* k_raster;

@@ -322,6 +322,36 @@ def select(geo, q_pool, k_pool, keep, rows=None):
     return lists
 
 
+def block_scores_gated_f32(geo, q_pool, k_pool, gate):
+    """float32 [nbv, nbv] learned-gate scores ([REF2VA] "토큰 75%를 건너뛰는
+    VSA": a trained predictor, to_gate_compress, picks the tiles that matter).
+    Reading: the head's gate matrix G maps each pooled query row,
+    q~_c = sum_e G[c][e] q_e, and q~ is scored against the pooled key means.
+    Pooled values and G are rounded to float32 first, the products are taken
+    in float64 and the scores rounded to float32."""
+    qp = np.asarray(q_pool, dtype=np.float32).astype(np.float64)[geo.nbp:]
+    kp = np.asarray(k_pool, dtype=np.float32).astype(np.float64)[geo.nbp:]
+    G = np.asarray(gate, dtype=np.float32).astype(np.float64)
+    return ((qp @ G.T) @ kp.T).astype(np.float32)
+
+
+def select_gated(geo, q_pool, k_pool, keep, gate, rows=None):
+    """select() with the learned-gate scores of one head's gate matrix."""
+    S = block_scores_gated_f32(geo, q_pool, k_pool, gate)
+    lists = []
+    every = np.arange(geo.nb, dtype=np.int64)
+    wanted = None if rows is None else set(int(r) for r in rows)
+    for i in range(geo.nb):
+        if wanted is not None and i not in wanted:
+            lists.append(None)
+        elif i < geo.nbp:
+            lists.append(every)
+        else:
+            vid = np.asarray(topk_row(S[i - geo.nbp], keep), dtype=np.int64) + geo.nbp
+            lists.append(np.concatenate([np.arange(geo.nbp, dtype=np.int64), vid]))
+    return lists
+
+
 # --------------------------------------------------------------------------
 # attention
 # --------------------------------------------------------------------------
@@ -386,6 +416,43 @@ def forward(prob, q, k, v, lists_override=None):
 
 
 # --------------------------------------------------------------------------
+# backward: gradients through the block-sparse attention
+# --------------------------------------------------------------------------
+# [PRISM] "같은 계산량 안에서 볼 곳을 고르는 Prism": the sparse attention is
+# also used in training (a 2K training step from 26.5 to 10.6 minutes), so
+# the same kept tiles carry the gradients.  With P the row-softmax of the
+# masked logits and O = P V, for a loss whose gradient at O is dO:
+#   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
+#   dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
+# Pad query rows have O = 0 by definition, so nothing flows through them.
+def kept_mask(geo, perm, lists):
+    """bool [N, N] in block order: query slot -> key slot is attended (its
+    key block is in the query block's list and the key is a real token)."""
+    kept = np.zeros((geo.nb, geo.nb), dtype=bool)
+    for i, lst in enumerate(lists):
+        kept[i, np.asarray(lst, dtype=np.int64)] = True
+    blk = np.arange(geo.N) // BLOCK
+    return kept[blk[:, None], blk[None, :]] & slot_valid(geo, perm)[None, :]
+
+
+def block_sparse_attention_grad(geo, perm, q_perm, k_perm, v_perm, do_perm, lists, scale):
+    """(dq, dk, dv), float64 [N, d] in block order, of one (batch, head)."""
+    q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q_perm, k_perm, v_perm, do_perm))
+    mask = kept_mask(geo, perm, lists)
+    logits = np.where(mask, (q @ k.T) * scale, -np.inf)
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    p = e / e.sum(axis=1, keepdims=True)
+    p[~slot_valid(geo, perm)] = 0.0
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    delta = (do * o).sum(axis=1, keepdims=True)
+    ds = p * (dp - delta)
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+# --------------------------------------------------------------------------
 # helpers used by the pins (brute force on tiny inputs)
 # --------------------------------------------------------------------------
 def topk_bruteforce(scores_row, k):
@@ -400,3 +467,83 @@ def topk_bruteforce(scores_row, k):
             found.append(sorted(sub))
     assert len(found) == 1
     return found[0]
+
+
+# --------------------------------------------------------------------------
+# window heads: spatial and temporal attention patterns, tile classes
+# --------------------------------------------------------------------------
+# [SVG] "Sparse VideoGen의 핵심 아이디어": a spatial head attends within the
+# same or nearby frames, a temporal head to the same spatial neighbourhood
+# across frames.  Both are written here as one window per head, (w_t, w_y,
+# w_x): query token (t, y, x) attends to video key (t', y', x') when
+# |t' - t| <= w_t, |y' - y| <= w_y and |x' - x| <= w_x, an axis with
+# UNBOUNDED (-1) being free.  The conditioning prefix stays dense as in
+# [REF2VA] "조건 토큰은 왜 다르게 다루나": every query attends to every prefix
+# key and prefix queries attend to every key.  Pad keys are excluded and pad
+# query rows are 0, as everywhere else.
+# [SVG] "이론적 sparsity와 물리적 sparsity의 차이": a 64 x 64 tile of block
+# pairs is full (every pair of real tokens attended), boundary (some) or
+# empty (none, skipped).
+UNBOUNDED = -1
+
+
+def token_coords(geo):
+    """int64 [N, 3]: (t, y, x) of every raster token; -1 for prefix tokens."""
+    c = np.full((geo.N, 3), -1, dtype=np.int64)
+    t, y, x = np.meshgrid(np.arange(geo.T), np.arange(geo.H), np.arange(geo.W), indexing="ij")
+    c[geo.P:, 0] = t.reshape(-1)
+    c[geo.P:, 1] = y.reshape(-1)
+    c[geo.P:, 2] = x.reshape(-1)
+    return c
+
+
+def window_mask(geo, window, rows=None):
+    """bool [N, N] in raster order: may query token n attend to key token m.
+    A negative window entry leaves its axis free.  With `rows` (raster query
+    indices) only those query rows are built: [len(rows), N]."""
+    c = token_coords(geo)
+    cq = c if rows is None else c[np.asarray(rows)]
+    vid = c[:, 0] >= 0
+    ok = np.ones((len(cq), geo.N), dtype=bool)
+    for a in range(3):
+        w = int(window[a])
+        if w >= 0:
+            ok &= np.abs(cq[:, None, a] - c[None, :, a]) <= w
+    ok |= ~vid[None, :]                  # prefix keys: every query
+    ok |= (cq[:, 0] < 0)[:, None]        # prefix queries: every key
+    return ok & geo.token_valid()[None, :]
+
+
+def window_attention(geo, q_bh, k_bh, v_bh, window, scale, rows=None):
+    """[N, d] raster-order output of one (batch, head) under its window:
+    logits over the allowed valid keys of each query, two-pass softmax,
+    pad query rows 0.  With `rows` only those raster query rows are
+    computed ([len(rows), d])."""
+    q = np.asarray(q_bh, dtype=np.float64)
+    k = np.asarray(k_bh, dtype=np.float64)
+    v = np.asarray(v_bh, dtype=np.float64)
+    idx = np.arange(geo.N) if rows is None else np.asarray(rows)
+    mask = window_mask(geo, window, idx)
+    logits = np.where(mask, (q[idx] @ k.T) * scale, -np.inf)
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    out = (e @ v) / e.sum(axis=1, keepdims=True)
+    out[~geo.token_valid()[idx]] = 0.0
+    return out
+
+
+def tile_classes(geo, perm, window):
+    """int64 [nb, nb] over block pairs in block order: 0 empty, 1 boundary,
+    2 full, judged on the pairs of real tokens (query block i, key block j)."""
+    mask = window_mask(geo, window)[perm][:, perm]            # block order
+    ok = slot_valid(geo, perm)
+    out = np.zeros((geo.nb, geo.nb), dtype=np.int64)
+    for i in range(geo.nb):
+        qi = np.arange(i * BLOCK, (i + 1) * BLOCK)
+        qi = qi[ok[qi]]
+        for j in range(geo.nb):
+            kj = np.arange(j * BLOCK, (j + 1) * BLOCK)
+            kj = kj[ok[kj]]
+            sub = mask[np.ix_(qi, kj)]
+            out[i, j] = 2 if sub.all() else (1 if sub.any() else 0)
+    return out

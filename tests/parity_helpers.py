@@ -42,11 +42,15 @@ def assert_close(got, want, what=""):
 class GpuRun:
     """The whole six-call sequence on device buffers, kept for inspection."""
 
-    def __init__(self, cfg, q, k, v, keep=None, dense=False):
+    def __init__(self, cfg, q, k, v, keep=None, dense=False, raster=False):
         self.cfg = cfg
+        self.raster = raster
         self.prob = problem(cfg, keep)
         self.attn = bsa.BlockSparseAttention(self.prob)
-        self.out = self.attn(q, k, v, dense=dense)
+        if raster:
+            self.out = self.attn.raster_call(q, k, v)
+        else:
+            self.out = self.attn(q, k, v, dense=dense)
         torch.cuda.synchronize()
         self.attn.check_status()
         s = self.attn.sizes

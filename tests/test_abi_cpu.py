@@ -31,7 +31,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol():
     names = declared_functions()
-    assert len(names) == 16, names
+    assert len(names) == 23, names
     for n in names:
         assert hasattr(bsa.lib(), n), n
     assert set(names) == set(bsa._SIGS), "binding and header disagree"
@@ -230,3 +230,22 @@ def test_last_error_is_per_thread():
     (st_b, msg_b), = seen["batch"]
     assert st_d == 3 and b"head_dim" in msg_d
     assert st_b == 2 and b"B and heads" in msg_b
+
+
+def test_raster_attention_validation():
+    """The raster attention call needs heads contiguous in a token row
+    (stride_h == head_dim) and is refused before any launch otherwise."""
+    p = base()              # head_dim 64
+    L = bsa.lib()
+    P = ctypes.byref(p)
+    args = lambda sh, osh=64: (P, 16, 16, 16, 16, 4096, 128, sh, 16, 16, 16, 4096, 128, osh,
+                               None, None)
+    assert L.bsa_sparse_attn_fwd_raster(*args(128)) == 3
+    assert b"stride_h" in L.bsa_last_error()
+    assert L.bsa_sparse_attn_fwd_raster(*args(60)) == 1        # not a multiple of 8
+    assert L.bsa_sparse_attn_fwd_raster(P, 16, 16, 16, 16, 4096, 128, 64, None, 16, 16, 4096,
+                                        128, 64, None, None) == 1
+    assert b"idx" in L.bsa_last_error()
+    assert L.bsa_pool_raster(P, 16, 16, 24, 4096, 128, 64, 16, 16, None) == 1
+    if not torch.cuda.is_available():
+        assert L.bsa_sparse_attn_fwd_raster(*args(64)) == 5    # valid: stops at the device check

@@ -46,18 +46,38 @@ def bh_sample(cfg, rng, count=3):
     return sorted(pairs)
 
 
-@pytest.mark.parametrize("name,over", FULL, ids=["%s%s" % (n, "-" + "-".join("%s=%s" % kv for kv in o.items()) if o else "") for n, o in FULL])
+# the permute-free path (raster tensors read through tensor-map boxes)
+FULL_RASTER = [
+    ("720p", {}),
+    ("720p_dyn", {}),
+    ("ref_prefix", {}),
+    ("lowres", {}),
+]
+
+
+def _ids(cases):
+    return ["%s%s" % (n, "-" + "-".join("%s=%s" % kv for kv in o.items()) if o else "")
+            for n, o in cases]
+
+
+@pytest.mark.parametrize("name,over", FULL, ids=_ids(FULL))
 def test_full_size_parity(name, over):
     check_full_size(name, over)
 
 
-def check_full_size(name, over):
+@pytest.mark.parametrize("name,over", FULL_RASTER, ids=_ids(FULL_RASTER))
+def test_full_size_parity_raster(name, over):
+    check_full_size(name, over, raster=True)
+
+
+def check_full_size(name, over, raster=False):
     """The checks of one full-size workload (also used by the maximum-size
-    test, which runs last)."""
+    test, which runs last).  raster=True runs the permute-free path, which
+    has no permuted tensors to compare."""
     cfg = config(name, **over)
     rng = np.random.default_rng(1234)
     q, k, v = make_qkv(cfg, 42000 + len(name), pad_fill=1e4, device="cuda")
-    run = GpuRun(cfg, q, k, v)
+    run = GpuRun(cfg, q, k, v, raster=raster)
     geo = O.Geometry(cfg)
     keep = run.prob.keep_blocks
     assert keep == O.keep_count(geo.nbv, cfg["keep_ratio"])
@@ -95,7 +115,8 @@ def check_full_size(name, over):
         op = [O.permute(geo, perm, x) for x in host]
         # permuted rows, bit-exact
         for t_dev, ref in zip((run.attn.qp, run.attn.kp, run.attn.vp), op):
-            assert np.array_equal(to_np64(t_dev[b, hh]), ref)
+            if not raster:
+                assert np.array_equal(to_np64(t_dev[b, hh]), ref)
         qpool, kpool = O.pool(geo, perm, op[0]), O.pool(geo, perm, op[1])
         np.testing.assert_allclose(gq_pool[b, hh], qpool, rtol=1e-5, atol=1e-5)
         np.testing.assert_allclose(gk_pool[b, hh], kpool, rtol=1e-5, atol=1e-5)

@@ -240,8 +240,9 @@ def test_rescale_path_growing_logits(name):
     assert int(run.attn.status.item()) == 0
 
 
+@pytest.mark.parametrize("raster", [False, True], ids=["perm", "raster"])
 @pytest.mark.parametrize("name", ["tiny", "ragged", "dyn"])
-def test_host_call_pipelined_by_head_groups(name):
+def test_host_call_pipelined_by_head_groups(name, raster):
     """bsa_forward_host on pinned host tensors, one head per group (so every
     case runs several groups; the dynamic case copies K whole first): same
     oracle bar as the device path."""
@@ -249,7 +250,7 @@ def test_host_call_pipelined_by_head_groups(name):
     (q, k, v), (qn, kn, vn) = seeded_inputs(cfg, seed=4242)
     run = GpuRun(cfg, q, k, v)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-    out = run.attn.host_call(qh, kh, vh, heads_per_group=1)
+    out = run.attn.host_call(qh, kh, vh, heads_per_group=1, raster=raster)
     torch.cuda.synchronize()
     run.attn.check_status()
     assert not out.is_cuda
@@ -262,3 +263,31 @@ def test_host_call_pipelined_by_head_groups(name):
     assert not got[:, ~geo.token_valid()].any(), "pad tokens must come out as 0"
     dev = to_np64(run.out)
     assert np.abs(got - dev).max() <= 3e-2
+
+
+def test_raster_path_matches_permuted_path_and_oracle(case):
+    """The permute-free sequence (layout -> pool_raster -> select ->
+    sparse_attn_fwd_raster) on Q, K, V sliced out of one fused
+    [B, N, 3, heads, d] tensor (token stride 3*heads*d) and O written into a
+    wider buffer: pooled means, index lists and the output are bit-identical
+    to the permuted path's, and the output matches the oracle."""
+    cfg, geo, run = case["cfg"], case["geo"], case["run"]
+    q, k, v = case["dev"]
+    B, N, h, d = q.shape
+    qkv = torch.stack([q, k, v], dim=2).contiguous()           # [B, N, 3, h, d]
+    qr, kr, vr = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    wide = torch.full((B, N, h, 2 * d), float("nan"), dtype=q.dtype, device=q.device)
+    out = wide[..., :d]
+    attn = bsa.BlockSparseAttention(run.prob)
+    attn.raster_call(qr, kr, vr, out=out)
+    torch.cuda.synchronize()
+    attn.check_status()
+    assert torch.equal(attn.q_pool, run.attn.q_pool) and torch.equal(attn.k_pool, run.attn.k_pool)
+    assert torch.equal(attn.cnt, run.attn.cnt)
+    nbp, kcap = geo.nbp, run.attn.sizes.list_capacity
+    assert torch.equal(attn.idx[:, :, nbp:], run.attn.idx[:, :, nbp:])
+    assert torch.equal(out, run.out)
+    assert torch.isnan(wide[..., d:]).all(), "wrote outside the output view"
+    want = oracle_forward_matched(cfg, case["host"], attn.idx.cpu().numpy(),
+                                  run.prob.keep_blocks)
+    assert_close(to_np64(out), want, cfg["name"] + " raster")
