@@ -80,6 +80,20 @@ def peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# tcgen05 dense bf16 rate per SM and clock (4,096 multiply-adds; measured
+# back-to-back with M=128, N>=128) and the SM count of a B200
+MMA_FLOP_PER_CLK_SM = 8192
+N_SM = 148
+
+
+def mma_rate_frac(tflops, clocks):
+    """The kernel's rate over the tensor cores' rate at the SM clock sampled
+    during the timed region (both sides at the same clock)."""
+    if not clocks or not clocks.get("sm_mhz"):
+        return None
+    return tflops / (MMA_FLOP_PER_CLK_SM * N_SM * clocks["sm_mhz"] * 1e6 / 1e12)
+
+
 def kept_tiles(cfg, keep):
     """64x64 tiles attention touches: video query blocks keep every prefix
     block plus `keep` video blocks; prefix query blocks keep every block."""
@@ -646,7 +660,8 @@ def main():
                              "true" if PATH["path"] == "raster" else "false",
                              "raster tensors" if PATH["path"] == "raster" else "permuted tensors"),
                          "peak_kind": "%s bf16 sustained" % pk_kind,
-                         "frac_of_burst": attn_tflops / pk["bf16_tflops"]},
+                         "frac_of_burst": attn_tflops / pk["bf16_tflops"],
+                         "frac_of_mma_rate_at_clock": mma_rate_frac(attn_tflops, res["clocks"])},
             "stage_ms": res["stage_ms"],
             "stage_gbs": stage_bandwidth(cfg, res["stage_ms"]),
             "gpu_launches": launches_per_step(cfg) * args.steps,

@@ -71,3 +71,11 @@ def test_stage_bandwidth():
     dyn = bench.stage_bandwidth(config("720p_dyn"), {"layout": 1.2, "permute": 1.9})
     assert dyn["layout"] == pytest.approx(R / 1.2e-3 / 1e9, rel=1e-3)
     assert bench.stage_bandwidth(cfg, {}) == {}
+
+
+def test_mma_rate_fraction_at_clock():
+    # 148 SMs x 8,192 FLOP per clock at 1,000 MHz is 1,212.4 TFLOP/s
+    assert bench.mma_rate_frac(1212.416, {"sm_mhz": 1000.0}) == pytest.approx(1.0)
+    assert bench.mma_rate_frac(606.208, {"sm_mhz": 1000.0}) == pytest.approx(0.5)
+    assert bench.mma_rate_frac(500.0, None) is None
+    assert bench.mma_rate_frac(500.0, {"sm_mhz": None}) is None
