@@ -105,6 +105,21 @@ __device__ __forceinline__ void report_timeout(volatile int* abort_flag, int32_t
   atomicCAS(status, 0, int32_t(BSA_ERR_TIMEOUT));
 }
 
+// Non-blocking probe of an mbarrier phase that is only issued once `dep`
+// has been computed: it lands among the exponentials, and its ~150-cycle
+// latency is spent on the ones that follow it.
+__device__ __forceinline__ bool mbar_test_after(uint32_t bar, uint32_t parity, float dep) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "f"(dep)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool bit_of(uint32_t lo, uint32_t hi, int c) {
   return ((c < 32 ? (lo >> c) : (hi >> (c - 32))) & 1u) != 0u;
 }
@@ -585,8 +600,12 @@ __global__ void __launch_bounds__(512, 1)
     ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
     const int n = ok ? *n_steps_sm : 0;
     const uint64_t* bm_row = bmask + int64_t(b) * g.nb;
+    // s_next: the next pair's S was ready when probed after this step's
+    // exponentials (a completed phase stays completed until this group
+    // frees S again)
+    bool s_next = false;
     for (int j = wg; ok && j < n; j += 2, ++k) {
-      const bool s_ready = __all_sync(0xffffffffu, mbar_test(bar_s, k & 1));
+      const bool s_ready = __all_sync(0xffffffffu, s_next || mbar_test(bar_s, k & 1));
       const uint32_t entry = steps[j];
       const int tile = int(entry & kTileMask);
       const uint32_t flags = entry >> kFlagShift;
@@ -629,9 +648,6 @@ __global__ void __launch_bounds__(512, 1)
           for (int c = 0; c < 64; ++c)
             if (bit_of(lo, hi, c)) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
         }
-        // the previous PV has normally finished by now: probe it here, use
-        // the answer after the exponentials
-        o_ready = k == 0 || __all_sync(0xffffffffu, mbar_test(bar_o + 8 * wg, (k - 1) & 1));
         const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
         if (mxs > m_used + 8.f) {
           if (m_used != -INFINITY) {
@@ -641,10 +657,14 @@ __global__ void __launch_bounds__(512, 1)
           m_used = mxs;
         }
         float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        // the previous PV of this group: probed halfway through the
+        // exponentials, the answer used after them
+        bool o_probe = true;
         if (all_valid) {
           // two columns per instruction for the scaling and the row sum
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
+            if (c == 32 && k > 0) o_probe = mbar_test_after(bar_o + 8 * wg, (k - 1) & 1, sum[0]);
             float x0, x1;
             fma_f32x2(x0, x1, __uint_as_float(r[c]), __uint_as_float(r[c + 1]), sl2, sl2, -m_used,
                       -m_used);
@@ -657,6 +677,7 @@ __global__ void __launch_bounds__(512, 1)
         } else {
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
+            if (c == 32 && k > 0) o_probe = mbar_test_after(bar_o + 8 * wg, (k - 1) & 1, sum[0]);
             const float p0 =
                 bit_of(lo, hi, c) ? ex2_approx(fmaf(__uint_as_float(r[c]), sl2, -m_used)) : 0.f;
             const float p1 = bit_of(lo, hi, c + 1)
@@ -667,7 +688,10 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
         l_sum = l_sum * factor + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+        s_next = mbar_test_after(bar_s, (k + 1) & 1, l_sum);
+        o_ready = __all_sync(0xffffffffu, o_probe);
       } else {
+        s_next = false;
         tc_fence_before();
         mbar_arrive(bar_sfree);
 #pragma unroll
