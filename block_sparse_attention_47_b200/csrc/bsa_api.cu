@@ -377,10 +377,12 @@ static bool make_pool_map(CUtensorMap* m, const Geo& g, const float* k_pool) {
   if (!fn) return false;
   cuuint64_t dims[2] = {cuuint64_t(g.d), cuuint64_t(g.B) * g.h * g.nb};
   cuuint64_t strides[1] = {cuuint64_t(g.d) * 4};
-  cuuint32_t box[2] = {32, 256};
+  // 64-row boxes of 16 channels (64-byte rows): a chunk of pooled keys is
+  // fetched by several issuing warps
+  cuuint32_t box[2] = {16, 64};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(k_pool), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

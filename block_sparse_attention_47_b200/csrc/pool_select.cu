@@ -109,12 +109,101 @@ __global__ void __launch_bounds__(kPoolThreads) pool_raster_kernel(
 }
 
 // ---- selection --------------------------------------------------------------
+// A CTA scores kSelRows query blocks per row group of kSelThreads threads
+// (RG groups share every staged key chunk) and then takes one query block
+// per warp in the top-k phase.
 constexpr int kSelThreads = 256;
-constexpr int kSelRows = 8;  // query blocks per CTA, one per warp in the top-k phase
+constexpr int kSelRows = 8;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+// One 256-bin radix pass of the top-k over a row's keys: counts the keys
+// that pass `in_set` by `digit_of`, then finds the digit D holding the
+// want-th largest (count(digit > D) < want <= count(digit >= D)); returns D,
+// lowers `want` by count(digit > D) and sets `at` to count(digit == D).
+template <class InSet, class DigitOf>
+__device__ __forceinline__ int radix_pass(const uint32_t* key, int nbv, uint32_t* hist, int lane,
+                                          int& want, int& at, InSet in_set, DigitOf digit_of) {
+  for (int i = lane; i < 256; i += 32) hist[i] = 0;
+  __syncwarp();
+  // eight keys in flight per lane before their histogram updates
+  for (int base = 0; base < nbv; base += 8 * 32) {
+    uint32_t u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int jv = base + 32 * i + lane;
+      u[i] = jv < nbv ? key[jv] : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (base + 32 * i + lane < nbv && in_set(u[i])) atomicAdd(&hist[digit_of(u[i])], 1u);
+  }
+  __syncwarp();
+  // lane l owns digits [8*(31-l), 8*(31-l)+8), scanned from the top
+  uint32_t local[8];
+  uint32_t tot = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    local[q] = hist[8 * (31 - lane) + (7 - q)];  // descending digits
+    tot += local[q];
+  }
+  uint32_t incl = tot;  // inclusive prefix over lanes (higher digits first)
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  const uint32_t excl = incl - tot;
+  const bool mine = (excl < uint32_t(want)) && (incl >= uint32_t(want));
+  const uint32_t who = __ballot_sync(0xffffffffu, mine);
+  const int src = __ffs(who) - 1;
+  int digit = 0, above = 0, here = 0;
+  if (mine) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (run + local[q] >= uint32_t(want)) {
+        digit = 8 * (31 - lane) + (7 - q);
+        above = int(run);
+        here = int(local[q]);
+        break;
+      }
+      run += local[q];
+    }
+  }
+  digit = __shfl_sync(0xffffffffu, digit, src);
+  above = __shfl_sync(0xffffffffu, above, src);
+  at = __shfl_sync(0xffffffffu, here, src);
+  want -= above;
+  __syncwarp();
+  return digit;
+}
+
+// The smallest key u in [lo, hi) with pred(u) (pred monotone: false then
+// true), or hi when there is none; 32 probes per step, so a 32-bit range
+// takes at most eight steps (twelve are allowed).
+template <class Pred>
+__device__ __forceinline__ uint64_t first_key_where(uint64_t lo, uint64_t hi, int lane, Pred pred) {
+  for (int it = 0; it < 12 && lo < hi; ++it) {
+    const uint64_t span = hi - lo;
+    const uint64_t p = lo + (span * uint64_t(lane)) / 32u;
+    const uint32_t b = __ballot_sync(0xffffffffu, pred(uint32_t(p)));
+    if (b == 0u) {
+      lo = __shfl_sync(0xffffffffu, p, 31) + 1u;
+    } else {
+      const int l = __ffs(b) - 1;
+      const uint64_t at = __shfl_sync(0xffffffffu, p, l);
+      const uint64_t before = __shfl_sync(0xffffffffu, p, l > 0 ? l - 1 : 0);
+      hi = at;
+      if (l > 0) lo = before + 1u;
+    }
+  }
+  return hi;
 }
 
 // Score tiles: KPT key blocks per thread, so kSelThreads * KPT pooled key
@@ -123,15 +212,19 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // consecutive rows hit 8 distinct bank quads).
 constexpr int kSelChunk = 32;
 constexpr int kSelStride = kSelChunk + 4;
+// the TMA form stages 16 channels (one 64-byte row) of 256 * KPT pooled keys
+// per chunk
+constexpr int kSelChunkTma = 16;
 
 template <int KPT>
 constexpr size_t select_tile_floats() {
   return size_t(kSelThreads) * KPT * kSelStride;
 }
 
-// dynamic smem: q rows [kSelRows][d] fp32, keys [kSelRows][nbv] u32, then
-// the key tile (KPT > 0), whose space the histograms [8 warps][256] u32 of
-// the top-k phase reuse.
+// dynamic smem: q rows [ROWS][d] fp32, keys [ROWS][nbv] u32, then the key
+// tile (KPT > 0), whose space the histograms [ROWS warps][256] u32 of the
+// top-k phase reuse.  ROWS = 8 * RG query blocks, NT = 256 * RG threads:
+// thread t takes key slot t % 256 (+ 256 u) for the 8 rows of group t / 256.
 //
 // KPT > 0: every score is one fmaf chain over the channels in ascending
 // order, as in the KPT == 0 form (one key block per thread read straight
@@ -144,38 +237,42 @@ constexpr size_t select_tile_floats() {
 // pooled query row is first mapped through its head's gate matrix,
 // q~_c = sum_e G[c][e] q_e (one fmaf chain in e order), and the key blocks
 // are scored against q~.  G = identity gives the ungated scores bit for bit.
-template <int KPT, bool TMA>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(
+template <int KPT, bool TMA, int RG>
+__global__ void __launch_bounds__(kSelThreads * RG) select_kernel(
     const __grid_constant__ CUtensorMap kmap, Geo g, const float* __restrict__ qpool,
     const float* __restrict__ kpool, const float* __restrict__ gate, int32_t* __restrict__ idx,
     int32_t* __restrict__ cnt) {
+  constexpr int NT = kSelThreads * RG, ROWS = kSelRows * RG;
   extern __shared__ __align__(16) unsigned char smem[];
   float* sq = reinterpret_cast<float*>(smem);
-  uint32_t* skey = reinterpret_cast<uint32_t*>(sq + kSelRows * g.d);
-  float* stile = reinterpret_cast<float*>(skey + ((kSelRows * g.nbv + 3) & ~3));
-  uint32_t* shist = KPT > 0 ? reinterpret_cast<uint32_t*>(stile) : skey + kSelRows * g.nbv;
+  uint32_t* skey = reinterpret_cast<uint32_t*>(sq + ROWS * g.d);
+  float* stile = reinterpret_cast<float*>(skey + ((ROWS * g.nbv + 3) & ~3));
+  uint32_t* shist = KPT > 0 ? reinterpret_cast<uint32_t*>(stile) : skey + ROWS * g.nbv;
 
   const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kSelRows;  // first video query block of this CTA
-  const int rows = min(kSelRows, g.nbv - i0);
+  const int i0 = blockIdx.x * ROWS;  // first video query block of this CTA
+  const int rows = min(ROWS, g.nbv - i0);
   const int64_t pool0 = int64_t(bh) * g.nb * g.d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = threadIdx.x % kSelThreads;  // key slot
+  const float* sqg = sq + (threadIdx.x / kSelThreads) * kSelRows * g.d;  // this group's rows
+  uint32_t* skeyg = skey + (threadIdx.x / kSelThreads) * kSelRows * g.nbv;
 
   // prefix query blocks attend densely: mark them once per (b, h)
   if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < g.nbp; i += kSelThreads) cnt[int64_t(bh) * g.nb + i] = -1;
+    for (int i = threadIdx.x; i < g.nbp; i += NT) cnt[int64_t(bh) * g.nb + i] = -1;
 
-  for (int e = threadIdx.x; e < kSelRows * g.d; e += kSelThreads) {
+  for (int e = threadIdx.x; e < ROWS * g.d; e += NT) {
     const int r = e / g.d, c = e % g.d;
     sq[e] = r < rows ? qpool[pool0 + int64_t(g.nbp + i0 + r) * g.d + c] : 0.f;
   }
   __syncthreads();
   if (gate) {
-    // 8 rows x d outputs, at most 4 per thread (d <= 128)
+    // ROWS rows x d outputs, at most 4 per thread (d <= 128)
     const float* G = gate + int64_t(bh % g.h) * g.d * g.d;
-    float gq[(kSelRows * 128) / kSelThreads];
+    float gq[(ROWS * 128) / NT];
     int n_out = 0;
-    for (int e = threadIdx.x; e < kSelRows * g.d; e += kSelThreads, ++n_out) {
+    for (int e = threadIdx.x; e < ROWS * g.d; e += NT, ++n_out) {
       const int r = e / g.d, c = e % g.d;
       const float4* gr = reinterpret_cast<const float4*>(G + int64_t(c) * g.d);
       const float4* qr = reinterpret_cast<const float4*>(sq + r * g.d);
@@ -191,42 +288,51 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     }
     __syncthreads();
     n_out = 0;
-    for (int e = threadIdx.x; e < kSelRows * g.d; e += kSelThreads, ++n_out) sq[e] = gq[n_out];
+    for (int e = threadIdx.x; e < ROWS * g.d; e += NT, ++n_out) sq[e] = gq[n_out];
     __syncthreads();
   }
 
   if constexpr (TMA) {
     // scores, register-tiled as below, with the pooled-key chunks (KT rows x
-    // 32 channels) brought in by TMA into two 128-byte-swizzled buffers: the
-    // next chunk's copy runs while this one is multiplied
+    // 16 channels, 64-byte rows) brought in by TMA into two 64-byte-swizzled
+    // buffers: the next chunk's copy runs while this one is multiplied.  A
+    // chunk is 64-row boxes spread over the warps (one thread keeps only ~25
+    // bytes per cycle of bulk copies in flight).  Each thread holds a
+    // channel quad of its 8 query rows in registers and sweeps its KPT keys
+    // with it: 8 broadcast and KPT 512-byte shared loads per 32 KPT FMAs.
+    constexpr int CH = kSelChunkTma;
     constexpr int KT = kSelThreads * KPT;
-    constexpr int TILE = KT * 128;
+    constexpr int TILE = KT * CH * 4;
+    constexpr int PARTS = KT / 64;
+    constexpr int ISSUERS = PARTS < NT / 32 ? PARTS : NT / 32;
+    static_assert(PARTS % ISSUERS == 0, "whole boxes per issuing warp");
     const uint32_t tiles = (smem_u32(stile) + 1023u) & ~1023u;
     const uint32_t bar = tiles + 2 * TILE;
-    const int ncpp = g.d / kSelChunk;                     // chunks per pass
+    const int ncpp = g.d / CH;                            // chunks per pass
     const int total = ((g.nbv + KT - 1) / KT) * ncpp;
     const int row0 = bh * g.nb + g.nbp;                   // this (b, h)'s first video key row
     if (threadIdx.x == 0) {
-      mbar_init(bar, 1);
-      mbar_init(bar + 8, 1);
+      mbar_init(bar, ISSUERS);
+      mbar_init(bar + 8, ISSUERS);
       fence_mbar_init();
     }
     __syncthreads();
+    // lane 0 of warp w < ISSUERS: boxes w, w + ISSUERS, .. of chunk c
+    const bool issuer = lane == 0 && warp < ISSUERS;
     auto issue = [&](int c) {
-      const int kb = (c / ncpp) * KT, cc = (c % ncpp) * kSelChunk;
+      const int kb = (c / ncpp) * KT, cc = (c % ncpp) * CH;
       const uint32_t b8 = bar + 8u * uint32_t(c & 1);
-      mbar_arrive_expect_tx(b8, TILE);
-#pragma unroll
-      for (int part = 0; part < KT / 256; ++part)
-        tma_load_2d(tiles + (c & 1) * TILE + part * 256 * 128, &kmap, b8, cc,
-                    row0 + kb + part * 256);
+      mbar_arrive_expect_tx(b8, TILE / ISSUERS);
+      for (int part = warp; part < PARTS; part += ISSUERS)
+        tma_load_2d(tiles + (c & 1) * TILE + part * 64 * CH * 4, &kmap, b8, cc,
+                    row0 + kb + part * 64);
     };
-    if (threadIdx.x == 0) issue(0);
+    if (issuer) issue(0);
     float acc[kSelRows][KPT];
     for (int c = 0; c < total; ++c) {
       // buffer (c+1)&1 was last read in chunk c-1, which ended in a barrier
-      if (threadIdx.x == 0 && c + 1 < total) issue(c + 1);
-      const int kb = (c / ncpp) * KT, cc = (c % ncpp) * kSelChunk;
+      if (issuer && c + 1 < total) issue(c + 1);
+      const int kb = (c / ncpp) * KT, cc = (c % ncpp) * CH;
       if (cc == 0) {
 #pragma unroll
         for (int r = 0; r < kSelRows; ++r)
@@ -236,37 +342,50 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       mbar_wait(bar + 8u * uint32_t(c & 1), (c >> 1) & 1, nullptr);
       const uint32_t buf = tiles + (c & 1) * TILE;
 #pragma unroll
-      for (int c4 = 0; c4 < kSelChunk / 4; ++c4) {
+      for (int c4 = 0; c4 < CH / 4; ++c4) {
         float4 kv[KPT];
 #pragma unroll
         for (int u = 0; u < KPT; ++u) {
-          const int rr = threadIdx.x + kSelThreads * u;
-          kv[u] = ld_shared_f4(buf + rr * 128 + ((c4 ^ (rr & 7)) << 4));
+          // 64-byte swizzle: 16-byte unit c4 of row rr sits at c4 ^ ((rr >> 1) & 3)
+          const int rr = kt + kSelThreads * u;
+          kv[u] = ld_shared_f4(buf + rr * 64 + ((c4 ^ ((rr >> 1) & 3)) << 4));
         }
+        float4 qv[kSelRows];
 #pragma unroll
-        for (int r = 0; r < kSelRows; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(sq + r * g.d + cc + 4 * c4);
+        for (int r = 0; r < kSelRows; ++r)
+          qv[r] = *reinterpret_cast<const float4*>(sqg + r * g.d + cc + 4 * c4);
+        // component-major, so that 8*KPT independent chains sit between two
+        // dependent FMAs (each chain still adds channels in ascending order)
 #pragma unroll
-          for (int u = 0; u < KPT; ++u) {
-            acc[r][u] = fmaf(qv.x, kv[u].x, acc[r][u]);
-            acc[r][u] = fmaf(qv.y, kv[u].y, acc[r][u]);
-            acc[r][u] = fmaf(qv.z, kv[u].z, acc[r][u]);
-            acc[r][u] = fmaf(qv.w, kv[u].w, acc[r][u]);
-          }
-        }
+        for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) acc[r][u] = fmaf(qv[r].x, kv[u].x, acc[r][u]);
+#pragma unroll
+        for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) acc[r][u] = fmaf(qv[r].y, kv[u].y, acc[r][u]);
+#pragma unroll
+        for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) acc[r][u] = fmaf(qv[r].z, kv[u].z, acc[r][u]);
+#pragma unroll
+        for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) acc[r][u] = fmaf(qv[r].w, kv[u].w, acc[r][u]);
       }
-      if (cc + kSelChunk == g.d) {
+      if (cc + CH == g.d) {
 #pragma unroll
         for (int u = 0; u < KPT; ++u) {
-          const int jv = kb + threadIdx.x + kSelThreads * u;
+          const int jv = kb + kt + kSelThreads * u;
           if (jv < g.nbv)
 #pragma unroll
-            for (int r = 0; r < kSelRows; ++r) skey[r * g.nbv + jv] = order_key(acc[r][u]);
+            for (int r = 0; r < kSelRows; ++r) skeyg[r * g.nbv + jv] = order_key(acc[r][u]);
         }
       }
       __syncthreads();
     }
   } else if constexpr (KPT > 0) {
+    static_assert(RG == 1, "one row group without TMA");
     // scores, register-tiled: thread t owns key blocks kb + t + 256*u
     // (u < KPT) for all 8 rows
     constexpr int KT = kSelThreads * KPT;
@@ -343,54 +462,75 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   if (warp < rows) {
     const uint32_t* key = skey + warp * g.nbv;
     uint32_t* hist = shist + warp * 256;
-    uint32_t prefix = 0;  // high bits decided so far
-    int want = g.keep;    // how many still to take among keys matching prefix
+    // First pass: 256 bins linear in the score value between the row's
+    // minimum and maximum (monotone in the key).  The top bits of float keys
+    // fall in a handful of bins (one per binade), which would serialise the
+    // histogram's atomics; value-linear bins spread them.  Then the usual
+    // four 8-bit passes over the keys, restricted to the chosen bin.
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int jv = lane; jv < g.nbv; jv += 32) {
+      const uint32_t u = key[jv];
+      kmin = min(kmin, u);
+      kmax = max(kmax, u);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const float fmin = key_value(kmin), fmax = key_value(kmax);
+    float scale = 256.f / (fmax - fmin);
+    if (!(scale < 3.0e38f)) scale = 0.f;  // equal or non-finite range: one bin
+    auto bin_of = [&](uint32_t u) {
+      return int(fminf((key_value(u) - fmin) * scale, 255.f));
+    };
+    int want = g.keep, at = 0;
+    const int vbin =
+        radix_pass(key, g.nbv, hist, lane, want, at, [](uint32_t) { return true; }, bin_of);
+    const uint32_t below = (1u << lane) - 1u;
+    // the bin is a contiguous key range [blo, bhi): bins grow with the key
+    const uint64_t kend = uint64_t(kmax) + 1u;
+    const uint64_t blo =
+        first_key_where(kmin, kend, lane, [&](uint32_t u) { return bin_of(u) >= vbin; });
+    const uint64_t bhi =
+        first_key_where(blo, kend, lane, [&](uint32_t u) { return bin_of(u) > vbin; });
+    auto in_bin = [&](uint32_t u) { return uint64_t(u) >= blo && uint64_t(u) < bhi; };
+    // the keys of that bin, gathered into a short list when they fit (the
+    // staging space after the histograms holds CAND keys per warp)
+    constexpr int CAND = KPT > 0 ? 512 : 0;
+    uint32_t* cand = shist + ROWS * 256 + warp * CAND;
+    int ncand = 0;
+    if constexpr (CAND > 0) {
+      for (int base = 0; base < g.nbv; base += 4 * 32) {
+        uint32_t u[4];
+        bool in[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int jv = base + 32 * i + lane;
+          u[i] = jv < g.nbv ? key[jv] : 0u;
+          in[i] = jv < g.nbv && in_bin(u[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t bal = __ballot_sync(0xffffffffu, in[i]);
+          const int pos = ncand + __popc(bal & below);
+          if (in[i] && pos < CAND) cand[pos] = u[i];
+          ncand += __popc(bal);
+        }
+      }
+      __syncwarp();
+    }
+    const bool short_list = CAND > 0 && ncand <= CAND;
+    uint32_t prefix = 0;  // high key bits decided so far
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       const uint32_t hi_mask = pass ? (0xFFFFFFFFu << (32 - 8 * pass)) : 0u;
-      for (int i = lane; i < 256; i += 32) hist[i] = 0;
-      __syncwarp();
-      for (int jv = lane; jv < g.nbv; jv += 32) {
-        const uint32_t u = key[jv];
-        if ((u & hi_mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFF], 1u);
-      }
-      __syncwarp();
-      // find the digit D: count(digit > D) < want <= count(digit >= D).
-      // lane l owns digits [8*(31-l), 8*(31-l)+8), scanned from the top.
-      uint32_t local[8];
-      uint32_t tot = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        local[q] = hist[8 * (31 - lane) + (7 - q)];  // descending digits
-        tot += local[q];
-      }
-      uint32_t incl = tot;  // inclusive prefix over lanes (higher digits first)
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-      }
-      const uint32_t excl = incl - tot;
-      const bool mine = (excl < uint32_t(want)) && (incl >= uint32_t(want));
-      const uint32_t who = __ballot_sync(0xffffffffu, mine);
-      const int src = __ffs(who) - 1;
-      int digit = 0, above = 0;
-      if (mine) {
-        uint32_t run = excl;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (run + local[q] >= uint32_t(want)) {
-            digit = 8 * (31 - lane) + (7 - q);
-            above = int(run);
-            break;
-          }
-          run += local[q];
-        }
-      }
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      want -= above;
+      auto digit_of = [&](uint32_t u) { return int((u >> shift) & 0xFFu); };
+      const int digit =
+          short_list
+              ? radix_pass(cand, ncand, hist, lane, want, at,
+                           [&](uint32_t u) { return (u & hi_mask) == prefix; }, digit_of)
+              : radix_pass(key, g.nbv, hist, lane, want, at,
+                           [&](uint32_t u) { return (u & hi_mask) == prefix && in_bin(u); },
+                           digit_of);
       prefix |= uint32_t(digit) << shift;
-      __syncwarp();
     }
     // prefix is now the exact key of the k-th best; `want` ties are needed
     const uint32_t thr = prefix;
@@ -398,17 +538,47 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     int32_t* out = idx + row * g.kcap;
     for (int p = lane; p < g.nbp; p += 32) out[p] = p;
     int written = g.nbp, ties = 0;
-    for (int base = 0; base < g.nbv; base += 32) {
-      const int jv = base + lane;
-      const uint32_t u = jv < g.nbv ? key[jv] : 0u;
-      const bool tie = (jv < g.nbv) && (u == thr);
-      const uint32_t tie_bal = __ballot_sync(0xffffffffu, tie);
-      const int tie_rank = ties + __popc(tie_bal & ((1u << lane) - 1u));
-      const bool take = (jv < g.nbv) && (u > thr || (tie && tie_rank < want));
-      const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      if (take) out[written + __popc(bal & ((1u << lane) - 1u))] = g.nbp + jv;
-      written += __popc(bal);
-      ties += __popc(tie_bal);
+    if (want == at) {
+      // every key equal to the k-th best is kept: take u >= thr
+      for (int base = 0; base < g.nbv; base += 4 * 32) {
+        uint32_t u[4];
+        bool take[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int jv = base + 32 * i + lane;
+          u[i] = jv < g.nbv ? key[jv] : 0u;
+          take[i] = jv < g.nbv && u[i] >= thr;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t bal = __ballot_sync(0xffffffffu, take[i]);
+          if (take[i]) out[written + __popc(bal & below)] = g.nbp + base + 32 * i + lane;
+          written += __popc(bal);
+        }
+      }
+    } else
+    for (int base = 0; base < g.nbv; base += 4 * 32) {
+      // four keys per lane loaded and voted on before the running counts
+      uint32_t u[4], tie_bal[4];
+      bool in[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int jv = base + 32 * i + lane;
+        in[i] = jv < g.nbv;
+        u[i] = in[i] ? key[jv] : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tie_bal[i] = __ballot_sync(0xffffffffu, in[i] && u[i] == thr);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool tie = (tie_bal[i] >> lane) & 1u;
+        const int tie_rank = ties + __popc(tie_bal[i] & below);
+        const bool take = in[i] && (u[i] > thr || (tie && tie_rank < want));
+        const uint32_t bal = __ballot_sync(0xffffffffu, take);
+        if (take) out[written + __popc(bal & below)] = g.nbp + base + 32 * i + lane;
+        written += __popc(bal);
+        ties += __popc(tie_bal[i]);
+      }
     }
     if (lane == 0) cnt[row] = g.nbp + g.keep;
   }
@@ -443,38 +613,43 @@ size_t select_tiled_smem_bytes(const Geo& g) {
          sizeof(float) * select_tile_floats<KPT>();
 }
 
-// the TMA form: two 128-byte-swizzled chunk buffers (1024-byte aligned) and
-// their two barriers after the row scores
-template <int KPT>
+// the TMA form: the rows of RG groups, two 128-byte-swizzled chunk buffers
+// (1024-byte aligned) and their two barriers
+template <int KPT, int RG>
 size_t select_tma_smem_bytes(const Geo& g) {
-  return sizeof(float) * kSelRows * g.d + sizeof(uint32_t) * ((kSelRows * g.nbv + 3) & ~3) +
-         1024 + 2 * size_t(kSelThreads) * KPT * 128 + 16;
+  const int rows = kSelRows * RG;
+  return sizeof(float) * rows * g.d + sizeof(uint32_t) * ((rows * g.nbv + 3) & ~3) + 1024 +
+         2 * size_t(kSelThreads) * KPT * kSelChunkTma * 4 + 16;
 }
 
-template <int KPT, bool TMA>
+template <int KPT, bool TMA, int RG = 1>
 cudaError_t launch_select_t(const Geo& g, size_t smem, const CUtensorMap* kmap,
                             const float* qpool, const float* kpool, const float* gate,
                             int32_t* idx, int32_t* cnt, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT, TMA>,
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT, TMA, RG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   CUtensorMap none{};
-  const int ctas = (g.nbv + kSelRows - 1) / kSelRows;
-  select_kernel<KPT, TMA><<<dim3(ctas, g.B * g.h), kSelThreads, smem, st>>>(
+  const int rows = kSelRows * RG;
+  const int ctas = (g.nbv + rows - 1) / rows;
+  select_kernel<KPT, TMA, RG><<<dim3(ctas, g.B * g.h), kSelThreads * RG, smem, st>>>(
       kmap ? *kmap : none, g, qpool, kpool, gate, idx, cnt);
   return cudaGetLastError();
 }
 }  // namespace
 
-// The TMA-fed form when a pooled-key map is given and its two buffers fit
-// next to the row scores; else the widest register tile that fits; else one
-// key block per thread.
+// The TMA-fed form when a pooled-key map is given and its buffers fit next
+// to the row scores (16 query blocks per CTA, else 8); else the widest
+// register tile that fits; else one key block per thread.
 cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, const float* gate,
                           const CUtensorMap* kmap, int32_t* idx, int32_t* cnt, cudaStream_t st) {
   constexpr size_t kMax = 227 * 1024;
-  if (kmap && select_tma_smem_bytes<2>(g) <= kMax)
-    return launch_select_t<2, true>(g, select_tma_smem_bytes<2>(g), kmap, qpool, kpool, gate, idx,
-                                    cnt, st);
+  if (kmap && select_tma_smem_bytes<2, 2>(g) <= kMax)
+    return launch_select_t<2, true, 2>(g, select_tma_smem_bytes<2, 2>(g), kmap, qpool, kpool,
+                                       gate, idx, cnt, st);
+  if (kmap && select_tma_smem_bytes<2, 1>(g) <= kMax)
+    return launch_select_t<2, true>(g, select_tma_smem_bytes<2, 1>(g), kmap, qpool, kpool, gate,
+                                    idx, cnt, st);
   if (select_tiled_smem_bytes<4>(g) <= kMax)
     return launch_select_t<4, false>(g, select_tiled_smem_bytes<4>(g), nullptr, qpool, kpool, gate,
                                      idx, cnt, st);
