@@ -114,12 +114,16 @@ def tile_flops(cfg):
 def stage_bandwidth(cfg, stage_ms):
     """Achieved GB/s of the memory-bound stages: algorithmic bytes (one bf16
     [B, N, heads, d] tensor is R bytes) over each stage's time.  permute
-    reads and writes Q, K, V (6R), pool reads permuted Q and K (2R),
-    unpermute reads and writes O (2R), the dynamic layout reads K (R); the
-    pooled outputs and index lists are small and not counted."""
+    (with the pooling fused in) reads and writes Q, K, V (6R), a separate
+    pool would read permuted Q and K (2R), unpermute reads and writes O (2R),
+    the dynamic layout reads K (R); the pooled outputs and index lists are
+    small and not counted."""
     s = derived_sizes(cfg)
     R = cfg["B"] * s["N"] * cfg["heads"] * cfg["head_dim"] * 2
-    nbytes = {"permute": 6 * R, "pool": 2 * R, "unpermute": 2 * R}
+    if PATH["path"] == "raster":
+        nbytes = {"pool": 2 * R}   # pool_raster reads raster Q and K
+    else:
+        nbytes = {"permute": 6 * R, "unpermute": 2 * R}
     if cfg["block_mode"] == 1:
         nbytes["layout"] = R
     return {k: round(v / (stage_ms[k] * 1e-3) / 1e9, 1)
@@ -261,16 +265,13 @@ def run_step(bsa, attn, q, k, v, out, ev):
     if ev:
         ev[1].record()
     if not raster:
-        bsa.permute(p, L, q, attn.qp)
-        bsa.permute(p, L, k, attn.kp)
-        bsa.permute(p, L, v, attn.vp)
+        # the permutes and the pooling in one pass (its time is the
+        # "permute" stage; "pool" stays empty)
+        bsa.permute_pool(p, L, q, k, v, attn.qp, attn.kp, attn.vp, attn.q_pool, attn.k_pool)
     if ev:
         ev[2].record()
-    if windows is None:
-        if raster:
-            bsa.pool_raster(p, L, q, k, attn.q_pool, attn.k_pool)
-        else:
-            bsa.pool(p, L, attn.qp, attn.kp, attn.q_pool, attn.k_pool)
+    if windows is None and raster:
+        bsa.pool_raster(p, L, q, k, attn.q_pool, attn.k_pool)
     if ev:
         ev[3].record()
     if windows is not None:
@@ -302,7 +303,7 @@ def launches_per_step(cfg):
         return layout + 1
     if PATH["path"] == "raster":
         return layout + 1 + 1 + 1
-    return layout + 3 + 1 + 1 + 1 + 1
+    return layout + 1 + 1 + 1 + 1
 
 
 def window_heads(cfg, pattern):

@@ -105,6 +105,8 @@ _SIGS = {
     "bsa_layout": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _I64, _I64, _I64, _P, _P]),
     "bsa_permute": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _I64, _I64, _I64, _P, _P]),
     "bsa_pool": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P]),
+    "bsa_permute_pool": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _I64, _I64, _I64,
+                                        _P, _P, _P, _P, _P, _P]),
     "bsa_select_topk": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P]),
     "bsa_sparse_attn_fwd": (ctypes.c_int, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _P,
                                            _P, _P]),
@@ -197,6 +199,19 @@ def permute(prob, layout_buf, x_raster, x_perm, stream=None):
 def pool(prob, layout_buf, q_perm, k_perm, q_pool, k_pool, stream=None):
     _check(lib().bsa_pool(ctypes.byref(prob), _ptr(layout_buf), _ptr(q_perm), _ptr(k_perm),
                           _ptr(q_pool), _ptr(k_pool), _stream(stream)))
+
+
+def permute_pool(prob, layout_buf, q_raster, k_raster, v_raster, q_perm, k_perm, v_perm, q_pool,
+                 k_pool, stream=None):
+    """permute(Q), permute(K), permute(V) and pool in one pass; Q, K and V
+    must share their strides."""
+    sb, sn, sh = _raster_strides(q_raster)
+    if _raster_strides(k_raster) != (sb, sn, sh) or _raster_strides(v_raster) != (sb, sn, sh):
+        raise ValueError("permute_pool: q, k and v must share their strides")
+    _check(lib().bsa_permute_pool(ctypes.byref(prob), _ptr(layout_buf), _ptr(q_raster),
+                                  _ptr(k_raster), _ptr(v_raster), sb, sn, sh, _ptr(q_perm),
+                                  _ptr(k_perm), _ptr(v_perm), _ptr(q_pool), _ptr(k_pool),
+                                  _stream(stream)))
 
 
 def select_topk(prob, q_pool, k_pool, idx, cnt, stream=None):
@@ -395,8 +410,16 @@ class BlockSparseAttention:
         p = self.prob
         if out is None:
             out = torch.empty_like(q)
-        self.plan(q, k, stream)
-        permute(p, self.layout_buf, v, self.vp, stream)
+        layout(p, k, self.layout_buf, stream)
+        if _raster_strides(q) == _raster_strides(k) == _raster_strides(v):
+            permute_pool(p, self.layout_buf, q, k, v, self.qp, self.kp, self.vp, self.q_pool,
+                         self.k_pool, stream)
+        else:
+            permute(p, self.layout_buf, q, self.qp, stream)
+            permute(p, self.layout_buf, k, self.kp, stream)
+            permute(p, self.layout_buf, v, self.vp, stream)
+            pool(p, self.layout_buf, self.qp, self.kp, self.q_pool, self.k_pool, stream)
+        select_topk(p, self.q_pool, self.k_pool, self.idx, self.cnt, stream)
         if dense:
             dense_attn_fwd(p, self.layout_buf, self.qp, self.kp, self.vp, self.op, self.status,
                            stream)

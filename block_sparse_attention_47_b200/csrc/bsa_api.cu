@@ -369,8 +369,36 @@ bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void*
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_pool launch");
 }
 
+bsa_status bsa_permute_pool(const bsa_problem* prob, const void* layout_buf, const void* q_raster,
+                            const void* k_raster, const void* v_raster, int64_t stride_b,
+                            int64_t stride_n, int64_t stride_h, void* q_perm, void* k_perm,
+                            void* v_perm, float* q_pool, float* k_pool, void* stream) {
+  g_last_error[0] = 0;
+  BSA_RANGE();
+  Geo g;
+  BSA_TRY(make_geo(prob, &g));
+  BSA_TRY(check_ptr(layout_buf, "layout_buf"));
+  BSA_TRY(check_ptr(q_raster, "q_raster"));
+  BSA_TRY(check_ptr(k_raster, "k_raster"));
+  BSA_TRY(check_ptr(v_raster, "v_raster"));
+  BSA_TRY(check_ptr(q_perm, "q_perm"));
+  BSA_TRY(check_ptr(k_perm, "k_perm"));
+  BSA_TRY(check_ptr(v_perm, "v_perm"));
+  BSA_TRY(check_ptr(q_pool, "q_pool"));
+  BSA_TRY(check_ptr(k_pool, "k_pool"));
+  BSA_TRY(check_strides(g, stride_b, stride_n, stride_h, "q_raster"));
+  BSA_TRY(check_device());
+  cudaError_t e = bsa::launch_permute_pool(
+      g, bsa::layout_ptrs(g, const_cast<void*>(layout_buf)),
+      static_cast<const __nv_bfloat16*>(q_raster), static_cast<const __nv_bfloat16*>(k_raster),
+      static_cast<const __nv_bfloat16*>(v_raster), stride_b, stride_n, stride_h,
+      static_cast<__nv_bfloat16*>(q_perm), static_cast<__nv_bfloat16*>(k_perm),
+      static_cast<__nv_bfloat16*>(v_perm), q_pool, k_pool, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_permute_pool launch");
+}
+
 // 2-D map over the pooled keys [B*heads*nb rows, d] fp32 for the TMA-fed
-// score tiles (32 channels x 256 rows per box, 128-byte swizzle); false when
+// score tiles (16 channels x 64 rows per box, 64-byte swizzle); false when
 // the driver offers no encoder (the select kernel then loads the tiles itself)
 static bool make_pool_map(CUtensorMap* m, const Geo& g, const float* k_pool) {
   EncodeTiledFn fn = encode_fn();
@@ -840,10 +868,8 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
       BSA_TRY(bsa_sparse_attn_fwd_raster(&sub, buf->layout_buf, rq, rk, rv, sb, sn, sh, idx, cnt,
                                          ro, sb, sn, sh, dev_status, st));
     } else {
-      BSA_TRY(bsa_permute(&sub, buf->layout_buf, rq, sb, sn, sh, pq, st));
-      BSA_TRY(bsa_permute(&sub, buf->layout_buf, rk, sb, sn, sh, pk, st));
-      BSA_TRY(bsa_permute(&sub, buf->layout_buf, rv, sb, sn, sh, pv, st));
-      BSA_TRY(bsa_pool(&sub, buf->layout_buf, pq, pk, qpool, kpool, st));
+      BSA_TRY(bsa_permute_pool(&sub, buf->layout_buf, rq, rk, rv, sb, sn, sh, pq, pk, pv, qpool,
+                               kpool, st));
       BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
       BSA_TRY(bsa_sparse_attn_fwd(&sub, buf->layout_buf, pq, pk, pv, idx, cnt, po, dev_status,
                                   st));

@@ -96,6 +96,10 @@ cudaError_t launch_permute(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* x, 
 cudaError_t launch_unpermute(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* op,
                              __nv_bfloat16* o, int64_t sb, int64_t sn, int64_t sh,
                              cudaStream_t st);
+cudaError_t launch_permute_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* q,
+                                const __nv_bfloat16* k, const __nv_bfloat16* v, int64_t sb,
+                                int64_t sn, int64_t sh, __nv_bfloat16* qp, __nv_bfloat16* kp,
+                                __nv_bfloat16* vp, float* qpool, float* kpool, cudaStream_t st);
 cudaError_t launch_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* qp,
                         const __nv_bfloat16* kp, float* qpool, float* kpool, cudaStream_t st);
 // kmap (optional): 2-D map over the pooled keys [B*heads*nb rows, d] fp32,

@@ -110,10 +110,8 @@ extern "C" bsa_status bsa_forward_noalloc(const bsa_problem* prob, const void* q
     if (s_ != BSA_OK) return s_;   \
   } while (0)
   BSA_STEP(bsa_layout(prob, k_raster, stride_b, stride_n, stride_h, layout, stream));
-  BSA_STEP(bsa_permute(prob, layout, q_raster, stride_b, stride_n, stride_h, qp, stream));
-  BSA_STEP(bsa_permute(prob, layout, k_raster, stride_b, stride_n, stride_h, kp, stream));
-  BSA_STEP(bsa_permute(prob, layout, v_raster, stride_b, stride_n, stride_h, vp, stream));
-  BSA_STEP(bsa_pool(prob, layout, qp, kp, q_pool, k_pool, stream));
+  BSA_STEP(bsa_permute_pool(prob, layout, q_raster, k_raster, v_raster, stride_b, stride_n,
+                            stride_h, qp, kp, vp, q_pool, k_pool, stream));
   BSA_STEP(bsa_select_topk(prob, q_pool, k_pool, idx, cnt, stream));
   BSA_STEP(bsa_sparse_attn_fwd(prob, layout, qp, kp, vp, idx, cnt, op, dev_status, stream));
   BSA_STEP(bsa_unpermute(prob, layout, op, o_raster, o_stride_b, o_stride_n, o_stride_h, stream));

@@ -21,6 +21,7 @@
  * The call sequence for one attention layer:
  *   bsa_layout -> bsa_permute (Q, K, V) -> bsa_pool -> bsa_select_topk
  *   -> bsa_sparse_attn_fwd -> bsa_unpermute
+ * (bsa_permute_pool does the permutes and the pooling in one pass).
  * bsa_dense_attn_fwd is the same attention kernel over every tile (the
  * speed-up denominator).
  *
@@ -154,6 +155,19 @@ bsa_status bsa_permute(const bsa_problem* prob, const void* layout_buf, const vo
  * its 64 tokens). */
 bsa_status bsa_pool(const bsa_problem* prob, const void* layout_buf, const void* q_perm,
                     const void* k_perm, float* q_pool, float* k_pool, void* stream);
+
+/* bsa_permute of Q, K and V and bsa_pool in one pass: the block means are
+ * summed from the rows as they are moved, so the permuted Q and K are not
+ * read back (the Prism section's block means; Sparse VideoGen on TPU,
+ * aibase.it, section "실무에서 배울 최적화 기준": the permutation is part of
+ * the cost to be measured).  Outputs equal those of the separate calls bit
+ * for bit.  q_raster, k_raster and v_raster share the element strides
+ * (stride_b, stride_n, stride_h); q_perm, k_perm, v_perm, q_pool and k_pool
+ * are laid out as for bsa_permute and bsa_pool. */
+bsa_status bsa_permute_pool(const bsa_problem* prob, const void* layout_buf, const void* q_raster,
+                            const void* k_raster, const void* v_raster, int64_t stride_b,
+                            int64_t stride_n, int64_t stride_h, void* q_perm, void* k_perm,
+                            void* v_perm, float* q_pool, float* k_pool, void* stream);
 
 /* Per (batch, head) and video query block i: scores S[i, j] = q_pool[i] .
  * k_pool[j] (fp32) over video key blocks j; keep the keep_blocks best by

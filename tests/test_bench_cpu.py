@@ -60,17 +60,23 @@ def test_traffic_figure_only_for_its_workload(monkeypatch):
     assert bench.attn_traffic(cfg, 0.25) is None
 
 
-def test_stage_bandwidth():
+def test_stage_bandwidth(monkeypatch):
     cfg = config("720p")
     R = 2 * 122880 * 24 * 128 * 2                      # one raster tensor, 1.51 GB
-    gbs = bench.stage_bandwidth(cfg, {"permute": 1.9, "pool": 0.6, "unpermute": 0.65,
-                                      "layout": 0.009, "select": 4.7})
-    assert gbs["permute"] == pytest.approx(6 * R / 1.9e-3 / 1e9, rel=1e-3)
-    assert gbs["pool"] == pytest.approx(2 * R / 0.6e-3 / 1e9, rel=1e-3)
-    assert set(gbs) == {"permute", "pool", "unpermute"}  # fixed layout reads nothing
+    # permuted path: permute (pooling fused in) moves Q, K, V; no pool stage
+    gbs = bench.stage_bandwidth(cfg, {"permute": 1.4, "pool": 0.003, "unpermute": 0.65,
+                                      "layout": 0.009, "select": 2.9})
+    assert gbs["permute"] == pytest.approx(6 * R / 1.4e-3 / 1e9, rel=1e-3)
+    assert gbs["unpermute"] == pytest.approx(2 * R / 0.65e-3 / 1e9, rel=1e-3)
+    assert set(gbs) == {"permute", "unpermute"}  # fixed layout reads nothing
     dyn = bench.stage_bandwidth(config("720p_dyn"), {"layout": 1.2, "permute": 1.9})
     assert dyn["layout"] == pytest.approx(R / 1.2e-3 / 1e9, rel=1e-3)
     assert bench.stage_bandwidth(cfg, {}) == {}
+    # permute-free path: pool_raster reads raster Q and K
+    monkeypatch.setitem(bench.PATH, "path", "raster")
+    gbs = bench.stage_bandwidth(cfg, {"permute": 0.0, "pool": 0.6, "unpermute": 0.0})
+    assert set(gbs) == {"pool"}
+    assert gbs["pool"] == pytest.approx(2 * R / 0.6e-3 / 1e9, rel=1e-3)
 
 
 def test_mma_rate_fraction_at_clock():

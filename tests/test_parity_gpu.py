@@ -115,6 +115,25 @@ def test_pool(case):
             np.testing.assert_allclose(gk[b, hh], O.pool(geo, perm, ok_), rtol=1e-5, atol=1e-5)
 
 
+def test_permute_pool_equals_separate_calls(case):
+    """The fused permute + pool (what the forward call runs) against
+    bsa_permute x3 and bsa_pool on the same layout: bit for bit."""
+    run = case["run"]
+    q, k, v = case["dev"]
+    p, L = run.prob, run.attn.layout_buf
+    qp, kp, vp = (torch.empty_like(t) for t in (run.attn.qp, run.attn.kp, run.attn.vp))
+    qpool, kpool = torch.empty_like(run.attn.q_pool), torch.empty_like(run.attn.k_pool)
+    bsa.permute(p, L, q, qp)
+    bsa.permute(p, L, k, kp)
+    bsa.permute(p, L, v, vp)
+    bsa.pool(p, L, qp, kp, qpool, kpool)
+    torch.cuda.synchronize()
+    for a, b in ((qp, run.attn.qp), (kp, run.attn.kp), (vp, run.attn.vp)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for a, b in ((qpool, run.attn.q_pool), (kpool, run.attn.k_pool)):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
 def test_select_lists(case):
     cfg, geo, run = case["cfg"], case["geo"], case["run"]
     qn, kn, vn = case["host"]
