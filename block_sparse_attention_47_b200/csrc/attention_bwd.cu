@@ -17,10 +17,18 @@
 //        the query blocks that kept them (transposed lists, built as
 //        bitmaps); per step S^T = K Q^T and dP^T = V dO^T (M=128 N=64), P^T
 //        and dS^T in registers, then dV += P^T dO and dK += dS^T Q.
-// One thread issues the copies and MMAs in step order; the 128 row threads
-// turn each step's S/dP into P/dS.  K/V (dQ) or Q/dO (dKdV) tiles are
-// double-buffered so the next step's copies run under the current step.
-// Every wait is bounded (2 s) and reports BSA_ERR_TIMEOUT as the forward.
+// P needs no running maximum (the forward's statistics fix it), so steps
+// are independent: two groups of row threads take alternate steps, each
+// with its own S/dP columns in tensor memory, and one thread issues the
+// copies and MMAs so that the tensor pipe always holds the next step's
+// S/dP while a group turns the previous one into P/dS:
+//     iteration j:  S/dP of step j,  then the accumulation of step j-1.
+// Step tiles (K/V, or Q/dO with their rows' lse2 and D) go through a
+// 4-stage ring loaded one step ahead.  In dKdV, P^T and dS^T are written
+// over the group's own S and dP columns (the two accumulators fill the
+// rest of tensor memory), so a group's next S/dP waits for its previous
+// accumulation to finish.  Every wait is bounded (2 s) and reports
+// BSA_ERR_TIMEOUT as the forward.
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -31,30 +39,84 @@ constexpr uint32_t kTileMask = 0x1FFFu, kFlagShift = 13;
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kThreads = 256;             // warps 0-3 rows, 4 issuer, 5-7 idle
+  // warps 0-3 / 4-7: row groups 0 / 1 (alternate steps); 8: issuer; 9: steps
+  static constexpr int kThreads = 320;
   static constexpr int KB = D / 64;                // 64-column boxes
+  static constexpr int NS = 4;                     // step-tile ring stages
   static constexpr int TILE64 = 64 * D * 2;        // one 64-row tile
   static constexpr int TILE128 = 128 * D * 2;      // the CTA's own 128-row tile
   static constexpr int BOX64 = 64 * 128, BOX128 = 128 * 128;
-  // dQ: own = Q | dO (128 rows each); stages = K | V (64 rows) x 2
-  // dKdV: own = K | V; stages = Q | dO x 2, plus lse2 | delta (64 floats) x 2
+  // dQ: own = Q | dO (128 rows each); stages = K | V (64 rows)
+  // dKdV: own = K | V; stages = Q | dO, plus lse2 | delta (64 floats)
   static constexpr int OFF_OWN_A = 0;
   static constexpr int OFF_OWN_B = TILE128;
-  static constexpr int OFF_STG = 2 * TILE128;             // [stage][a | b] 64-row tiles
-  static constexpr int OFF_VEC = OFF_STG + 4 * TILE64;    // [stage][lse2 | delta][64] fp32
-  static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * 64 * 4;
-  // full[2] empty[2] mma1 ready own steps done drain
-  static constexpr int N_BARS = 10;
-  static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;     // uint32 A, B, F [kMaxWords]
+  static constexpr int OFF_STG = 2 * TILE128;              // [stage][a | b] 64-row tiles
+  static constexpr int OFF_VEC = OFF_STG + NS * 2 * TILE64; // [stage][lse2 | delta][64] fp32
+  static constexpr int OFF_BAR = OFF_VEC + NS * 2 * 64 * 4;
+  // full[NS] empty[NS] s_ready[2] sfree[2] x_ready[2] x_free[2] own steps done drain
+  static constexpr int N_BARS = 2 * NS + 8 + 4;
+  static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;      // uint32 A, B, F [kMaxWords]
   static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
   static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  // tensor memory: S [0,64) | dP [64,128) | P or dS [128,160) | dS [160,192)
-  // | accumulators from 256 (dQ; or dV then dK)
-  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_X = 128, COL_Y = 160, COL_ACC = 256;
+  // tensor memory: group w's S at 128w, dP at 128w + 64.  dQ: dS of group w
+  // at 256 + 32w, the accumulator at 384.  dKdV: P^T over S, dS^T over dP,
+  // dV at 256 and dK at 256 + D.
+  static constexpr uint32_t COL_DQ_X = 256, COL_DQ_ACC = 384, COL_DV = 256, COL_DK = 256 + D;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(COL_DK + D <= TMEM_COLS, "tensor memory budget");
 };
+
+struct BwdBars {
+  uint32_t full, empty, s_ready, sfree, x_ready, x_free, own, steps, done, drain;
+};
+
+template <int D>
+__device__ __forceinline__ BwdBars bwd_bars(uint32_t bar0) {
+  using C = BwdCfg<D>;
+  BwdBars b;
+  b.full = bar0;
+  b.empty = bar0 + 8 * C::NS;
+  b.s_ready = bar0 + 16 * C::NS;
+  b.sfree = b.s_ready + 16;
+  b.x_ready = b.s_ready + 32;
+  b.x_free = b.s_ready + 48;
+  b.own = b.s_ready + 64;
+  b.steps = b.own + 8;
+  b.done = b.own + 16;
+  b.drain = b.own + 24;
+  return b;
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_init_bars(const BwdBars& b) {
+  using C = BwdCfg<D>;
+  for (int s = 0; s < C::NS; ++s) {
+    mbar_init(b.full + 8 * s, 1);
+    mbar_init(b.empty + 8 * s, 1);
+  }
+  for (int w = 0; w < 2; ++w) {
+    mbar_init(b.s_ready + 8 * w, 1);
+    mbar_init(b.sfree + 8 * w, 128);
+    mbar_init(b.x_ready + 8 * w, 128);
+    mbar_init(b.x_free + 8 * w, 1);
+  }
+  mbar_init(b.own, 256);
+  mbar_init(b.steps, 32);
+  mbar_init(b.done, 1);
+  mbar_init(b.drain, 1);
+}
+
+#define BSA_TMEM_ST16(taddr, r)                                                               \
+  asm volatile(                                                                               \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "                                        \
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"                         \
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),                                          \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),       \
+      "r"(r[15])                                                                              \
+      : "memory")
 
 __device__ __forceinline__ void report_timeout(volatile int* abort_flag, int32_t* status) {
   *abort_flag = 1;
@@ -117,62 +179,22 @@ __device__ __forceinline__ void store_row_swizzled(uint32_t tile, int box_bytes,
   }
 }
 
-// ============================================================================
-// dQ: CTA = query pair, walk = union of the two key lists
-// ============================================================================
-template <int D>
-__global__ void __launch_bounds__(256, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-                       Geo g, const BwdIO io) {
-  using C = BwdCfg<D>;
-  extern __shared__ unsigned char smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* sm = smem_raw + (base - raw);
-  const uint32_t sQ = base + C::OFF_OWN_A, sdO = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
-  const uint32_t bar0 = base + C::OFF_BAR;
-  const uint32_t bar_full = bar0, bar_empty = bar0 + 16, bar_mma1 = bar0 + 32;
-  const uint32_t bar_ready = bar0 + 40, bar_own = bar0 + 48, bar_steps = bar0 + 56;
-  const uint32_t bar_done = bar0 + 64, bar_drain = bar0 + 72;
-  uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
-  uint32_t* bmB = bmA + kMaxWords;
-  uint32_t* bmF = bmA + 2 * kMaxWords;
-  uint16_t* steps = reinterpret_cast<uint16_t*>(sm + C::OFF_STEPS);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
-  int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
-  auto stage_a = [&](int s) { return sStg + s * 2 * C::TILE64; };  // K
-  auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // V
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+// The walk of a CTA (run by warp 9): bitmaps A and B over the walked blocks
+// (query pair: the kept key blocks of its two query blocks; key pair: the
+// query blocks that kept either key block), bmF marks blocks without pad
+// slots, then the step table.
+__device__ __forceinline__ void bwd_walk(const Geo& g, const BwdIO& io, bool transposed, int pair,
+                                         int bh, int b, int nw, uint32_t* bmA, uint32_t* bmB,
+                                         uint32_t* bmF, uint16_t* steps, int* n_steps_sm,
+                                         uint32_t bar_steps, int lane) {
+  if (transposed) {
+    const uint32_t* kt = io.kmask + (int64_t(bh) * g.nb) * nw;
+    for (int w = lane; w < nw; w += 32) {
+      bmA[w] = 2 * pair < g.nb ? __ldg(kt + int64_t(2 * pair) * nw + w) : 0u;
+      bmB[w] = 2 * pair + 1 < g.nb ? __ldg(kt + int64_t(2 * pair + 1) * nw + w) : 0u;
     }
-    mbar_init(bar_mma1, 1);
-    mbar_init(bar_ready, 128);
-    mbar_init(bar_own, 128);
-    mbar_init(bar_steps, 32);
-    mbar_init(bar_done, 1);
-    mbar_init(bar_drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 4) {
-    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int nw = (g.nb + 31) >> 5;
-
-  if (warp == 5) {
-    // ---- the walk: union of the two query blocks' key lists (a dense row
-    // keeps every block); bmF marks key blocks without pad slots
+  } else {
+    // a dense row keeps every block
     for (int w = lane; w < nw; w += 32) bmA[w] = bmB[w] = 0u;
     __syncwarp();
     for (int hf = 0; hf < 2; ++hf) {
@@ -194,40 +216,120 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
     }
-    for (int w = lane; w < nw; w += 32) {
-      uint32_t f = 0u;
-      for (int i = 0; i < 32; ++i)
-        if (32 * w + i < g.nb && __ldg(io.bfull + int64_t(b) * g.nb + 32 * w + i)) f |= 1u << i;
-      bmF[w] = f;
-    }
-    __syncwarp();
-    const int n = build_steps(bmA, bmB, bmF, nw, steps, lane);
-    if (lane == 0) *n_steps_sm = n;
-    __syncwarp();
-    mbar_arrive(bar_steps);
-  } else if (warp == 4) {
+  }
+  for (int w = lane; w < nw; w += 32) {
+    uint32_t f = 0u;
+    for (int i = 0; i < 32; ++i)
+      if (32 * w + i < g.nb && __ldg(io.bfull + int64_t(b) * g.nb + 32 * w + i)) f |= 1u << i;
+    bmF[w] = f;
+  }
+  __syncwarp();
+  const int n = build_steps(bmA, bmB, bmF, nw, steps, lane);
+  if (lane == 0) *n_steps_sm = n;
+  __syncwarp();
+  mbar_arrive(bar_steps);
+}
+
+// ============================================================================
+// dQ: CTA = query pair, walk = union of the two key lists
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                       Geo g, const BwdIO io) {
+  using C = BwdCfg<D>;
+  constexpr int NS = C::NS;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sm = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::OFF_OWN_A, sdO = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
+  const BwdBars bb = bwd_bars<D>(base + C::OFF_BAR);
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
+  uint32_t* bmB = bmA + kMaxWords;
+  uint32_t* bmF = bmA + 2 * kMaxWords;
+  uint16_t* steps = reinterpret_cast<uint16_t*>(sm + C::OFF_STEPS);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
+  int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
+  auto stage_a = [&](int s) { return sStg + s * 2 * C::TILE64; };  // K
+  auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // V
+
+  if (threadIdx.x == 0) {
+    bwd_init_bars<D>(bb);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nw = (g.nb + 31) >> 5;
+
+  if (warp == 9) {
+    bwd_walk(g, io, false, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bb.steps, lane);
+  } else if (warp == 8) {
     // ---- the issuer: copies and MMAs in step order
     if (lane == 0) {
       constexpr uint32_t idesc_sn = idesc_bf16_f32(128, 64, false);  // S, dP: B K-major
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);   // dQ: B N-major
       tma_prefetch_desc(&mk);
       tma_prefetch_desc(&mv);
-      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      bool ok = mbar_wait(bb.steps, 0, abort_flag);
       const int n = ok ? *n_steps_sm : 0;
       auto load = [&](int j) {
-        const int s = j & 1, t = int(steps[j] & kTileMask);
-        mbar_arrive_expect_tx(bar_full + 8 * s, 2 * C::TILE64);
+        const int s = j % NS, t = int(steps[j] & kTileMask);
+        mbar_arrive_expect_tx(bb.full + 8 * s, 2 * C::TILE64);
         for (int bx = 0; bx < C::KB; ++bx) {
-          tma_load_3d(stage_a(s) + bx * C::BOX64, &mk, bar_full + 8 * s, 64 * bx, t * 64, bh);
-          tma_load_3d(stage_b(s) + bx * C::BOX64, &mv, bar_full + 8 * s, 64 * bx, t * 64, bh);
+          tma_load_3d(stage_a(s) + bx * C::BOX64, &mk, bb.full + 8 * s, 64 * bx, t * 64, bh);
+          tma_load_3d(stage_b(s) + bx * C::BOX64, &mv, bb.full + 8 * s, 64 * bx, t * 64, bh);
         }
       };
-      for (int j = 0; j < n && j < 2; ++j) load(j);
-      ok = ok && mbar_wait(bar_own, 0, abort_flag);
+      // step j's accumulation, dQ += dS_j K_j: A = group w's dS (tensor
+      // memory), B = the K tile read N-major
+      auto accumulate = [&](int j) -> bool {
+        const int w = j & 1, s = j % NS;
+        if (!mbar_wait(bb.x_ready + 8 * w, (j >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts(tmem + C::COL_DQ_ACC, tmem + C::COL_DQ_X + 32u * w + 8u * kk,
+                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bb.x_free + 8 * w);
+        tc_commit(bb.empty + 8 * s);
+        return true;
+      };
+      int loaded = 0;  // steps whose copies have been issued
+      if (n > 0) {
+        load(0);
+        loaded = 1;
+      }
+      ok = ok && mbar_wait(bb.own, 0, abort_flag);
       int j = 0;
       for (; ok && j < n; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(bar_full + 8 * s, (j >> 1) & 1, abort_flag)) {
+        const int w = j & 1, k = j >> 1, s = j % NS;
+        // the next step's copies; its stage last held step j + 1 - NS,
+        // whose accumulation was issued one iteration ago at the latest
+        if (j + 1 < n) {
+          if (j + 1 >= NS &&
+              !mbar_wait(bb.empty + 8 * ((j + 1) % NS), ((j + 1 - NS) / NS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          load(j + 1);
+          loaded = j + 2;
+        }
+        // S_j = Q K_j^T and dP_j = dO V_j^T into group w's columns, once the
+        // group has read its previous S and dP
+        if (!mbar_wait(bb.full + 8 * s, (j / NS) & 1, abort_flag) ||
+            (k > 0 && !mbar_wait(bb.sfree + 8 * w, (k - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -236,73 +338,70 @@ __global__ void __launch_bounds__(256, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
           const uint32_t offo = (kk / 4) * C::BOX128 + (kk % 4) * 32;
-          tc_mma_ss(tmem + C::COL_S, sdesc_sw128(sQ + offo, 16, 1024),
+          tc_mma_ss(tmem + 128u * w, sdesc_sw128(sQ + offo, 16, 1024),
                     sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
-          tc_mma_ss(tmem + C::COL_DP, sdesc_sw128(sdO + offo, 16, 1024),
+          tc_mma_ss(tmem + 128u * w + 64u, sdesc_sw128(sdO + offo, 16, 1024),
                     sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
         }
-        tc_commit(bar_mma1);
-        if (!mbar_wait(bar_ready, j & 1, abort_flag)) {
+        tc_commit(bb.s_ready + 8 * w);
+        // then the previous step's accumulation (the other group's)
+        if (j > 0 && !accumulate(j - 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        // dQ += dS K: A = dS (tensor memory), B = K as [keys x D] read N-major
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_X + 8u * kk,
-                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar_empty + 8 * s);
-        if (j + 2 < n) {
-          if (!mbar_wait(bar_empty + 8 * s, (j >> 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          load(j + 2);
-        }
       }
+      if (ok && n > 0) ok = accumulate(n - 1);
       if (!ok) {
         report_timeout(abort_flag, io.status);
-        // copies that may still be in flight: the steps loaded but not used
-        for (int jj = j; jj < n && jj < j + 2; ++jj)
-          mbar_wait(bar_full + 8 * (jj & 1), (jj >> 1) & 1, nullptr, 200000000ull);
+        // copies that may still be in flight: loaded steps from j on
+        for (int jj = j; jj < loaded; ++jj)
+          mbar_wait(bb.full + 8 * (jj % NS), (jj / NS) & 1, nullptr, 200000000ull);
       }
-      tc_commit(bar_done);
-      tc_commit(bar_drain);
-      mbar_wait(bar_drain, 0, nullptr, 200000000ull);
+      tc_commit(bb.done);
+      tc_commit(bb.drain);
+      mbar_wait(bb.drain, 0, nullptr, 200000000ull);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ---- row threads: row r of the pair = TMEM lane r
-    const int row = threadIdx.x, half = row >> 6, qb = 2 * pair + half;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+  } else {
+    // ---- row groups: group grp takes steps grp, grp + 2, ..; thread r of a
+    // group owns row r of the pair = TMEM lane r
+    const int grp = warp >> 2, quad = warp & 3;
+    const int row = quad * 32 + lane, half = row >> 6, qb = 2 * pair + half;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const bool q_exists = qb < g.nb;
     const int64_t slot = int64_t(pair) * 128 + row;
     const bool row_valid =
         q_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + qb) >> (row & 63)) & 1ull);
     const int64_t prow = int64_t(bh) * g.N + slot;
-    // Q and dO rows into shared memory (A operands of S and dP)
-    store_row_swizzled(sQ, C::BOX128, row, q_exists ? io.q + prow * D : nullptr, D);
-    store_row_swizzled(sdO, C::BOX128, row, row_valid ? io.dout + prow * D : nullptr, D);
+    // Q rows (group 0) and dO rows (group 1) into shared memory: the A
+    // operands of S and dP
+    if (grp == 0)
+      store_row_swizzled(sQ, C::BOX128, row, q_exists ? io.q + prow * D : nullptr, D);
+    else
+      store_row_swizzled(sdO, C::BOX128, row, row_valid ? io.dout + prow * D : nullptr, D);
     fence_proxy_async_smem();
-    mbar_arrive(bar_own);
+    mbar_arrive(bb.own);
     const float lse2 = row_valid ? __ldg(io.lse + prow) : INFINITY;
     const float dlt = row_valid ? __ldg(io.delta + prow) : 0.f;
     const float sl2 = g.scale * 1.4426950408889634f;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const uint32_t tS = tmem + 128u * grp + lane_base, tDP = tS + 64u;
+    const uint32_t tX = tmem + C::COL_DQ_X + 32u * grp + lane_base;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bb.steps, 0, abort_flag));
     const int n = ok ? *n_steps_sm : 0;
-    for (int j = 0; ok && j < n; ++j) {
+    int k = 0;
+    for (int j = grp; ok && j < n; j += 2, ++k) {
       const uint32_t entry = steps[j];
       const int tile = int(entry & kTileMask);
       const uint32_t flags = entry >> kFlagShift;
       const bool member = row_valid && ((flags >> half) & 1u);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_mma1, j & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bb.s_ready + 8 * grp, k & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t sv[64], dp[64], pk[32];
-      BSA_TMEM_LD64(tmem + C::COL_S + lane_base, sv);
-      BSA_TMEM_LD64(tmem + C::COL_DP + lane_base, dp);
+      BSA_TMEM_LD64(tS, sv);
+      BSA_TMEM_LD64(tDP, dp);
+      tc_fence_before();
+      mbar_arrive(bb.sfree + 8 * grp);
       const uint64_t vm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
       const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
 #pragma unroll
@@ -319,21 +418,28 @@ __global__ void __launch_bounds__(256, 1)
         }
         pk[c / 2] = pack_bf16x2(d0, d1);
       }
-      BSA_TMEM_ST32(tmem + C::COL_X + lane_base, pk);
+      // dS goes where the group's previous dS was: its accumulation is done
+      if (k > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bb.x_free + 8 * grp, (k - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      BSA_TMEM_ST32(tX, pk);
       tc_fence_before();
-      mbar_arrive(bar_ready);
+      mbar_arrive(bb.x_ready + 8 * grp);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bb.done, 0, abort_flag));
     if (!ok) {
       if (lane == 0) report_timeout(abort_flag, io.status);
     } else if (q_exists) {
+      // group grp writes channels [grp * D/2, (grp + 1) * D/2)
       tc_fence_after();
       __nv_bfloat16* dst = io.dq + prow * D;
       const bool live = row_valid && n > 0;  // no steps: the accumulator was never written
 #pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = grp * (D / 64); ch < (grp + 1) * (D / 64); ++ch) {
         uint32_t a[32];
-        BSA_TMEM_LD32(tmem + C::COL_ACC + 32u * ch + lane_base, a);
+        BSA_TMEM_LD32(tmem + C::COL_DQ_ACC + 32u * ch + lane_base, a);
         uint32_t w16[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -348,7 +454,7 @@ __global__ void __launch_bounds__(256, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -358,10 +464,11 @@ __global__ void __launch_bounds__(256, 1)
 // dK, dV: CTA = key pair, walk = union of the query blocks that kept them
 // ============================================================================
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq,
                          const __grid_constant__ CUtensorMap mdo, Geo g, const BwdIO io) {
   using C = BwdCfg<D>;
+  constexpr int NS = C::NS;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -369,10 +476,7 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t sK = base + C::OFF_OWN_A, sV = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
   const uint32_t sVec = base + C::OFF_VEC;
   const float* vec = reinterpret_cast<const float*>(sm + C::OFF_VEC);
-  const uint32_t bar0 = base + C::OFF_BAR;
-  const uint32_t bar_full = bar0, bar_empty = bar0 + 16, bar_mma1 = bar0 + 32;
-  const uint32_t bar_ready = bar0 + 40, bar_own = bar0 + 48, bar_steps = bar0 + 56;
-  const uint32_t bar_done = bar0 + 64, bar_drain = bar0 + 72;
+  const BwdBars bb = bwd_bars<D>(base + C::OFF_BAR);
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
   uint32_t* bmB = bmA + kMaxWords;
   uint32_t* bmF = bmA + 2 * kMaxWords;
@@ -386,20 +490,11 @@ __global__ void __launch_bounds__(256, 1)
   auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // dO
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
-    }
-    mbar_init(bar_mma1, 1);
-    mbar_init(bar_ready, 128);
-    mbar_init(bar_own, 128);
-    mbar_init(bar_steps, 32);
-    mbar_init(bar_done, 1);
-    mbar_init(bar_drain, 1);
+    bwd_init_bars<D>(bb);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -409,49 +504,69 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem = *tmem_holder;
   const int nw = (g.nb + 31) >> 5;
 
-  if (warp == 5) {
-    // ---- the walk: query blocks that kept key block 2*pair (A) or
-    // 2*pair + 1 (B), from the transposed bitmaps; bmF marks query blocks
-    // without pad slots
-    const uint32_t* kt = io.kmask + (int64_t(bh) * g.nb) * nw;
-    for (int w = lane; w < nw; w += 32) {
-      bmA[w] = 2 * pair < g.nb ? __ldg(kt + int64_t(2 * pair) * nw + w) : 0u;
-      bmB[w] = 2 * pair + 1 < g.nb ? __ldg(kt + int64_t(2 * pair + 1) * nw + w) : 0u;
-      uint32_t f = 0u;
-      for (int i = 0; i < 32; ++i)
-        if (32 * w + i < g.nb && __ldg(io.bfull + int64_t(b) * g.nb + 32 * w + i)) f |= 1u << i;
-      bmF[w] = f;
-    }
-    __syncwarp();
-    const int n = build_steps(bmA, bmB, bmF, nw, steps, lane);
-    if (lane == 0) *n_steps_sm = n;
-    __syncwarp();
-    mbar_arrive(bar_steps);
-  } else if (warp == 4) {
+  if (warp == 9) {
+    bwd_walk(g, io, true, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bb.steps, lane);
+  } else if (warp == 8) {
     if (lane == 0) {
       constexpr uint32_t idesc_sn = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
       tma_prefetch_desc(&mq);
       tma_prefetch_desc(&mdo);
-      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      bool ok = mbar_wait(bb.steps, 0, abort_flag);
       const int n = ok ? *n_steps_sm : 0;
       auto load = [&](int j) {
-        const int s = j & 1, t = int(steps[j] & kTileMask);
+        const int s = j % NS, t = int(steps[j] & kTileMask);
         const int64_t r0 = int64_t(bh) * g.N + int64_t(t) * 64;
-        mbar_arrive_expect_tx(bar_full + 8 * s, 2 * C::TILE64 + 2 * 256);
+        mbar_arrive_expect_tx(bb.full + 8 * s, 2 * C::TILE64 + 2 * 256);
         for (int bx = 0; bx < C::KB; ++bx) {
-          tma_load_3d(stage_a(s) + bx * C::BOX64, &mq, bar_full + 8 * s, 64 * bx, t * 64, bh);
-          tma_load_3d(stage_b(s) + bx * C::BOX64, &mdo, bar_full + 8 * s, 64 * bx, t * 64, bh);
+          tma_load_3d(stage_a(s) + bx * C::BOX64, &mq, bb.full + 8 * s, 64 * bx, t * 64, bh);
+          tma_load_3d(stage_b(s) + bx * C::BOX64, &mdo, bb.full + 8 * s, 64 * bx, t * 64, bh);
         }
-        bulk_load(sVec + s * 512, io.lse + r0, 256, bar_full + 8 * s);
-        bulk_load(sVec + s * 512 + 256, io.delta + r0, 256, bar_full + 8 * s);
+        bulk_load(sVec + s * 512, io.lse + r0, 256, bb.full + 8 * s);
+        bulk_load(sVec + s * 512 + 256, io.delta + r0, 256, bb.full + 8 * s);
       };
-      for (int j = 0; j < n && j < 2; ++j) load(j);
-      ok = ok && mbar_wait(bar_own, 0, abort_flag);
+      // step j's accumulation: dV += P^T dO and dK += dS^T Q, A = group w's
+      // P^T / dS^T (over its S / dP columns), B read N-major
+      auto accumulate = [&](int j) -> bool {
+        const int w = j & 1, s = j % NS;
+        if (!mbar_wait(bb.x_ready + 8 * w, (j >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          tc_mma_ts(tmem + C::COL_DV, tmem + 128u * w + 8u * kk,
+                    sdesc_sw128(stage_b(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + C::COL_DK, tmem + 128u * w + 64u + 8u * kk,
+                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bb.x_free + 8 * w);
+        tc_commit(bb.empty + 8 * s);
+        return true;
+      };
+      int loaded = 0;
+      if (n > 0) {
+        load(0);
+        loaded = 1;
+      }
+      ok = ok && mbar_wait(bb.own, 0, abort_flag);
       int j = 0;
       for (; ok && j < n; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(bar_full + 8 * s, (j >> 1) & 1, abort_flag)) {
+        const int w = j & 1, k = j >> 1, s = j % NS;
+        if (j + 1 < n) {
+          if (j + 1 >= NS &&
+              !mbar_wait(bb.empty + 8 * ((j + 1) % NS), ((j + 1 - NS) / NS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          load(j + 1);
+          loaded = j + 2;
+        }
+        // S^T_j = K Q_j^T and dP^T_j = V dO_j^T into group w's columns, once
+        // the accumulation of its previous step (which reads P^T and dS^T
+        // from those columns) has finished
+        if (!mbar_wait(bb.full + 8 * s, (j / NS) & 1, abort_flag) ||
+            (k > 0 && !mbar_wait(bb.x_free + 8 * w, (k - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -460,130 +575,121 @@ __global__ void __launch_bounds__(256, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
           const uint32_t offo = (kk / 4) * C::BOX128 + (kk % 4) * 32;
-          tc_mma_ss(tmem + C::COL_S, sdesc_sw128(sK + offo, 16, 1024),
+          tc_mma_ss(tmem + 128u * w, sdesc_sw128(sK + offo, 16, 1024),
                     sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
-          tc_mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offo, 16, 1024),
+          tc_mma_ss(tmem + 128u * w + 64u, sdesc_sw128(sV + offo, 16, 1024),
                     sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
         }
-        tc_commit(bar_mma1);
-        if (!mbar_wait(bar_ready, j & 1, abort_flag)) {
+        tc_commit(bb.s_ready + 8 * w);
+        if (j > 0 && !accumulate(j - 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q (A from tensor memory, B N-major)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_X + 8u * kk,
-                    sdesc_sw128(stage_b(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_ts(tmem + C::COL_ACC + D, tmem + C::COL_Y + 8u * kk,
-                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar_empty + 8 * s);
-        if (j + 2 < n) {
-          if (!mbar_wait(bar_empty + 8 * s, (j >> 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          load(j + 2);
-        }
       }
+      if (ok && n > 0) ok = accumulate(n - 1);
       if (!ok) {
         report_timeout(abort_flag, io.status);
-        for (int jj = j; jj < n && jj < j + 2; ++jj)
-          mbar_wait(bar_full + 8 * (jj & 1), (jj >> 1) & 1, nullptr, 200000000ull);
+        for (int jj = j; jj < loaded; ++jj)
+          mbar_wait(bb.full + 8 * (jj % NS), (jj / NS) & 1, nullptr, 200000000ull);
       }
-      tc_commit(bar_done);
-      tc_commit(bar_drain);
-      mbar_wait(bar_drain, 0, nullptr, 200000000ull);
+      tc_commit(bb.done);
+      tc_commit(bb.drain);
+      mbar_wait(bb.drain, 0, nullptr, 200000000ull);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ---- row threads: key row r of the pair = TMEM lane r
-    const int row = threadIdx.x, half = row >> 6, kb = 2 * pair + half;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+  } else {
+    // ---- row groups: key row r of the pair = TMEM lane r
+    const int grp = warp >> 2, quad = warp & 3;
+    const int row = quad * 32 + lane, half = row >> 6, kb = 2 * pair + half;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const bool k_exists = kb < g.nb;
     const int64_t prow = int64_t(bh) * g.N + int64_t(pair) * 128 + row;
     const bool key_valid =
         k_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + kb) >> (row & 63)) & 1ull);
-    store_row_swizzled(sK, C::BOX128, row, k_exists ? io.k + prow * D : nullptr, D);
-    store_row_swizzled(sV, C::BOX128, row, k_exists ? io.v + prow * D : nullptr, D);
+    if (grp == 0)
+      store_row_swizzled(sK, C::BOX128, row, k_exists ? io.k + prow * D : nullptr, D);
+    else
+      store_row_swizzled(sV, C::BOX128, row, k_exists ? io.v + prow * D : nullptr, D);
     fence_proxy_async_smem();
-    mbar_arrive(bar_own);
+    mbar_arrive(bb.own);
     const float sl2 = g.scale * 1.4426950408889634f;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const uint32_t tS = tmem + 128u * grp + lane_base, tDP = tS + 64u;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bb.steps, 0, abort_flag));
     const int n = ok ? *n_steps_sm : 0;
-    for (int j = 0; ok && j < n; ++j) {
+    int k = 0;
+    for (int j = grp; ok && j < n; j += 2, ++k) {
       const uint32_t entry = steps[j];
       const int tile = int(entry & kTileMask);
       const uint32_t flags = entry >> kFlagShift;
       const bool member = key_valid && ((flags >> half) & 1u);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_mma1, j & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bb.s_ready + 8 * grp, k & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[64], dp[64], pk[32], dk[32];
-      BSA_TMEM_LD64(tmem + C::COL_S + lane_base, sv);
-      BSA_TMEM_LD64(tmem + C::COL_DP + lane_base, dp);
+      uint32_t sv[64], dp[64];
+      BSA_TMEM_LD64(tS, sv);
+      BSA_TMEM_LD64(tDP, dp);
       // query slots of block `tile`: real tokens only (pad queries have no output)
       const uint64_t qm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
       const uint32_t lo = uint32_t(qm), hi = uint32_t(qm >> 32);
-      const float* lse = vec + (j & 1) * 128;
+      const float* lse = vec + (j % NS) * 128;
       const float* dlt = lse + 64;
+      // P^T over S and dS^T over dP, 32 query columns (16 packed) at a time:
+      // every column of S and dP is already in registers
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-        if (member) {
-          if (bit_of(lo, hi, c)) {
-            p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse[c]));
-            d0 = p0 * (__uint_as_float(dp[c]) - dlt[c]);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int c = 32 * h2; c < 32 * h2 + 32; c += 2) {
+          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+          if (member) {
+            if (bit_of(lo, hi, c)) {
+              p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse[c]));
+              d0 = p0 * (__uint_as_float(dp[c]) - dlt[c]);
+            }
+            if (bit_of(lo, hi, c + 1)) {
+              p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse[c + 1]));
+              d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt[c + 1]);
+            }
           }
-          if (bit_of(lo, hi, c + 1)) {
-            p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse[c + 1]));
-            d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt[c + 1]);
-          }
+          pk[(c - 32 * h2) / 2] = pack_bf16x2(p0, p1);
+          dk[(c - 32 * h2) / 2] = pack_bf16x2(d0, d1);
         }
-        pk[c / 2] = pack_bf16x2(p0, p1);
-        dk[c / 2] = pack_bf16x2(d0, d1);
+        BSA_TMEM_ST16(tS + 16u * h2, pk);
+        BSA_TMEM_ST16(tDP + 16u * h2, dk);
       }
-      BSA_TMEM_ST32(tmem + C::COL_X + lane_base, pk);
-      BSA_TMEM_ST32(tmem + C::COL_Y + lane_base, dk);
       tc_fence_before();
-      mbar_arrive(bar_ready);
+      mbar_arrive(bb.x_ready + 8 * grp);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bb.done, 0, abort_flag));
     if (!ok) {
       if (lane == 0) report_timeout(abort_flag, io.status);
     } else if (k_exists) {
+      // group 0 writes dV, group 1 dK (scaled)
       tc_fence_after();
+      __nv_bfloat16* dst = (grp ? io.dk : io.dv) + prow * D;
+      const float f = grp ? g.scale : 1.f;
+      // a key block no query kept has no steps and zero gradients (its
+      // accumulators were never written)
+      const bool live = key_valid && n > 0;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
-        __nv_bfloat16* dst = (which ? io.dk : io.dv) + prow * D;
-        const float f = which ? g.scale : 1.f;
-        // a key block no query kept has no steps and zero gradients (its
-        // accumulators were never written)
-        const bool live = key_valid && n > 0;
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t a[32];
-          BSA_TMEM_LD32(tmem + C::COL_ACC + uint32_t(which * D) + 32u * ch + lane_base, a);
-          uint32_t w16[16];
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t a[32];
+        BSA_TMEM_LD32(tmem + (grp ? C::COL_DK : C::COL_DV) + 32u * ch + lane_base, a);
+        uint32_t w16[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w16[i] = pack_bf16x2(live ? __uint_as_float(a[2 * i]) * f : 0.f,
-                                 live ? __uint_as_float(a[2 * i + 1]) * f : 0.f);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+        for (int i = 0; i < 16; ++i)
+          w16[i] = pack_bf16x2(live ? __uint_as_float(a[2 * i]) * f : 0.f,
+                               live ? __uint_as_float(a[2 * i + 1]) * f : 0.f);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            d4[i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
-        }
+        for (int i = 0; i < 4; ++i)
+          d4[i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
