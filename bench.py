@@ -44,12 +44,12 @@ from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per sparse-attention launch from one ncu capture
-# of a B=1 x 4-head launch of the 720p grid (1.555 GB read + 0.126 GB
+# of a B=1 x 4-head launch of the 720p grid (1.885 GB read + 0.125 GB
 # written), scaled by the number of (batch, head) problems.  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
 # workload on the permuted path; null otherwise.
-ATTN_TRAFFIC = {"sha256": "c20bdf7196b5db994bfb8b1aecc059712513c15137fecd1905ad5ee04af3cbf0",
-                "bytes_per_bh": 1.680738e9 / 4, "workload": ("720p", 0.25, 0)}
+ATTN_TRAFFIC = {"sha256": "a0b2d535ead32d6354527b56ba4cabf27e85b251a2ecf363ec761465a7261823",
+                "bytes_per_bh": (1.884679e9 + 0.125296e9) / 4, "workload": ("720p", 0.25, 0)}
 
 
 def attn_traffic(cfg, keep_ratio):
