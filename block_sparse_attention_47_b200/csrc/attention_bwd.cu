@@ -639,20 +639,28 @@ __global__ void __launch_bounds__(320, 1)
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int c = 32 * h2; c < 32 * h2 + 32; c += 2) {
-          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-          if (member) {
-            if (bit_of(lo, hi, c)) {
-              p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse[c]));
-              d0 = p0 * (__uint_as_float(dp[c]) - dlt[c]);
+        for (int c4 = 8 * h2; c4 < 8 * h2 + 8; ++c4) {
+          // four columns' lse2 and D in one 16-byte load each
+          const float4 l4 = reinterpret_cast<const float4*>(lse)[c4];
+          const float4 t4 = reinterpret_cast<const float4*>(dlt)[c4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+          for (int u = 0; u < 4; u += 2) {
+            const int c = 4 * c4 + u;
+            float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+            if (member) {
+              if (bit_of(lo, hi, c)) {
+                p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
+                d0 = p0 * (__uint_as_float(dp[c]) - dv[u]);
+              }
+              if (bit_of(lo, hi, c + 1)) {
+                p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lv[u + 1]));
+                d1 = p1 * (__uint_as_float(dp[c + 1]) - dv[u + 1]);
+              }
             }
-            if (bit_of(lo, hi, c + 1)) {
-              p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse[c + 1]));
-              d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt[c + 1]);
-            }
+            pk[(c - 32 * h2) / 2] = pack_bf16x2(p0, p1);
+            dk[(c - 32 * h2) / 2] = pack_bf16x2(d0, d1);
           }
-          pk[(c - 32 * h2) / 2] = pack_bf16x2(p0, p1);
-          dk[(c - 32 * h2) / 2] = pack_bf16x2(d0, d1);
         }
         BSA_TMEM_ST16(tS + 16u * h2, pk);
         BSA_TMEM_ST16(tDP + 16u * h2, dk);

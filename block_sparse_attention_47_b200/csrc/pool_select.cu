@@ -268,27 +268,34 @@ __global__ void __launch_bounds__(kSelThreads * RG) select_kernel(
   }
   __syncthreads();
   if (gate) {
-    // ROWS rows x d outputs, at most 4 per thread (d <= 128)
+    // q~ = G q for every row: thread t takes channel c = t % d of rows t / d,
+    // t / d + NT / d, .. (NT is a multiple of d), so each thread reads row c
+    // of G once for all its outputs; each output is one fmaf chain in e order
     const float* G = gate + int64_t(bh % g.h) * g.d * g.d;
-    float gq[(ROWS * 128) / NT];
-    int n_out = 0;
-    for (int e = threadIdx.x; e < ROWS * g.d; e += NT, ++n_out) {
-      const int r = e / g.d, c = e % g.d;
-      const float4* gr = reinterpret_cast<const float4*>(G + int64_t(c) * g.d);
-      const float4* qr = reinterpret_cast<const float4*>(sq + r * g.d);
-      float acc = 0.f;
-      for (int e4 = 0; e4 < g.d / 4; ++e4) {
-        const float4 gv = __ldg(gr + e4), qv = qr[e4];
-        acc = fmaf(gv.x, qv.x, acc);
-        acc = fmaf(gv.y, qv.y, acc);
-        acc = fmaf(gv.z, qv.z, acc);
-        acc = fmaf(gv.w, qv.w, acc);
+    constexpr int MAXO = (ROWS * 128) / NT;  // outputs per thread at d = 128
+    const int c = threadIdx.x % g.d, r0 = threadIdx.x / g.d, rstep = NT / g.d;
+    const int nout = ROWS * g.d / NT;
+    float acc[MAXO];
+#pragma unroll
+    for (int o = 0; o < MAXO; ++o) acc[o] = 0.f;
+    const float4* gr = reinterpret_cast<const float4*>(G + int64_t(c) * g.d);
+    for (int e4 = 0; e4 < g.d / 4; ++e4) {
+      const float4 gv = __ldg(gr + e4);
+#pragma unroll
+      for (int o = 0; o < MAXO; ++o) {
+        if (o < nout) {
+          const float4 qv = reinterpret_cast<const float4*>(sq + (r0 + rstep * o) * g.d)[e4];
+          acc[o] = fmaf(gv.x, qv.x, acc[o]);
+          acc[o] = fmaf(gv.y, qv.y, acc[o]);
+          acc[o] = fmaf(gv.z, qv.z, acc[o]);
+          acc[o] = fmaf(gv.w, qv.w, acc[o]);
+        }
       }
-      gq[n_out] = acc;
     }
     __syncthreads();
-    n_out = 0;
-    for (int e = threadIdx.x; e < ROWS * g.d; e += NT, ++n_out) sq[e] = gq[n_out];
+#pragma unroll
+    for (int o = 0; o < MAXO; ++o)
+      if (o < nout) sq[(r0 + rstep * o) * g.d + c] = acc[o];
     __syncthreads();
   }
 
