@@ -20,9 +20,9 @@
 // P needs no running maximum (the forward's statistics fix it), so steps
 // are independent: two groups of row threads take alternate steps, each
 // with its own S/dP columns in tensor memory, and one thread issues the
-// copies and MMAs so that the tensor pipe always holds the next step's
-// S/dP while a group turns the previous one into P/dS:
-//     iteration j:  S/dP of step j,  then the accumulation of step j-1.
+// copies and MMAs so that both groups compute while the tensor pipe runs:
+//     dQ    iteration j:  S/dP of step j, then the accumulation of step j-2;
+//     dKdV  iteration j:  the accumulation of step j-2, then S/dP of step j.
 // Step tiles (K/V, or Q/dO with their rows' lse2 and D) go through a
 // 4-stage ring loaded one step ahead.  In dKdV, P^T and dS^T are written
 // over the group's own S and dP columns (the two accumulators fill the
@@ -344,13 +344,15 @@ __global__ void __launch_bounds__(320, 1)
                     sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
         }
         tc_commit(bb.s_ready + 8 * w);
-        // then the previous step's accumulation (the other group's)
-        if (j > 0 && !accumulate(j - 1)) {
+        // then the accumulation of this group's previous step: both groups
+        // are computing while the pipe runs
+        if (j >= 2 && !accumulate(j - 2)) {
           ok = false;
           break;
         }
       }
-      if (ok && n > 0) ok = accumulate(n - 1);
+      if (ok && n >= 2) ok = accumulate(n - 2);
+      if (ok && n >= 1) ok = accumulate(n - 1);
       if (!ok) {
         report_timeout(abort_flag, io.status);
         // copies that may still be in flight: loaded steps from j on
@@ -402,21 +404,35 @@ __global__ void __launch_bounds__(320, 1)
       BSA_TMEM_LD64(tDP, dp);
       tc_fence_before();
       mbar_arrive(bb.sfree + 8 * grp);
-      const uint64_t vm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
-      const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
+      if (member && (flags & 4u)) {
+        // every key slot is a real token: two lanes per instruction
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float d0 = 0.f, d1 = 0.f;
-        if (member) {
-          const float p0 =
-              bit_of(lo, hi, c) ? ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2)) : 0.f;
-          const float p1 = bit_of(lo, hi, c + 1)
-                               ? ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2))
-                               : 0.f;
-          d0 = p0 * (__uint_as_float(dp[c]) - dlt);
-          d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt);
+        for (int c = 0; c < 64; c += 2) {
+          float x0, x1, t0, t1, d0, d1;
+          fma_f32x2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2, -lse2,
+                    -lse2);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          add_f32x2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), -dlt, -dlt);
+          fma_f32x2(d0, d1, p0, p1, t0, t1, 0.f, 0.f);
+          pk[c / 2] = pack_bf16x2(d0, d1);
         }
-        pk[c / 2] = pack_bf16x2(d0, d1);
+      } else {
+        const uint64_t vm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
+        const uint32_t lo = uint32_t(vm), hi = uint32_t(vm >> 32);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float d0 = 0.f, d1 = 0.f;
+          if (member) {
+            const float p0 =
+                bit_of(lo, hi, c) ? ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2)) : 0.f;
+            const float p1 = bit_of(lo, hi, c + 1)
+                                 ? ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2))
+                                 : 0.f;
+            d0 = p0 * (__uint_as_float(dp[c]) - dlt);
+            d1 = p1 * (__uint_as_float(dp[c + 1]) - dlt);
+          }
+          pk[c / 2] = pack_bf16x2(d0, d1);
+        }
       }
       // dS goes where the group's previous dS was: its accumulation is done
       if (k > 0) {
@@ -562,9 +578,13 @@ __global__ void __launch_bounds__(320, 1)
           load(j + 1);
           loaded = j + 2;
         }
-        // S^T_j = K Q_j^T and dP^T_j = V dO_j^T into group w's columns, once
-        // the accumulation of its previous step (which reads P^T and dS^T
-        // from those columns) has finished
+        // the accumulation of this group's previous step, then S^T_j = K Q_j^T
+        // and dP^T_j = V dO_j^T into group w's columns once that accumulation
+        // (which reads P^T and dS^T from those columns) has finished
+        if (j >= 2 && !accumulate(j - 2)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(bb.full + 8 * s, (j / NS) & 1, abort_flag) ||
             (k > 0 && !mbar_wait(bb.x_free + 8 * w, (k - 1) & 1, abort_flag))) {
           ok = false;
@@ -581,12 +601,9 @@ __global__ void __launch_bounds__(320, 1)
                     sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
         }
         tc_commit(bb.s_ready + 8 * w);
-        if (j > 0 && !accumulate(j - 1)) {
-          ok = false;
-          break;
-        }
       }
-      if (ok && n > 0) ok = accumulate(n - 1);
+      if (ok && n >= 2) ok = accumulate(n - 2);
+      if (ok && n >= 1) ok = accumulate(n - 1);
       if (!ok) {
         report_timeout(abort_flag, io.status);
         for (int jj = j; jj < loaded; ++jj)
@@ -648,7 +665,17 @@ __global__ void __launch_bounds__(320, 1)
           for (int u = 0; u < 4; u += 2) {
             const int c = 4 * c4 + u;
             float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-            if (member) {
+            if (member && (flags & 4u)) {
+              // every query slot is a real token: two lanes per instruction
+              float x0, x1, t0, t1;
+              fma_f32x2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2,
+                        -lv[u], -lv[u + 1]);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+              add_f32x2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), -dv[u],
+                        -dv[u + 1]);
+              fma_f32x2(d0, d1, p0, p1, t0, t1, 0.f, 0.f);
+            } else if (member) {
               if (bit_of(lo, hi, c)) {
                 p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
                 d0 = p0 * (__uint_as_float(dp[c]) - dv[u]);

@@ -1,8 +1,8 @@
 """A discrete-event model of the backward kernels' barrier protocol (CPU
 only), in the style of the forward's model: the issuer (step tiles through
-a 4-stage ring loaded one step ahead; per step j the S/dP MMAs of step j,
-then the accumulation of step j-1), two row groups taking alternate steps,
-and the barriers between them.
+a 4-stage ring loaded one step ahead; per step j, in dQ the S/dP MMAs of
+step j then the accumulation of step j-2, in dKdV the other way round), two
+row groups taking alternate steps, and the barriers between them.
 
 Two variants, as in csrc/attention_bwd.cu:
   dQ    a group's S/dP columns are reused once the group has read them
@@ -146,6 +146,8 @@ def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wa
                     yield ("wait", empty[(j + 1) % stages], ((j + 1 - stages) // stages) & 1)
                 start_load(j + 1)
                 yield ("copy", full[(j + 1) % stages], 100, lambda j=j: landed(j + 1))
+            if variant == "dkdv" and j >= 2:
+                yield from accumulate(j - 2)
             yield ("wait", full[j % stages], (j // stages) & 1)
             if k > 0:
                 if variant == "dq":
@@ -154,10 +156,10 @@ def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wa
                     yield ("wait", x_free[w], (k - 1) & 1)
             burst(j)
             yield mma(700, [s_ready[w]])
-            if j > 0:
-                yield from accumulate(j - 1)
-        if n > 0:
-            yield from accumulate(n - 1)
+            if variant == "dq" and j >= 2:
+                yield from accumulate(j - 2)
+        for jj in range(max(0, n - 2), n):
+            yield from accumulate(jj)
 
     def group_warp(w, quad):
         yield ("delay", rng.randint(50, 600))
