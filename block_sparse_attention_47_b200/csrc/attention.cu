@@ -294,6 +294,15 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
 
+  // the step-table warp starts its first global loads (the two lists'
+  // lengths) before the set-up barrier, so their latency overlaps it
+  int pre_cnt[2] = {-1, -1};
+  if (MODE == kModeLists && warp == 8) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf)
+      if (2 * pair + hf < g.nb) pre_cnt[hf] = __ldg(cnt + int64_t(bh) * g.nb + 2 * pair + hf);
+  }
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < KS; ++s) {
       mbar_init(kfull(s), C::KB);
@@ -366,37 +375,54 @@ __global__ void __launch_bounds__(512, 1)
             continue;
           }
         }
-        const int c = MODE != kModeLists ? -1 : __ldg(cnt + int64_t(bh) * g.nb + qb);
-        if (c < 0) {
+        // a dense row keeps every block (lists are read below, both at once)
+        if (MODE != kModeLists || pre_cnt[hf] < 0) {
           for (int w = lane; w < nw; w += 32) {
             const int rem = g.nb - 32 * w;
             bm[w] = rem >= 32 ? ~0u : ((1u << rem) - 1u);
           }
-        } else {
-          const int n = c < g.kcap ? c : g.kcap;
-          const int32_t* src = idx + (int64_t(bh) * g.nb + qb) * g.kcap;
-          for (int base = 0; base < n; base += 8 * 32) {
-            int v[8];
+        }
+      }
+      if constexpr (MODE == kModeLists) {
+        // the two index lists, loaded together so that their latencies overlap
+        const int nA = pre_cnt[0] < 0 ? 0 : (pre_cnt[0] < g.kcap ? pre_cnt[0] : g.kcap);
+        const int nB = pre_cnt[1] < 0 ? 0 : (pre_cnt[1] < g.kcap ? pre_cnt[1] : g.kcap);
+        const int32_t* srcA = idx + (int64_t(bh) * g.nb + 2 * pair) * g.kcap;
+        const int32_t* srcB = srcA + g.kcap;
+        const int nmax = nA > nB ? nA : nB;
+        for (int base = 0; base < nmax; base += 4 * 32) {
+          int va[4], vb[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int i = base + 32 * u + lane;
-              v[u] = i < n ? __ldg(src + i) : -1;
-            }
+          for (int u = 0; u < 4; ++u) {
+            const int i = base + 32 * u + lane;
+            va[u] = i < nA ? __ldg(srcA + i) : -1;
+            vb[u] = i < nB ? __ldg(srcB + i) : -1;
+          }
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              if (v[u] >= 0 && v[u] < g.nb) atomicOr(bm + (v[u] >> 5), 1u << (v[u] & 31));
+          for (int u = 0; u < 4; ++u) {
+            if (va[u] >= 0 && va[u] < g.nb) atomicOr(bmA + (va[u] >> 5), 1u << (va[u] & 31));
+            if (vb[u] >= 0 && vb[u] < g.nb) atomicOr(bmB + (vb[u] >> 5), 1u << (vb[u] & 31));
           }
         }
       }
       // F: blocks whose 64 slots are all real tokens (no valid-slot mask needed)
       const uint8_t* full_row = bfull + int64_t(b) * g.nb;
+      const bool words = ((int64_t(b) * g.nb) & 3) == 0;  // 4-byte aligned flags
       for (int w = lane; w < nw; w += 32) {
-        uint8_t by[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) by[i] = 32 * w + i < g.nb ? __ldg(full_row + 32 * w + i) : 0;
         uint32_t f = 0u;
+        if (words && 32 * w + 32 <= g.nb) {
+          // eight 4-byte loads of the 32 flag bytes (each byte 0 or 1)
+          const uint32_t* f4 = reinterpret_cast<const uint32_t*>(full_row + 32 * w);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) f |= uint32_t(by[i] != 0) << i;
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t x = __ldg(f4 + i);
+            f |= (((x & 0xFFu) != 0u) | (((x >> 8) & 0xFFu) != 0u) << 1 |
+                  (((x >> 16) & 0xFFu) != 0u) << 2 | ((x >> 24) != 0u) << 3) << (4 * i);
+          }
+        } else {
+          for (int i = 0; i < 32; ++i)
+            if (32 * w + i < g.nb && __ldg(full_row + 32 * w + i)) f |= 1u << i;
+        }
         bmF[w] = f;
       }
       __syncwarp();
