@@ -390,16 +390,16 @@ __global__ void __launch_bounds__(512, 1)
         const int32_t* srcA = idx + (int64_t(bh) * g.nb + 2 * pair) * g.kcap;
         const int32_t* srcB = srcA + g.kcap;
         const int nmax = nA > nB ? nA : nB;
-        for (int base = 0; base < nmax; base += 4 * 32) {
-          int va[4], vb[4];
+        for (int base = 0; base < nmax; base += 8 * 32) {
+          int va[8], vb[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 8; ++u) {
             const int i = base + 32 * u + lane;
             va[u] = i < nA ? __ldg(srcA + i) : -1;
             vb[u] = i < nB ? __ldg(srcB + i) : -1;
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 8; ++u) {
             if (va[u] >= 0 && va[u] < g.nb) atomicOr(bmA + (va[u] >> 5), 1u << (va[u] & 31));
             if (vb[u] >= 0 && vb[u] < g.nb) atomicOr(bmB + (vb[u] >> 5), 1u << (vb[u] & 31));
           }

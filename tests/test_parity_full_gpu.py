@@ -29,6 +29,9 @@ FULL = [
     ("sweep", {"keep_ratio": 0.10}),
     ("sweep", {"keep_ratio": 0.03}),
     ("sweep", {"keep_ratio": 0.01}),
+    # 2,560 blocks: the selection's 8-query-block form (16 do not fit next to
+    # the scores in shared memory)
+    ("720p", {"B": 1, "heads": 2, "H": 64, "H_valid": 64}),
 ]
 
 
