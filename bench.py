@@ -44,12 +44,12 @@ from gen import SWEEP_KEEP_RATIOS, config, derived_sizes, make_qkv  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per sparse-attention launch from one ncu capture
-# of a B=1 x 4-head launch of the 720p grid (1.885 GB read + 0.125 GB
+# of a B=1 x 4-head launch of the 720p grid (2.119 GB read + 0.126 GB
 # written), scaled by the number of (batch, head) problems.  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
 # workload on the permuted path; null otherwise.
-ATTN_TRAFFIC = {"sha256": "a0b2d535ead32d6354527b56ba4cabf27e85b251a2ecf363ec761465a7261823",
-                "bytes_per_bh": (1.884679e9 + 0.125296e9) / 4, "workload": ("720p", 0.25, 0)}
+ATTN_TRAFFIC = {"sha256": "049ff65fc9c444e7de9b63a04d0dd7d36a92d669cfbfff03206733a198ad2296",
+                "bytes_per_bh": (2.118633e9 + 0.125721e9) / 4, "workload": ("720p", 0.25, 0)}
 
 
 def attn_traffic(cfg, keep_ratio):
