@@ -3,10 +3,11 @@
 // whole tiles once tokens are permuted).  Pure data movement, HBM-bound:
 // every 16-byte vector is read once and written once.
 //
-// Thread mapping: consecutive threads take consecutive 16-byte vectors of
+// permute_kernel: consecutive threads take consecutive 16-byte vectors of
 // one raster token row [heads, head_dim] (contiguous), so raster-side
-// accesses are fully coalesced and block-order accesses are whole
-// head_dim rows (128 or 256 contiguous bytes).
+// accesses are fully coalesced and block-order accesses are whole head_dim
+// rows (128 or 256 contiguous bytes).  The fused permute + pool and the
+// unpermute take one block of one head per CTA instead.
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -37,31 +38,6 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(
     }
     __nv_bfloat16* dst = xp + ((int64_t(b) * g.h + hh) * g.N + slot) * g.d + v * 8;
     *reinterpret_cast<uint4*>(dst) = val;
-  }
-}
-
-__global__ void __launch_bounds__(kThreads) unpermute_kernel(
-    Geo g, const int32_t* __restrict__ iperm, const __nv_bfloat16* __restrict__ op,
-    __nv_bfloat16* __restrict__ o, int64_t sb, int64_t sn, int64_t sh) {
-  const int vec_per_row = g.d / 8;
-  const int64_t per_token = int64_t(g.h) * vec_per_row;
-  const int64_t total = int64_t(g.B) * g.N * per_token;
-  for (int64_t i = blockIdx.x * int64_t(kThreads) + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * kThreads) {
-    const int v = int(i % vec_per_row);
-    const int64_t rest = i / vec_per_row;
-    const int hh = int(rest % g.h);
-    const int64_t bn = rest / g.h;  // b * N + raster
-    const int b = int(bn / g.N);
-    const int raster = int(bn % g.N);
-    const uint32_t is = uint32_t(iperm[bn]);
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (!(is & kPad)) {
-      const int slot = int(is);
-      val = *reinterpret_cast<const uint4*>(op + ((int64_t(b) * g.h + hh) * g.N + slot) * g.d +
-                                            v * 8);
-    }
-    *reinterpret_cast<uint4*>(o + b * sb + raster * sn + hh * sh + v * 8) = val;
   }
 }
 
@@ -142,6 +118,35 @@ __global__ void __launch_bounds__(kThreads) permute_pool_kernel(
   }
 }
 
+// Block order back to raster order, one CTA per (block, head, batch
+// element): the block's 64 rows are read as one contiguous 16 KB (d = 128)
+// run and each row is written to its token's place (a whole 256-byte
+// segment); pad slots write zeros to their pad tokens, so every raster row
+// is written once.
+template <int D>
+__global__ void __launch_bounds__(kThreads) unpermute_block_kernel(
+    Geo g, const int32_t* __restrict__ perm, const __nv_bfloat16* __restrict__ op,
+    __nv_bfloat16* __restrict__ o, int64_t sb, int64_t sn, int64_t sh) {
+  constexpr int VEC = D / 8, GROUPS = kThreads / VEC, RPT = kBlock / GROUPS;
+  const int j = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int v8 = threadIdx.x % VEC, rg = threadIdx.x / VEC;
+  const int64_t src0 = ((int64_t(b) * g.h + hh) * g.N + int64_t(j) * kBlock) * D + v8 * 8;
+  uint4 val[RPT];
+  uint32_t pr[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int slot = rg + GROUPS * i;
+    pr[i] = uint32_t(__ldg(perm + int64_t(b) * g.N + int64_t(j) * kBlock + slot));
+    val[i] = *reinterpret_cast<const uint4*>(op + src0 + int64_t(slot) * D);
+  }
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int64_t raster = int64_t(pr[i] & ~kPad);
+    *reinterpret_cast<uint4*>(o + b * sb + raster * sn + hh * sh + v8 * 8) =
+        (pr[i] & kPad) ? make_uint4(0, 0, 0, 0) : val[i];
+  }
+}
+
 int grid_for(int64_t work) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -177,8 +182,11 @@ cudaError_t launch_permute_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16
 cudaError_t launch_unpermute(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* op,
                              __nv_bfloat16* o, int64_t sb, int64_t sn, int64_t sh,
                              cudaStream_t st) {
-  const int64_t work = int64_t(g.B) * g.N * g.h * (g.d / 8);
-  unpermute_kernel<<<grid_for(work), kThreads, 0, st>>>(g, lp.iperm, op, o, sb, sn, sh);
+  const dim3 grid(g.nb, g.h, g.B);
+  if (g.d == 128)
+    unpermute_block_kernel<128><<<grid, kThreads, 0, st>>>(g, lp.perm, op, o, sb, sn, sh);
+  else
+    unpermute_block_kernel<64><<<grid, kThreads, 0, st>>>(g, lp.perm, op, o, sb, sn, sh);
   return cudaGetLastError();
 }
 
