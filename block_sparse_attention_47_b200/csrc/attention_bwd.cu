@@ -21,13 +21,12 @@
 // are independent: two groups of row threads take alternate steps, each
 // with its own S/dP columns in tensor memory, and one thread issues the
 // copies and MMAs so that both groups compute while the tensor pipe runs:
-//     dQ    iteration j:  S/dP of step j, then the accumulation of step j-2;
-//     dKdV  iteration j:  the accumulation of step j-2, then S/dP of step j.
+//     iteration j:  the accumulation of step j-2, then S/dP of step j.
 // Step tiles (K/V, or Q/dO with their rows' lse2 and D) go through a
-// 4-stage ring loaded one step ahead.  In dKdV, P^T and dS^T are written
-// over the group's own S and dP columns (the two accumulators fill the
-// rest of tensor memory), so a group's next S/dP waits for its previous
-// accumulation to finish.  Every wait is bounded (2 s) and reports
+// 4-stage ring loaded one step ahead.  P/dS are written over the group's
+// own S and dP columns (in dQ, Q and dO sit in tensor memory as the A
+// operands of S and dP; in dKdV the two accumulators fill the rest), so a
+// group's next S/dP waits for its previous accumulation to finish.  Every wait is bounded (2 s) and reports
 // BSA_ERR_TIMEOUT as the forward.
 #include "bsa_internal.cuh"
 
@@ -53,23 +52,25 @@ struct BwdCfg {
   static constexpr int OFF_STG = 2 * TILE128;              // [stage][a | b] 64-row tiles
   static constexpr int OFF_VEC = OFF_STG + NS * 2 * TILE64; // [stage][lse2 | delta][64] fp32
   static constexpr int OFF_BAR = OFF_VEC + NS * 2 * 64 * 4;
-  // full[NS] empty[NS] s_ready[2] sfree[2] x_ready[2] x_free[2] own steps done drain
+  // full[NS] empty[NS] s_ready[2] (spare[2]) x_ready[2] x_free[2] own steps done drain
   static constexpr int N_BARS = 2 * NS + 8 + 4;
   static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;      // uint32 A, B, F [kMaxWords]
   static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
   static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  // tensor memory: group w's S at 128w, dP at 128w + 64.  dQ: dS of group w
-  // at 256 + 32w, the accumulator at 384.  dKdV: P^T over S, dS^T over dP,
-  // dV at 256 and dK at 256 + D.
-  static constexpr uint32_t COL_DQ_X = 256, COL_DQ_ACC = 384, COL_DV = 256, COL_DK = 256 + D;
+  // tensor memory.  dQ: Q and dO (the A operands of S and dP, bf16 pairs) at
+  // 0 and 64, group w's S at 128 + 128w (its dS written over it), dP 64
+  // further, the accumulator at 384.  dKdV: group w's S at 128w (P^T over
+  // it), dP at 128w + 64 (dS^T over it), dV at 256 and dK at 256 + D.
+  static constexpr uint32_t COL_DQ_Q = 0, COL_DQ_DO = 64, COL_DQ_S = 128, COL_DQ_ACC = 384;
+  static constexpr uint32_t COL_DV = 256, COL_DK = 256 + D;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(COL_DK + D <= TMEM_COLS, "tensor memory budget");
 };
 
 struct BwdBars {
-  uint32_t full, empty, s_ready, sfree, x_ready, x_free, own, steps, done, drain;
+  uint32_t full, empty, s_ready, x_ready, x_free, own, steps, done, drain;
 };
 
 template <int D>
@@ -79,7 +80,6 @@ __device__ __forceinline__ BwdBars bwd_bars(uint32_t bar0) {
   b.full = bar0;
   b.empty = bar0 + 8 * C::NS;
   b.s_ready = bar0 + 16 * C::NS;
-  b.sfree = b.s_ready + 16;
   b.x_ready = b.s_ready + 32;
   b.x_free = b.s_ready + 48;
   b.own = b.s_ready + 64;
@@ -98,7 +98,6 @@ __device__ __forceinline__ void bwd_init_bars(const BwdBars& b) {
   }
   for (int w = 0; w < 2; ++w) {
     mbar_init(b.s_ready + 8 * w, 1);
-    mbar_init(b.sfree + 8 * w, 128);
     mbar_init(b.x_ready + 8 * w, 128);
     mbar_init(b.x_free + 8 * w, 1);
   }
@@ -243,7 +242,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
-  const uint32_t sQ = base + C::OFF_OWN_A, sdO = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
+  const uint32_t sStg = base + C::OFF_STG;
   const BwdBars bb = bwd_bars<D>(base + C::OFF_BAR);
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
   uint32_t* bmB = bmA + kMaxWords;
@@ -292,14 +291,14 @@ __global__ void __launch_bounds__(320, 1)
         }
       };
       // step j's accumulation, dQ += dS_j K_j: A = group w's dS (tensor
-      // memory), B = the K tile read N-major
+      // memory, over its S columns), B = the K tile read N-major
       auto accumulate = [&](int j) -> bool {
         const int w = j & 1, s = j % NS;
         if (!mbar_wait(bb.x_ready + 8 * w, (j >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_ts(tmem + C::COL_DQ_ACC, tmem + C::COL_DQ_X + 32u * w + 8u * kk,
+          tc_mma_ts(tmem + C::COL_DQ_ACC, tmem + C::COL_DQ_S + 128u * w + 8u * kk,
                     sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
                     (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bb.x_free + 8 * w);
@@ -326,10 +325,16 @@ __global__ void __launch_bounds__(320, 1)
           load(j + 1);
           loaded = j + 2;
         }
-        // S_j = Q K_j^T and dP_j = dO V_j^T into group w's columns, once the
-        // group has read its previous S and dP
+        // the accumulation of this group's previous step, then S_j = Q K_j^T
+        // and dP_j = dO V_j^T into group w's columns once that accumulation
+        // (which reads dS from them) has finished; A = Q or dO from tensor
+        // memory, B = the K or V tile
+        if (j >= 2 && !accumulate(j - 2)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(bb.full + 8 * s, (j / NS) & 1, abort_flag) ||
-            (k > 0 && !mbar_wait(bb.sfree + 8 * w, (k - 1) & 1, abort_flag))) {
+            (k > 0 && !mbar_wait(bb.x_free + 8 * w, (k - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -337,19 +342,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
-          const uint32_t offo = (kk / 4) * C::BOX128 + (kk % 4) * 32;
-          tc_mma_ss(tmem + 128u * w, sdesc_sw128(sQ + offo, 16, 1024),
+          tc_mma_ts(tmem + C::COL_DQ_S + 128u * w, tmem + C::COL_DQ_Q + 8u * kk,
                     sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
-          tc_mma_ss(tmem + 128u * w + 64u, sdesc_sw128(sdO + offo, 16, 1024),
+          tc_mma_ts(tmem + C::COL_DQ_S + 128u * w + 64u, tmem + C::COL_DQ_DO + 8u * kk,
                     sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
         }
         tc_commit(bb.s_ready + 8 * w);
-        // then the accumulation of this group's previous step: both groups
-        // are computing while the pipe runs
-        if (j >= 2 && !accumulate(j - 2)) {
-          ok = false;
-          break;
-        }
       }
       if (ok && n >= 2) ok = accumulate(n - 2);
       if (ok && n >= 1) ok = accumulate(n - 1);
@@ -375,19 +373,34 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_valid =
         q_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + qb) >> (row & 63)) & 1ull);
     const int64_t prow = int64_t(bh) * g.N + slot;
-    // Q rows (group 0) and dO rows (group 1) into shared memory: the A
-    // operands of S and dP
-    if (grp == 0)
-      store_row_swizzled(sQ, C::BOX128, row, q_exists ? io.q + prow * D : nullptr, D);
-    else
-      store_row_swizzled(sdO, C::BOX128, row, row_valid ? io.dout + prow * D : nullptr, D);
-    fence_proxy_async_smem();
+    // Q rows (group 0) and dO rows (group 1) into tensor memory, bf16 pairs
+    // per column: the A operands of S and dP
+    {
+      const __nv_bfloat16* src = grp == 0 ? (q_exists ? io.q + prow * D : nullptr)
+                                          : (row_valid ? io.dout + prow * D : nullptr);
+      uint32_t rw[D / 2];
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        const uint4 u = src ? __ldg(reinterpret_cast<const uint4*>(src) + i)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        rw[4 * i] = u.x;
+        rw[4 * i + 1] = u.y;
+        rw[4 * i + 2] = u.z;
+        rw[4 * i + 3] = u.w;
+      }
+      const uint32_t dst = tmem + (grp == 0 ? C::COL_DQ_Q : C::COL_DQ_DO) + lane_base;
+      if constexpr (D == 128) {
+        BSA_TMEM_ST64(dst, rw);
+      } else {
+        BSA_TMEM_ST32(dst, rw);
+      }
+      tc_fence_before();
+    }
     mbar_arrive(bb.own);
     const float lse2 = row_valid ? __ldg(io.lse + prow) : INFINITY;
     const float dlt = row_valid ? __ldg(io.delta + prow) : 0.f;
     const float sl2 = g.scale * 1.4426950408889634f;
-    const uint32_t tS = tmem + 128u * grp + lane_base, tDP = tS + 64u;
-    const uint32_t tX = tmem + C::COL_DQ_X + 32u * grp + lane_base;
+    const uint32_t tS = tmem + C::COL_DQ_S + 128u * grp + lane_base, tDP = tS + 64u;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bb.steps, 0, abort_flag));
     const int n = ok ? *n_steps_sm : 0;
     int k = 0;
@@ -402,8 +415,6 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t sv[64], dp[64], pk[32];
       BSA_TMEM_LD64(tS, sv);
       BSA_TMEM_LD64(tDP, dp);
-      tc_fence_before();
-      mbar_arrive(bb.sfree + 8 * grp);
       if (member && (flags & 4u)) {
         // every key slot is a real token: two lanes per instruction
 #pragma unroll
@@ -434,13 +445,9 @@ __global__ void __launch_bounds__(320, 1)
           pk[c / 2] = pack_bf16x2(d0, d1);
         }
       }
-      // dS goes where the group's previous dS was: its accumulation is done
-      if (k > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bb.x_free + 8 * grp, (k - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-      tc_fence_after();
-      BSA_TMEM_ST32(tX, pk);
+      // dS over this step's S (already read; the previous accumulation, which
+      // read the previous dS there, finished before this step's S/dP)
+      BSA_TMEM_ST32(tS, pk);
       tc_fence_before();
       mbar_arrive(bb.x_ready + 8 * grp);
     }

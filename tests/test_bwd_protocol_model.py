@@ -1,23 +1,17 @@
 """A discrete-event model of the backward kernels' barrier protocol (CPU
 only), in the style of the forward's model: the issuer (step tiles through
-a 4-stage ring loaded one step ahead; per step j, in dQ the S/dP MMAs of
-step j then the accumulation of step j-2, in dKdV the other way round), two
-row groups taking alternate steps, and the barriers between them.
-
-Two variants, as in csrc/attention_bwd.cu:
-  dQ    a group's S/dP columns are reused once the group has read them
-        (sfree); its dS columns once the previous accumulation finished
-        (x_free, waited by the group).
-  dKdV  P^T and dS^T are written over the group's own S/dP columns, so the
-        issuer waits for the group's previous accumulation (x_free) before
-        its next S/dP.
+a 4-stage ring loaded one step ahead; per step j the accumulation of step
+j-2, then the S/dP MMAs of step j), two row groups taking alternate steps,
+and the barriers between them.  As in both kernels of csrc/attention_bwd.cu,
+a group writes its P/dS over its own S/dP columns, so the issuer waits for
+the group's previous accumulation (x_free) before its next S/dP.
 
 Hazard checks: a stage is never reloaded before the accumulation of the step
 it holds has finished, an MMA only reads a stage holding its own step, a
 burst never overwrites S/dP (or the P/dS stored over them) that is still to
 be read, a group's dS is never overwritten before its accumulation read it,
-and every role finishes.  The planted mistakes (dKdV without the x_free
-wait, and a stage reloaded without waiting for its accumulation) must be
+and every role finishes.  The planted mistakes (no x_free wait before an
+S/dP, and a stage reloaded without waiting for its accumulation) must be
 caught.
 """
 import random
@@ -44,7 +38,7 @@ class Then:
         self.bar.arrive(sim, weight, tx)
 
 
-def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wait=False,
+def simulate(n, seed, member_rate, skip_xfree_wait=False, skip_empty_wait=False,
              acc_cycles=300):
     stages = NS
     sim = Sim(seed)
@@ -52,17 +46,16 @@ def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wa
     full = [Barrier("full%d" % s, 1) for s in range(stages)]
     empty = [Barrier("empty%d" % s, 1) for s in range(stages)]
     s_ready = [Barrier("s_ready%d" % w, 1) for w in range(2)]
-    sfree = [Barrier("sfree%d" % w, 128) for w in range(2)]
     x_ready = [Barrier("x_ready%d" % w, 128) for w in range(2)]
     x_free = [Barrier("x_free%d" % w, 1) for w in range(2)]
     own = Barrier("own", 256)
     # stage contents: step held, landed, accumulation finished
     stage = {}
     # tensor memory per group: the step whose S/dP the columns hold, how many
-    # of the group's four warps have read it; dS (dQ) or P/dS (dKdV) written
-    cols = [{"step": None, "read": 4, "x": None, "x_used": True} for _ in range(2)]
-    # dQ: the dS columns of each group, per warp (each warp writes its rows)
-    dq_x = [[{"step": None, "used": True} for _ in range(4)] for _ in range(2)]
+    # of the group's four warps have read it, the step whose P/dS each warp
+    # has written over its own lanes, and whether the accumulation that reads
+    # them has finished
+    cols = [{"step": None, "read": 4, "x": [None] * 4, "x_used": True} for _ in range(2)]
 
     def start_load(j):
         s = j % stages
@@ -88,33 +81,25 @@ def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wa
         if c["step"] is not None and c["read"] < 4:
             raise Hazard("S/dP of step %d overwrites group %d's unread step %d"
                          % (j, w, c["step"]))
-        if variant == "dkdv" and not c["x_used"]:
-            raise Hazard("S/dP of step %d overwrites group %d's P/dS of step %d before "
-                         "its accumulation" % (j, w, c["x"]))
+        if not c["x_used"]:
+            raise Hazard("S/dP of step %d overwrites group %d's P/dS of steps %s before "
+                         "their accumulation" % (j, w, c["x"]))
         use_stage(j)
         c.update(step=j, read=0)
 
     def accumulate_mma(j):
         w = j & 1
         use_stage(j)
-        if variant == "dkdv":
-            c = cols[w]
-            if c["x"] != j:
-                raise Hazard("accumulation of step %d reads P/dS of step %s" % (j, c["x"]))
-        elif any(x["step"] != j for x in dq_x[w]):
-            raise Hazard("accumulation of step %d reads dS of steps %s"
-                         % (j, [x["step"] for x in dq_x[w]]))
+        c = cols[w]
+        if any(x != j for x in c["x"]):
+            raise Hazard("accumulation of step %d reads P/dS of steps %s" % (j, c["x"]))
+        c["x_used"] = False
 
     def stage_done(j):
         stage[j % stages][2] = True
 
     def x_done(j):
-        w = j & 1
-        if variant == "dkdv":
-            cols[w]["x_used"] = True
-        else:
-            for x in dq_x[w]:
-                x["used"] = True
+        cols[j & 1]["x_used"] = True
 
     def mma(cycles, commits):
         """Queue MMAs on the in-order pipe; their commits arrive when the pipe
@@ -146,18 +131,13 @@ def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wa
                     yield ("wait", empty[(j + 1) % stages], ((j + 1 - stages) // stages) & 1)
                 start_load(j + 1)
                 yield ("copy", full[(j + 1) % stages], 100, lambda j=j: landed(j + 1))
-            if variant == "dkdv" and j >= 2:
+            if j >= 2:
                 yield from accumulate(j - 2)
             yield ("wait", full[j % stages], (j // stages) & 1)
-            if k > 0:
-                if variant == "dq":
-                    yield ("wait", sfree[w], (k - 1) & 1)
-                elif not skip_xfree_wait:
-                    yield ("wait", x_free[w], (k - 1) & 1)
+            if k > 0 and not skip_xfree_wait:
+                yield ("wait", x_free[w], (k - 1) & 1)
             burst(j)
             yield mma(700, [s_ready[w]])
-            if variant == "dq" and j >= 2:
-                yield from accumulate(j - 2)
         for jj in range(max(0, n - 2), n):
             yield from accumulate(jj)
 
@@ -173,19 +153,10 @@ def simulate(n, seed, member_rate, variant, skip_xfree_wait=False, skip_empty_wa
                 raise Hazard("group %d read S/dP of step %s for step %d" % (w, c["step"], j))
             yield ("delay", rng.randint(50, 150))
             c["read"] += 1
-            if variant == "dq":
-                yield ("arrive", sfree[w], 32)
             busy = rng.random() < member_rate
             yield ("delay", rng.randint(lo, hi) if busy else rng.randint(20, 200))
-            if variant == "dq":
-                if k > 0:
-                    yield ("wait", x_free[w], (k - 1) & 1)
-                x = dq_x[w][quad]
-                if not x["used"]:
-                    raise Hazard("group %d warp %d overwrites dS of step %s" % (w, quad, x["step"]))
-                x.update(step=j, used=False)
-            else:
-                c.update(x=j, x_used=False)
+            # P/dS over the warp's own lanes of the S/dP columns just read
+            c["x"][quad] = j
             yield ("delay", rng.randint(30, 100))
             yield ("arrive", x_ready[w], 32)
 
@@ -207,21 +178,20 @@ def schedules(count):
                rng.choice([300, 1500, 4000]))
 
 
-@pytest.mark.parametrize("variant", ["dq", "dkdv"])
-def test_backward_protocol_has_no_hazard(variant):
-    for n, seed, rate, acc in schedules(300):
+def test_backward_protocol_has_no_hazard():
+    for n, seed, rate, acc in schedules(600):
         try:
-            result = simulate(n, seed, rate, variant, acc_cycles=acc)
+            result = simulate(n, seed, rate, acc_cycles=acc)
         except Hazard as e:
-            pytest.fail("%s n=%d seed=%d: %s" % (variant, n, seed, e))
-        assert result == "ok", "%s n=%d seed=%d: %s" % (variant, n, seed, result)
+            pytest.fail("n=%d seed=%d: %s" % (n, seed, e))
+        assert result == "ok", "n=%d seed=%d: %s" % (n, seed, result)
 
 
-def test_dkdv_without_accumulation_wait_is_caught():
+def test_burst_without_accumulation_wait_is_caught():
     caught = 0
     for n, seed, rate, acc in schedules(300):
         try:
-            caught += simulate(n, seed, rate, "dkdv", skip_xfree_wait=True, acc_cycles=acc) != "ok"
+            caught += simulate(n, seed, rate, skip_xfree_wait=True, acc_cycles=acc) != "ok"
         except Hazard:
             caught += 1
     assert caught > 0, "the model no longer sees P/dS overwritten before its accumulation"
@@ -231,7 +201,7 @@ def test_reload_without_empty_wait_is_caught():
     caught = 0
     for n, seed, rate, acc in schedules(300):
         try:
-            caught += simulate(n, seed, rate, "dq", skip_empty_wait=True, acc_cycles=acc) != "ok"
+            caught += simulate(n, seed, rate, skip_empty_wait=True, acc_cycles=acc) != "ok"
         except Hazard:
             caught += 1
     assert caught > 0, "the model no longer sees a stage reloaded under its accumulation"
