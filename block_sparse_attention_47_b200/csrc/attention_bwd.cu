@@ -8,26 +8,32 @@
 //     dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
 //
 // Two kernels, both tcgen05 with the accumulators in tensor memory and the
-// tiles in 128-byte-swizzled shared memory:
+// tiles in 128-byte-swizzled shared memory.  P needs no running maximum
+// (the forward's statistics fix it), so steps are independent; they are
+// taken in pairs, and each product of a pair is one N=128 MMA burst over
+// both steps' tiles (a 128-row B operand: two 64-row tiles stacked), since
+// an N=64 MMA takes as long to issue as an N=128 one.  Row group g (128
+// threads, thread r = TMEM lane r) computes step 2p+g from its 64-column
+// half of the burst.
 //   dQ   CTA = two adjacent query blocks (128 rows, as the forward), walking
-//        the union of their key lists; per step S and dP (two SS MMAs,
-//        M=128 N=64), dS from them in registers, then dQ += dS K (A = dS in
-//        tensor memory, B = the same K tile read N-major).
+//        the union of their key lists.  Per pair: S = Q [K_2p; K_2p+1]^T
+//        (A = Q in shared memory) and dP = dO [V_2p; V_2p+1]^T (A = dO in
+//        tensor memory), then dQ += dS_g K_(2p+g) for each group (A = dS in
+//        its own tensor-memory columns, B = the K tile read N-major).  The
+//        next pair's S/dP are issued as soon as both groups have read this
+//        pair's, so the tensor pipe runs them while the groups compute; a
+//        copy warp keeps a K ring (3 pairs, freed by the accumulations) and
+//        a V ring (2 pairs, freed by dP) filled.
 //   dKdV CTA = two adjacent key blocks (128 key rows), walking the union of
 //        the query blocks that kept them (transposed lists, built as
-//        bitmaps); per step S^T = K Q^T and dP^T = V dO^T (M=128 N=64), P^T
-//        and dS^T in registers, then dV += P^T dO and dK += dS^T Q.
-// P needs no running maximum (the forward's statistics fix it), so steps
-// are independent: two groups of row threads take alternate steps, each
-// with its own S/dP columns in tensor memory, and one thread issues the
-// copies and MMAs so that both groups compute while the tensor pipe runs:
-//     iteration j:  the accumulation of step j-2, then S/dP of step j.
-// Step tiles (K/V, or Q/dO with their rows' lse2 and D) go through a
-// 4-stage ring loaded one step ahead.  P/dS are written over the group's
-// own S and dP columns (in dQ, Q and dO sit in tensor memory as the A
-// operands of S and dP; in dKdV the two accumulators fill the rest), so a
-// group's next S/dP waits for its previous accumulation to finish.  Every wait is bounded (2 s) and reports
-// BSA_ERR_TIMEOUT as the forward.
+//        bitmaps).  Per pair: S^T = K [Q_2p; Q_2p+1]^T and dP^T = V [dO_2p;
+//        dO_2p+1]^T (A = K, V in shared memory), then each group writes P^T
+//        over its S^T columns (dV += P^T dO starts on it) and dS^T over its
+//        dP^T columns (dK += dS^T Q).  The two accumulators take half of
+//        tensor memory, so the next pair's S^T waits for dV and its dP^T for
+//        dK; the issuer loads the Q/dO ring (2 pairs, with the query rows'
+//        lse2 and D) one pair ahead.
+// Every wait is bounded (2 s) and reports BSA_ERR_TIMEOUT as the forward.
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -35,77 +41,6 @@ namespace {
 
 constexpr int kMaxWords = kAttnMaxBlocks / 32;
 constexpr uint32_t kTileMask = 0x1FFFu, kFlagShift = 13;
-
-template <int D>
-struct BwdCfg {
-  // warps 0-3 / 4-7: row groups 0 / 1 (alternate steps); 8: issuer; 9: steps
-  static constexpr int kThreads = 320;
-  static constexpr int KB = D / 64;                // 64-column boxes
-  static constexpr int NS = 4;                     // step-tile ring stages
-  static constexpr int TILE64 = 64 * D * 2;        // one 64-row tile
-  static constexpr int TILE128 = 128 * D * 2;      // the CTA's own 128-row tile
-  static constexpr int BOX64 = 64 * 128, BOX128 = 128 * 128;
-  // dQ: own = Q | dO (128 rows each); stages = K | V (64 rows)
-  // dKdV: own = K | V; stages = Q | dO, plus lse2 | delta (64 floats)
-  static constexpr int OFF_OWN_A = 0;
-  static constexpr int OFF_OWN_B = TILE128;
-  static constexpr int OFF_STG = 2 * TILE128;              // [stage][a | b] 64-row tiles
-  static constexpr int OFF_VEC = OFF_STG + NS * 2 * TILE64; // [stage][lse2 | delta][64] fp32
-  static constexpr int OFF_BAR = OFF_VEC + NS * 2 * 64 * 4;
-  // full[NS] empty[NS] s_ready[2] (spare[2]) x_ready[2] x_free[2] own steps done drain
-  static constexpr int N_BARS = 2 * NS + 8 + 4;
-  static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;      // uint32 A, B, F [kMaxWords]
-  static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
-  static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static constexpr uint32_t TMEM_COLS = 512;
-  // tensor memory.  dQ: Q and dO (the A operands of S and dP, bf16 pairs) at
-  // 0 and 64, group w's S at 128 + 128w (its dS written over it), dP 64
-  // further, the accumulator at 384.  dKdV: group w's S at 128w (P^T over
-  // it), dP at 128w + 64 (dS^T over it), dV at 256 and dK at 256 + D.
-  static constexpr uint32_t COL_DQ_Q = 0, COL_DQ_DO = 64, COL_DQ_S = 128, COL_DQ_ACC = 384;
-  static constexpr uint32_t COL_DV = 256, COL_DK = 256 + D;
-  static_assert(SMEM <= 227 * 1024, "shared memory budget");
-  static_assert(COL_DK + D <= TMEM_COLS, "tensor memory budget");
-};
-
-struct BwdBars {
-  uint32_t full, empty, s_ready, x_ready, x_free, own, steps, done, drain;
-};
-
-template <int D>
-__device__ __forceinline__ BwdBars bwd_bars(uint32_t bar0) {
-  using C = BwdCfg<D>;
-  BwdBars b;
-  b.full = bar0;
-  b.empty = bar0 + 8 * C::NS;
-  b.s_ready = bar0 + 16 * C::NS;
-  b.x_ready = b.s_ready + 32;
-  b.x_free = b.s_ready + 48;
-  b.own = b.s_ready + 64;
-  b.steps = b.own + 8;
-  b.done = b.own + 16;
-  b.drain = b.own + 24;
-  return b;
-}
-
-template <int D>
-__device__ __forceinline__ void bwd_init_bars(const BwdBars& b) {
-  using C = BwdCfg<D>;
-  for (int s = 0; s < C::NS; ++s) {
-    mbar_init(b.full + 8 * s, 1);
-    mbar_init(b.empty + 8 * s, 1);
-  }
-  for (int w = 0; w < 2; ++w) {
-    mbar_init(b.s_ready + 8 * w, 1);
-    mbar_init(b.x_ready + 8 * w, 128);
-    mbar_init(b.x_free + 8 * w, 1);
-  }
-  mbar_init(b.own, 256);
-  mbar_init(b.steps, 32);
-  mbar_init(b.done, 1);
-  mbar_init(b.drain, 1);
-}
 
 #define BSA_TMEM_ST16(taddr, r)                                                               \
   asm volatile(                                                                               \
@@ -233,17 +168,50 @@ __device__ __forceinline__ void bwd_walk(const Geo& g, const BwdIO& io, bool tra
 // dQ: CTA = query pair, walk = union of the two key lists
 // ============================================================================
 template <int D>
+struct DqCfg {
+  // warps 0-3 / 4-7: row groups 0 / 1; 8: MMA issuer; 9: steps, then copies
+  static constexpr int kThreads = 320;
+  static constexpr int KB = D / 64;                // 64-column boxes
+  static constexpr int NK = 3, NV = 2;             // K / V ring slots (pairs)
+  static constexpr int TILE64 = 64 * D * 2;        // one step's 64-row tile
+  static constexpr int PAIR = 2 * TILE64;          // [box][128 rows][128 B]
+  static constexpr int BOX64 = 64 * 128, BOX128 = 128 * 128;
+  static constexpr int OFF_Q = 0;                  // the CTA's Q rows (A of S)
+  static constexpr int OFF_K = PAIR;
+  static constexpr int OFF_V = OFF_K + NK * PAIR;
+  static constexpr int OFF_BAR = OFF_V + NV * PAIR;
+  // kfull[NK] kempty[NK] vfull[NV] vempty[NV] sd_ready read x_ready[2]
+  // x_free own steps done drain
+  static constexpr int N_BARS = 2 * NK + 2 * NV + 10;
+  static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;  // uint32 A, B, F [kMaxWords]
+  static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
+  static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // tensor memory: dO rows (bf16 pairs, the A operand of dP) at 0, S at 64
+  // (group g's half at 64 + 64g), dP at 192, dS at 320 (32 bf16-pair
+  // columns per group), the dQ accumulator at 384
+  static constexpr uint32_t COL_DO = 0, COL_S = 64, COL_DP = 192, COL_DS = 320, COL_ACC = 384;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(COL_ACC + D <= TMEM_COLS, "tensor memory budget");
+};
+
+template <int D>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                        Geo g, const BwdIO io) {
-  using C = BwdCfg<D>;
-  constexpr int NS = C::NS;
+  using C = DqCfg<D>;
+  constexpr int NK = C::NK, NV = C::NV;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
-  const uint32_t sStg = base + C::OFF_STG;
-  const BwdBars bb = bwd_bars<D>(base + C::OFF_BAR);
+  const uint32_t sQ = base + C::OFF_Q;
+  const uint32_t kfull = base + C::OFF_BAR, kempty = kfull + 8 * NK;
+  const uint32_t vfull = kempty + 8 * NK, vempty = vfull + 8 * NV;
+  const uint32_t sd_ready = vempty + 8 * NV, read = sd_ready + 8, x_ready = read + 8;
+  const uint32_t x_free = x_ready + 16, own = x_free + 8, bar_steps = own + 8;
+  const uint32_t done = bar_steps + 8, drain = done + 8;
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
   uint32_t* bmB = bmA + kMaxWords;
   uint32_t* bmF = bmA + 2 * kMaxWords;
@@ -253,11 +221,27 @@ __global__ void __launch_bounds__(320, 1)
   int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
-  auto stage_a = [&](int s) { return sStg + s * 2 * C::TILE64; };  // K
-  auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // V
+  auto kslot = [&](int p) { return base + C::OFF_K + (p % NK) * C::PAIR; };
+  auto vslot = [&](int p) { return base + C::OFF_V + (p % NV) * C::PAIR; };
 
   if (threadIdx.x == 0) {
-    bwd_init_bars<D>(bb);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(kfull + 8 * s, 1);
+      mbar_init(kempty + 8 * s, 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(vfull + 8 * s, 1);
+      mbar_init(vempty + 8 * s, 1);
+    }
+    mbar_init(sd_ready, 1);
+    mbar_init(read, 8);
+    mbar_init(x_ready, 4);
+    mbar_init(x_ready + 8, 4);
+    mbar_init(x_free, 1);
+    mbar_init(own, 8);
+    mbar_init(bar_steps, 32);
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -272,99 +256,107 @@ __global__ void __launch_bounds__(320, 1)
   const int nw = (g.nb + 31) >> 5;
 
   if (warp == 9) {
-    bwd_walk(g, io, false, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bb.steps, lane);
-  } else if (warp == 8) {
-    // ---- the issuer: copies and MMAs in step order
+    bwd_walk(g, io, false, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bar_steps, lane);
+    // ---- then the copies: K and V tiles of each pair into their rings
     if (lane == 0) {
-      constexpr uint32_t idesc_sn = idesc_bf16_f32(128, 64, false);  // S, dP: B K-major
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);   // dQ: B N-major
       tma_prefetch_desc(&mk);
       tma_prefetch_desc(&mv);
-      bool ok = mbar_wait(bb.steps, 0, abort_flag);
-      const int n = ok ? *n_steps_sm : 0;
-      auto load = [&](int j) {
-        const int s = j % NS, t = int(steps[j] & kTileMask);
-        mbar_arrive_expect_tx(bb.full + 8 * s, 2 * C::TILE64);
-        for (int bx = 0; bx < C::KB; ++bx) {
-          tma_load_3d(stage_a(s) + bx * C::BOX64, &mk, bb.full + 8 * s, 64 * bx, t * 64, bh);
-          tma_load_3d(stage_b(s) + bx * C::BOX64, &mv, bb.full + 8 * s, 64 * bx, t * 64, bh);
-        }
-      };
-      // step j's accumulation, dQ += dS_j K_j: A = group w's dS (tensor
-      // memory, over its S columns), B = the K tile read N-major
-      auto accumulate = [&](int j) -> bool {
-        const int w = j & 1, s = j % NS;
-        if (!mbar_wait(bb.x_ready + 8 * w, (j >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_ts(tmem + C::COL_DQ_ACC, tmem + C::COL_DQ_S + 128u * w + 8u * kk,
-                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bb.x_free + 8 * w);
-        tc_commit(bb.empty + 8 * s);
-        return true;
-      };
-      int loaded = 0;  // steps whose copies have been issued
-      if (n > 0) {
-        load(0);
-        loaded = 1;
-      }
-      ok = ok && mbar_wait(bb.own, 0, abort_flag);
-      int j = 0;
-      for (; ok && j < n; ++j) {
-        const int w = j & 1, k = j >> 1, s = j % NS;
-        // the next step's copies; its stage last held step j + 1 - NS,
-        // whose accumulation was issued one iteration ago at the latest
-        if (j + 1 < n) {
-          if (j + 1 >= NS &&
-              !mbar_wait(bb.empty + 8 * ((j + 1) % NS), ((j + 1 - NS) / NS) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          load(j + 1);
-          loaded = j + 2;
-        }
-        // the accumulation of this group's previous step, then S_j = Q K_j^T
-        // and dP_j = dO V_j^T into group w's columns once that accumulation
-        // (which reads dS from them) has finished; A = Q or dO from tensor
-        // memory, B = the K or V tile
-        if (j >= 2 && !accumulate(j - 2)) {
+      const int n = *n_steps_sm, np = (n + 1) >> 1;
+      bool ok = true;
+      int kl = 0, vl = 0;  // pairs whose K / V copies have been issued
+      for (int p = 0; p < np; ++p) {
+        const int ns = 2 * p + 1 < n ? 2 : 1;
+        if (p >= NK && !mbar_wait(kempty + 8 * (p % NK), ((p - NK) / NK) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(bb.full + 8 * s, (j / NS) & 1, abort_flag) ||
-            (k > 0 && !mbar_wait(bb.x_free + 8 * w, (k - 1) & 1, abort_flag))) {
+        mbar_arrive_expect_tx(kfull + 8 * (p % NK), ns * C::TILE64);
+        for (int h = 0; h < ns; ++h) {
+          const int t = int(steps[2 * p + h] & kTileMask);
+          for (int bx = 0; bx < C::KB; ++bx)
+            tma_load_3d(kslot(p) + bx * C::BOX128 + h * C::BOX64, &mk, kfull + 8 * (p % NK),
+                        64 * bx, t * 64, bh);
+        }
+        kl = p + 1;
+        if (p >= NV && !mbar_wait(vempty + 8 * (p % NV), ((p - NV) / NV) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(vfull + 8 * (p % NV), ns * C::TILE64);
+        for (int h = 0; h < ns; ++h) {
+          const int t = int(steps[2 * p + h] & kTileMask);
+          for (int bx = 0; bx < C::KB; ++bx)
+            tma_load_3d(vslot(p) + bx * C::BOX128 + h * C::BOX64, &mv, vfull + 8 * (p % NV),
+                        64 * bx, t * 64, bh);
+        }
+        vl = p + 1;
+      }
+      if (!ok) report_timeout(abort_flag, io.status);
+      if (!ok || *abort_flag) {
+        // the newest copy into each slot may still be landing
+        for (int p = kl > NK ? kl - NK : 0; p < kl; ++p)
+          mbar_wait(kfull + 8 * (p % NK), (p / NK) & 1, nullptr, 200000000ull);
+        for (int p = vl > NV ? vl - NV : 0; p < vl; ++p)
+          mbar_wait(vfull + 8 * (p % NV), (p / NV) & 1, nullptr, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ---- the issuer: per pair p, S/dP of p, then the accumulation of p-1
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);  // S, dP: B K-major
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);   // dQ: B N-major
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+      ok = ok && mbar_wait(own, 0, abort_flag);
+      // dQ += dS_g K_(2q+g): A = group g's dS, B = the K tile read N-major
+      auto accumulate = [&](int q) -> bool {
+        const int ns = 2 * q + 1 < n ? 2 : 1;
+        for (int h = 0; h < ns; ++h) {
+          if (!mbar_wait(x_ready + 8 * h, q & 1, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_DS + 32u * h + 8u * kk,
+                      sdesc_sw128(kslot(q) + h * C::BOX64 + kk * 2048, C::BOX128, 1024),
+                      idesc_acc, (q > 0 || h > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(x_free);
+        tc_commit(kempty + 8 * (q % NK));
+        return true;
+      };
+      for (int p = 0; ok && p < np; ++p) {
+        // S and dP of pair p once its tiles are in and both groups have
+        // read pair p-1's (they are overwritten)
+        if (!mbar_wait(kfull + 8 * (p % NK), (p / NK) & 1, abort_flag) ||
+            !mbar_wait(vfull + 8 * (p % NV), (p / NV) & 1, abort_flag) ||
+            (p > 0 && !mbar_wait(read, (p - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
-          tc_mma_ts(tmem + C::COL_DQ_S + 128u * w, tmem + C::COL_DQ_Q + 8u * kk,
-                    sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
-          tc_mma_ts(tmem + C::COL_DQ_S + 128u * w + 64u, tmem + C::COL_DQ_DO + 8u * kk,
-                    sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
+          const uint32_t off = (kk / 4) * C::BOX128 + (kk % 4) * 32;
+          tc_mma_ss(tmem + C::COL_S, sdesc_sw128(sQ + off, 16, 1024),
+                    sdesc_sw128(kslot(p) + off, 16, 1024), idesc_s, kk > 0);
+          tc_mma_ts(tmem + C::COL_DP, tmem + C::COL_DO + 8u * kk,
+                    sdesc_sw128(vslot(p) + off, 16, 1024), idesc_s, kk > 0);
         }
-        tc_commit(bb.s_ready + 8 * w);
+        tc_commit(sd_ready);
+        tc_commit(vempty + 8 * (p % NV));
+        if (p > 0 && !accumulate(p - 1)) ok = false;
       }
-      if (ok && n >= 2) ok = accumulate(n - 2);
-      if (ok && n >= 1) ok = accumulate(n - 1);
-      if (!ok) {
-        report_timeout(abort_flag, io.status);
-        // copies that may still be in flight: loaded steps from j on
-        for (int jj = j; jj < loaded; ++jj)
-          mbar_wait(bb.full + 8 * (jj % NS), (jj / NS) & 1, nullptr, 200000000ull);
-      }
-      tc_commit(bb.done);
-      tc_commit(bb.drain);
-      mbar_wait(bb.drain, 0, nullptr, 200000000ull);
+      if (ok && np > 0) ok = accumulate(np - 1);
+      if (!ok) report_timeout(abort_flag, io.status);
+      tc_commit(done);
+      tc_commit(drain);
+      mbar_wait(drain, 0, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
-    // ---- row groups: group grp takes steps grp, grp + 2, ..; thread r of a
-    // group owns row r of the pair = TMEM lane r
+    // ---- row groups: group grp takes step 2p + grp of every pair; thread r
+    // of a group owns row r of the query pair = TMEM lane r
     const int grp = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane, half = row >> 6, qb = 2 * pair + half;
     const uint32_t lane_base = uint32_t(quad * 32) << 16;
@@ -373,11 +365,13 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_valid =
         q_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + qb) >> (row & 63)) & 1ull);
     const int64_t prow = int64_t(bh) * g.N + slot;
-    // Q rows (group 0) and dO rows (group 1) into tensor memory, bf16 pairs
-    // per column: the A operands of S and dP
-    {
-      const __nv_bfloat16* src = grp == 0 ? (q_exists ? io.q + prow * D : nullptr)
-                                          : (row_valid ? io.dout + prow * D : nullptr);
+    if (grp == 0) {
+      // Q rows into shared memory: the A operand of S
+      store_row_swizzled(sQ, C::BOX128, row, q_exists ? io.q + prow * D : nullptr, D);
+      fence_proxy_async_smem();
+    } else {
+      // dO rows into tensor memory, bf16 pairs per column: the A operand of dP
+      const __nv_bfloat16* src = row_valid ? io.dout + prow * D : nullptr;
       uint32_t rw[D / 2];
 #pragma unroll
       for (int i = 0; i < D / 8; ++i) {
@@ -388,33 +382,46 @@ __global__ void __launch_bounds__(320, 1)
         rw[4 * i + 2] = u.z;
         rw[4 * i + 3] = u.w;
       }
-      const uint32_t dst = tmem + (grp == 0 ? C::COL_DQ_Q : C::COL_DQ_DO) + lane_base;
       if constexpr (D == 128) {
-        BSA_TMEM_ST64(dst, rw);
+        BSA_TMEM_ST64(tmem + C::COL_DO + lane_base, rw);
       } else {
-        BSA_TMEM_ST32(dst, rw);
+        BSA_TMEM_ST32(tmem + C::COL_DO + lane_base, rw);
       }
       tc_fence_before();
     }
-    mbar_arrive(bb.own);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(own);
     const float lse2 = row_valid ? __ldg(io.lse + prow) : INFINITY;
     const float dlt = row_valid ? __ldg(io.delta + prow) : 0.f;
     const float sl2 = g.scale * 1.4426950408889634f;
-    const uint32_t tS = tmem + C::COL_DQ_S + 128u * grp + lane_base, tDP = tS + 64u;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bb.steps, 0, abort_flag));
-    const int n = ok ? *n_steps_sm : 0;
-    int k = 0;
-    for (int j = grp; ok && j < n; j += 2, ++k) {
+    const uint32_t tS = tmem + C::COL_S + 64u * grp + lane_base;
+    const uint32_t tDP = tmem + C::COL_DP + 64u * grp + lane_base;
+    const uint32_t tDS = tmem + C::COL_DS + 32u * grp + lane_base;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+    for (int p = 0; ok && p < np; ++p) {
+      const int j = 2 * p + grp;
+      const bool mine = j < n;  // the last pair may hold one step
+      ok = __all_sync(0xffffffffu, mbar_wait(sd_ready, p & 1, abort_flag));
+      if (!ok) break;
+      if (!mine) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(read);
+        continue;
+      }
+      tc_fence_after();
+      uint32_t sv[64], dp[64];
+      BSA_TMEM_LD64(tS, sv);
+      BSA_TMEM_LD64(tDP, dp);
+      // S and dP read: the issuer may start the next pair's
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(read);
       const uint32_t entry = steps[j];
       const int tile = int(entry & kTileMask);
       const uint32_t flags = entry >> kFlagShift;
       const bool member = row_valid && ((flags >> half) & 1u);
-      ok = __all_sync(0xffffffffu, mbar_wait(bb.s_ready + 8 * grp, k & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sv[64], dp[64], pk[32];
-      BSA_TMEM_LD64(tS, sv);
-      BSA_TMEM_LD64(tDP, dp);
+      uint32_t pk[32];
       if (member && (flags & 4u)) {
         // every key slot is a real token: two lanes per instruction
 #pragma unroll
@@ -445,13 +452,19 @@ __global__ void __launch_bounds__(320, 1)
           pk[c / 2] = pack_bf16x2(d0, d1);
         }
       }
-      // dS over this step's S (already read; the previous accumulation, which
-      // read the previous dS there, finished before this step's S/dP)
-      BSA_TMEM_ST32(tS, pk);
+      // dS into the group's columns once the previous pair's accumulation,
+      // which reads them, has finished
+      if (p > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(x_free, (p - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      BSA_TMEM_ST32(tDS, pk);
       tc_fence_before();
-      mbar_arrive(bb.x_ready + 8 * grp);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_ready + 8 * grp);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bb.done, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag));
     if (!ok) {
       if (lane == 0) report_timeout(abort_flag, io.status);
     } else if (q_exists) {
@@ -462,7 +475,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll 1
       for (int ch = grp * (D / 64); ch < (grp + 1) * (D / 64); ++ch) {
         uint32_t a[32];
-        BSA_TMEM_LD32(tmem + C::COL_DQ_ACC + 32u * ch + lane_base, a);
+        BSA_TMEM_LD32(tmem + C::COL_ACC + 32u * ch + lane_base, a);
         uint32_t w16[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -487,19 +500,47 @@ __global__ void __launch_bounds__(320, 1)
 // dK, dV: CTA = key pair, walk = union of the query blocks that kept them
 // ============================================================================
 template <int D>
+struct DkdvCfg {
+  // warps 0-3 / 4-7: row groups 0 / 1; 8: issuer (MMAs and copies); 9: steps
+  static constexpr int kThreads = 320;
+  static constexpr int KB = D / 64;
+  static constexpr int NR = 2;                     // Q/dO ring slots (pairs)
+  static constexpr int TILE64 = 64 * D * 2;
+  static constexpr int PAIR = 2 * TILE64;          // [box][128 rows][128 B]
+  static constexpr int BOX64 = 64 * 128, BOX128 = 128 * 128;
+  static constexpr int OFF_K = 0, OFF_V = PAIR;    // the CTA's K and V rows
+  static constexpr int OFF_STG = 2 * PAIR;         // [slot][Q pair | dO pair]
+  static constexpr int OFF_VEC = OFF_STG + NR * 2 * PAIR;  // [slot][lse2 128 | D 128] fp32
+  static constexpr int OFF_BAR = OFF_VEC + NR * 1024;
+  // full[NR] sd_ready p_ready[2] ds_ready[2] xv_free xk_free own steps done drain
+  static constexpr int N_BARS = NR + 11;
+  static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;
+  static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
+  static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // tensor memory: S^T at 0 (group g's half at 64g, P^T written over it),
+  // dP^T at 128 (dS^T over it), dV at 256, dK at 256 + D
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(COL_DK + D <= TMEM_COLS, "tensor memory budget");
+};
+
+template <int D>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq,
                          const __grid_constant__ CUtensorMap mdo, Geo g, const BwdIO io) {
-  using C = BwdCfg<D>;
-  constexpr int NS = C::NS;
+  using C = DkdvCfg<D>;
+  constexpr int NR = C::NR;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
-  const uint32_t sK = base + C::OFF_OWN_A, sV = base + C::OFF_OWN_B, sStg = base + C::OFF_STG;
-  const uint32_t sVec = base + C::OFF_VEC;
-  const float* vec = reinterpret_cast<const float*>(sm + C::OFF_VEC);
-  const BwdBars bb = bwd_bars<D>(base + C::OFF_BAR);
+  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+  const uint32_t full = base + C::OFF_BAR, sd_ready = full + 8 * NR;
+  const uint32_t p_ready = sd_ready + 8, ds_ready = p_ready + 16;
+  const uint32_t xv_free = ds_ready + 16, xk_free = xv_free + 8, own = xk_free + 8;
+  const uint32_t bar_steps = own + 8, done = bar_steps + 8, drain = done + 8;
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
   uint32_t* bmB = bmA + kMaxWords;
   uint32_t* bmF = bmA + 2 * kMaxWords;
@@ -509,11 +550,23 @@ __global__ void __launch_bounds__(320, 1)
   int* n_steps_sm = reinterpret_cast<int*>(sm + C::OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
-  auto stage_a = [&](int s) { return sStg + s * 2 * C::TILE64; };  // Q
-  auto stage_b = [&](int s) { return stage_a(s) + C::TILE64; };    // dO
+  auto qslot = [&](int p) { return base + C::OFF_STG + (p % NR) * 2 * C::PAIR; };
+  auto doslot = [&](int p) { return qslot(p) + C::PAIR; };
+  auto vecslot = [&](int p) { return base + C::OFF_VEC + (p % NR) * 1024; };
 
   if (threadIdx.x == 0) {
-    bwd_init_bars<D>(bb);
+    for (int s = 0; s < NR; ++s) mbar_init(full + 8 * s, 1);
+    mbar_init(sd_ready, 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(p_ready + 8 * w, 4);
+      mbar_init(ds_ready + 8 * w, 4);
+    }
+    mbar_init(xv_free, 1);
+    mbar_init(xk_free, 1);
+    mbar_init(own, 8);
+    mbar_init(bar_steps, 32);
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -528,97 +581,109 @@ __global__ void __launch_bounds__(320, 1)
   const int nw = (g.nb + 31) >> 5;
 
   if (warp == 9) {
-    bwd_walk(g, io, true, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bb.steps, lane);
+    bwd_walk(g, io, true, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bar_steps, lane);
   } else if (warp == 8) {
     if (lane == 0) {
-      constexpr uint32_t idesc_sn = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
       tma_prefetch_desc(&mq);
       tma_prefetch_desc(&mdo);
-      bool ok = mbar_wait(bb.steps, 0, abort_flag);
-      const int n = ok ? *n_steps_sm : 0;
-      auto load = [&](int j) {
-        const int s = j % NS, t = int(steps[j] & kTileMask);
-        const int64_t r0 = int64_t(bh) * g.N + int64_t(t) * 64;
-        mbar_arrive_expect_tx(bb.full + 8 * s, 2 * C::TILE64 + 2 * 256);
-        for (int bx = 0; bx < C::KB; ++bx) {
-          tma_load_3d(stage_a(s) + bx * C::BOX64, &mq, bb.full + 8 * s, 64 * bx, t * 64, bh);
-          tma_load_3d(stage_b(s) + bx * C::BOX64, &mdo, bb.full + 8 * s, 64 * bx, t * 64, bh);
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+      // Q and dO tiles of pair p with their rows' lse2 and D
+      auto load = [&](int p) {
+        const int ns = 2 * p + 1 < n ? 2 : 1;
+        const uint32_t bar = full + 8 * (p % NR);
+        mbar_arrive_expect_tx(bar, ns * (2 * C::TILE64 + 512));
+        for (int h = 0; h < ns; ++h) {
+          const int t = int(steps[2 * p + h] & kTileMask);
+          const int64_t r0 = int64_t(bh) * g.N + int64_t(t) * 64;
+          for (int bx = 0; bx < C::KB; ++bx) {
+            tma_load_3d(qslot(p) + bx * C::BOX128 + h * C::BOX64, &mq, bar, 64 * bx, t * 64, bh);
+            tma_load_3d(doslot(p) + bx * C::BOX128 + h * C::BOX64, &mdo, bar, 64 * bx, t * 64,
+                        bh);
+          }
+          bulk_load(vecslot(p) + h * 256, io.lse + r0, 256, bar);
+          bulk_load(vecslot(p) + 512 + h * 256, io.delta + r0, 256, bar);
         }
-        bulk_load(sVec + s * 512, io.lse + r0, 256, bb.full + 8 * s);
-        bulk_load(sVec + s * 512 + 256, io.delta + r0, 256, bb.full + 8 * s);
-      };
-      // step j's accumulation: dV += P^T dO and dK += dS^T Q, A = group w's
-      // P^T / dS^T (over its S / dP columns), B read N-major
-      auto accumulate = [&](int j) -> bool {
-        const int w = j & 1, s = j % NS;
-        if (!mbar_wait(bb.x_ready + 8 * w, (j >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          tc_mma_ts(tmem + C::COL_DV, tmem + 128u * w + 8u * kk,
-                    sdesc_sw128(stage_b(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_ts(tmem + C::COL_DK, tmem + 128u * w + 64u + 8u * kk,
-                    sdesc_sw128(stage_a(s) + kk * 2048, C::BOX64, 1024), idesc_acc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bb.x_free + 8 * w);
-        tc_commit(bb.empty + 8 * s);
-        return true;
       };
       int loaded = 0;
-      if (n > 0) {
-        load(0);
-        loaded = 1;
-      }
-      ok = ok && mbar_wait(bb.own, 0, abort_flag);
-      int j = 0;
-      for (; ok && j < n; ++j) {
-        const int w = j & 1, k = j >> 1, s = j % NS;
-        if (j + 1 < n) {
-          if (j + 1 >= NS &&
-              !mbar_wait(bb.empty + 8 * ((j + 1) % NS), ((j + 1 - NS) / NS) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          load(j + 1);
-          loaded = j + 2;
-        }
-        // the accumulation of this group's previous step, then S^T_j = K Q_j^T
-        // and dP^T_j = V dO_j^T into group w's columns once that accumulation
-        // (which reads P^T and dS^T from those columns) has finished
-        if (j >= 2 && !accumulate(j - 2)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(bb.full + 8 * s, (j / NS) & 1, abort_flag) ||
-            (k > 0 && !mbar_wait(bb.x_free + 8 * w, (k - 1) & 1, abort_flag))) {
+      for (; loaded < np && loaded < NR; ++loaded) load(loaded);
+      ok = ok && mbar_wait(own, 0, abort_flag);
+      int p = 0;
+      for (; ok && p < np; ++p) {
+        const int ns = 2 * p + 1 < n ? 2 : 1;
+        // S^T of pair p once dV has read P^T of pair p-1 from its columns
+        if (!mbar_wait(full + 8 * (p % NR), (p / NR) & 1, abort_flag) ||
+            (p > 0 && !mbar_wait(xv_free, (p - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::BOX64 + (kk % 4) * 32;
-          const uint32_t offo = (kk / 4) * C::BOX128 + (kk % 4) * 32;
-          tc_mma_ss(tmem + 128u * w, sdesc_sw128(sK + offo, 16, 1024),
-                    sdesc_sw128(stage_a(s) + off, 16, 1024), idesc_sn, kk > 0);
-          tc_mma_ss(tmem + 128u * w + 64u, sdesc_sw128(sV + offo, 16, 1024),
-                    sdesc_sw128(stage_b(s) + off, 16, 1024), idesc_sn, kk > 0);
+          const uint32_t off = (kk / 4) * C::BOX128 + (kk % 4) * 32;
+          tc_mma_ss(tmem + C::COL_ST, sdesc_sw128(sK + off, 16, 1024),
+                    sdesc_sw128(qslot(p) + off, 16, 1024), idesc_s, kk > 0);
         }
-        tc_commit(bb.s_ready + 8 * w);
+        // dP^T once dK has read dS^T of pair p-1
+        if (p > 0 && !mbar_wait(xk_free, (p - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::BOX128 + (kk % 4) * 32;
+          tc_mma_ss(tmem + C::COL_DPT, sdesc_sw128(sV + off, 16, 1024),
+                    sdesc_sw128(doslot(p) + off, 16, 1024), idesc_s, kk > 0);
+        }
+        tc_commit(sd_ready);
+        // pair p+1 into the slot of pair p-1, whose accumulations finished
+        if (p >= 1 && p + 1 < np) {
+          load(p + 1);
+          loaded = p + 2;
+        }
+        // dV += P^T_g dO_(2p+g) as each group's P^T is in
+        for (int h = 0; h < ns && ok; ++h) {
+          if (!mbar_wait(p_ready + 8 * h, p & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ts(tmem + C::COL_DV, tmem + C::COL_ST + 64u * h + 8u * kk,
+                      sdesc_sw128(doslot(p) + h * C::BOX64 + kk * 2048, C::BOX128, 1024),
+                      idesc_acc, (p > 0 || h > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!ok) break;
+        tc_commit(xv_free);
+        // dK += dS^T_g Q_(2p+g)
+        for (int h = 0; h < ns && ok; ++h) {
+          if (!mbar_wait(ds_ready + 8 * h, p & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ts(tmem + C::COL_DK, tmem + C::COL_DPT + 64u * h + 8u * kk,
+                      sdesc_sw128(qslot(p) + h * C::BOX64 + kk * 2048, C::BOX128, 1024),
+                      idesc_acc, (p > 0 || h > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!ok) break;
+        tc_commit(xk_free);
       }
-      if (ok && n >= 2) ok = accumulate(n - 2);
-      if (ok && n >= 1) ok = accumulate(n - 1);
       if (!ok) {
         report_timeout(abort_flag, io.status);
-        for (int jj = j; jj < loaded; ++jj)
-          mbar_wait(bb.full + 8 * (jj % NS), (jj / NS) & 1, nullptr, 200000000ull);
+        // the newest copy into each slot may still be landing
+        for (int pp = loaded > NR ? loaded - NR : 0; pp < loaded; ++pp)
+          mbar_wait(full + 8 * (pp % NR), (pp / NR) & 1, nullptr, 200000000ull);
       }
-      tc_commit(bb.done);
-      tc_commit(bb.drain);
-      mbar_wait(bb.drain, 0, nullptr, 200000000ull);
+      tc_commit(done);
+      tc_commit(drain);
+      mbar_wait(drain, 0, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
@@ -630,79 +695,100 @@ __global__ void __launch_bounds__(320, 1)
     const int64_t prow = int64_t(bh) * g.N + int64_t(pair) * 128 + row;
     const bool key_valid =
         k_exists && ((__ldg(io.bmask + int64_t(b) * g.nb + kb) >> (row & 63)) & 1ull);
+    // K rows (group 0) and V rows (group 1): the A operands of S^T and dP^T
     if (grp == 0)
       store_row_swizzled(sK, C::BOX128, row, k_exists ? io.k + prow * D : nullptr, D);
     else
       store_row_swizzled(sV, C::BOX128, row, k_exists ? io.v + prow * D : nullptr, D);
     fence_proxy_async_smem();
-    mbar_arrive(bb.own);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(own);
     const float sl2 = g.scale * 1.4426950408889634f;
-    const uint32_t tS = tmem + 128u * grp + lane_base, tDP = tS + 64u;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bb.steps, 0, abort_flag));
-    const int n = ok ? *n_steps_sm : 0;
-    int k = 0;
-    for (int j = grp; ok && j < n; j += 2, ++k) {
+    const uint32_t tS = tmem + C::COL_ST + 64u * grp + lane_base;
+    const uint32_t tDP = tmem + C::COL_DPT + 64u * grp + lane_base;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_steps, 0, abort_flag));
+    const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+    for (int p = 0; ok && p < np; ++p) {
+      const int j = 2 * p + grp;
+      ok = __all_sync(0xffffffffu, mbar_wait(sd_ready, p & 1, abort_flag));
+      if (!ok || j >= n) continue;  // the last pair may hold one step
+      tc_fence_after();
       const uint32_t entry = steps[j];
       const int tile = int(entry & kTileMask);
       const uint32_t flags = entry >> kFlagShift;
       const bool member = key_valid && ((flags >> half) & 1u);
-      ok = __all_sync(0xffffffffu, mbar_wait(bb.s_ready + 8 * grp, k & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
+      const bool dense = member && (flags & 4u);  // every query slot is a real token
+      // S^T, and the first half of dP^T (its second half is read after P^T
+      // is stored, which keeps the registers under the budget)
       uint32_t sv[64], dp[64];
       BSA_TMEM_LD64(tS, sv);
-      BSA_TMEM_LD64(tDP, dp);
+      BSA_TMEM_LD32(tDP, dp);
       // query slots of block `tile`: real tokens only (pad queries have no output)
       const uint64_t qm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
       const uint32_t lo = uint32_t(qm), hi = uint32_t(qm >> 32);
-      const float* lse = vec + (j % NS) * 128;
-      const float* dlt = lse + 64;
-      // P^T over S and dS^T over dP, 32 query columns (16 packed) at a time:
-      // every column of S and dP is already in registers
+      const float* lse = reinterpret_cast<const float*>(sm + C::OFF_VEC + (p % NR) * 1024) + 64 * grp;
+      const float* dlt = lse + 128;
+      // P^T over S^T first, so that dV starts while dS^T is computed; the
+      // probabilities stay in sv.  32 query columns (16 packed) at a time.
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t pk[16], dk[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int c4 = 8 * h2; c4 < 8 * h2 + 8; ++c4) {
-          // four columns' lse2 and D in one 16-byte load each
           const float4 l4 = reinterpret_cast<const float4*>(lse)[c4];
-          const float4 t4 = reinterpret_cast<const float4*>(dlt)[c4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {t4.x, t4.y, t4.z, t4.w};
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int u = 0; u < 4; u += 2) {
             const int c = 4 * c4 + u;
-            float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-            if (member && (flags & 4u)) {
-              // every query slot is a real token: two lanes per instruction
-              float x0, x1, t0, t1;
+            float p0 = 0.f, p1 = 0.f;
+            if (dense) {
+              float x0, x1;
               fma_f32x2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2,
                         -lv[u], -lv[u + 1]);
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
-              add_f32x2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), -dv[u],
-                        -dv[u + 1]);
-              fma_f32x2(d0, d1, p0, p1, t0, t1, 0.f, 0.f);
             } else if (member) {
-              if (bit_of(lo, hi, c)) {
-                p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
-                d0 = p0 * (__uint_as_float(dp[c]) - dv[u]);
-              }
-              if (bit_of(lo, hi, c + 1)) {
+              if (bit_of(lo, hi, c)) p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
+              if (bit_of(lo, hi, c + 1))
                 p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lv[u + 1]));
-                d1 = p1 * (__uint_as_float(dp[c + 1]) - dv[u + 1]);
-              }
             }
+            sv[c] = __float_as_uint(p0);
+            sv[c + 1] = __float_as_uint(p1);
             pk[(c - 32 * h2) / 2] = pack_bf16x2(p0, p1);
-            dk[(c - 32 * h2) / 2] = pack_bf16x2(d0, d1);
           }
         }
         BSA_TMEM_ST16(tS + 16u * h2, pk);
-        BSA_TMEM_ST16(tDP + 16u * h2, dk);
       }
       tc_fence_before();
-      mbar_arrive(bb.x_ready + 8 * grp);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready + 8 * grp);
+      // dS^T = P^T * (dP^T - D) over dP^T
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        if (h2 == 1) BSA_TMEM_LD32(tDP + 32u, (dp + 32));
+        uint32_t pk[16];
+#pragma unroll
+        for (int c4 = 8 * h2; c4 < 8 * h2 + 8; ++c4) {
+          const float4 t4 = reinterpret_cast<const float4*>(dlt)[c4];
+          const float dv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+          for (int u = 0; u < 4; u += 2) {
+            const int c = 4 * c4 + u;
+            float t0, t1, d0, d1;
+            add_f32x2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), -dv[u],
+                      -dv[u + 1]);
+            fma_f32x2(d0, d1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), t0, t1, 0.f,
+                      0.f);
+            pk[(c - 32 * h2) / 2] = pack_bf16x2(d0, d1);
+          }
+        }
+        BSA_TMEM_ST16(tDP + 16u * h2, pk);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_ready + 8 * grp);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bb.done, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag));
     if (!ok) {
       if (lane == 0) report_timeout(abort_flag, io.status);
     } else if (k_exists) {
@@ -736,7 +822,6 @@ __global__ void __launch_bounds__(320, 1)
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
-
 // ============================================================================
 // D = rowsum(dO * O) and the transposed (key block -> query blocks) bitmaps
 // ============================================================================
@@ -791,7 +876,6 @@ __global__ void __launch_bounds__(256) bwd_transpose_kernel(Geo g, const int32_t
 
 template <int D>
 cudaError_t launch_bwd_t(const Geo& g, const CUtensorMap* maps, const BwdIO& io, cudaStream_t st) {
-  using C = BwdCfg<D>;
   const int nw = (g.nb + 31) >> 5;
   cudaError_t e = cudaMemsetAsync(io.kmask, 0, sizeof(uint32_t) * size_t(g.B) * g.h * g.nb * nw, st);
   if (e != cudaSuccess) return e;
@@ -799,14 +883,15 @@ cudaError_t launch_bwd_t(const Geo& g, const CUtensorMap* maps, const BwdIO& io,
   const int64_t rows = int64_t(g.B) * g.h * g.N;
   bwd_delta_kernel<<<unsigned((rows * 8 + 255) / 256), 256, 0, st>>>(g, io.o, io.dout, io.delta);
   e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::SMEM);
+                           DqCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::SMEM);
+                           DkdvCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid((g.nb + 1) / 2, g.B * g.h);
-  attn_bwd_dq_kernel<D><<<grid, C::kThreads, C::SMEM, st>>>(maps[0], maps[1], g, io);
-  attn_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::SMEM, st>>>(maps[2], maps[3], g, io);
+  attn_bwd_dq_kernel<D><<<grid, DqCfg<D>::kThreads, DqCfg<D>::SMEM, st>>>(maps[0], maps[1], g, io);
+  attn_bwd_dkdv_kernel<D><<<grid, DkdvCfg<D>::kThreads, DkdvCfg<D>::SMEM, st>>>(maps[2], maps[3],
+                                                                               g, io);
   return cudaGetLastError();
 }
 

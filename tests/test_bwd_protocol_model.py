@@ -1,18 +1,26 @@
 """A discrete-event model of the backward kernels' barrier protocol (CPU
-only), in the style of the forward's model: the issuer (step tiles through
-a 4-stage ring loaded one step ahead; per step j the accumulation of step
-j-2, then the S/dP MMAs of step j), two row groups taking alternate steps,
-and the barriers between them.  As in both kernels of csrc/attention_bwd.cu,
-a group writes its P/dS over its own S/dP columns, so the issuer waits for
-the group's previous accumulation (x_free) before its next S/dP.
+only), in the style of the forward's model.  Both kernels of
+csrc/attention_bwd.cu take their steps in pairs: one N=128 burst per product
+covers steps 2p and 2p+1, and row group g takes step 2p+g from its half of
+the burst's columns.
 
-Hazard checks: a stage is never reloaded before the accumulation of the step
-it holds has finished, an MMA only reads a stage holding its own step, a
-burst never overwrites S/dP (or the P/dS stored over them) that is still to
-be read, a group's dS is never overwritten before its accumulation read it,
-and every role finishes.  The planted mistakes (no x_free wait before an
-S/dP, and a stage reloaded without waiting for its accumulation) must be
-caught.
+dQ:   a copy warp fills a K ring (3 pair slots, freed by the accumulation)
+      and a V ring (2 pair slots, freed by the dP burst); the issuer runs,
+      per pair p, S(p) and dP(p) once both groups have read pair p-1's S
+      and dP, then the accumulation of pair p-1 (dQ += dS K) from each
+      group's dS columns.  A group writes dS(p) into its own dS columns once
+      the accumulation of pair p-1 has finished.
+dKdV: the issuer loads a 2-slot ring itself; per pair p: S^T(p) once dV of
+      pair p-1 has finished (P^T is written over S^T), dP^T(p) once dK of
+      pair p-1 has finished (dS^T over dP^T), then dV(p) from each group's
+      P^T as it is stored and dK(p) from each group's dS^T.
+
+Hazard checks: no ring slot is reloaded before the MMAs that read it have
+finished, every MMA reads a slot holding its own pair with its tiles
+landed, no burst overwrites columns still to be read or accumulated, every
+accumulation reads what its own pair wrote, the epilogue reads the
+accumulators after every accumulation, and every role finishes.  The
+planted mistakes (one wait left out at a time) must be caught.
 """
 import random
 
@@ -20,188 +28,336 @@ import pytest
 
 from test_ring_protocol_model import Barrier, Hazard, Sim
 
-NS = 4
+NK, NV, NR = 3, 2, 2
 # tcgen05.mma is asynchronous: the issuing thread only blocks while the
-# tensor pipe holds more than this many cycles of issued work, so it runs
-# ahead of its MMAs
+# tensor pipe holds more than this many cycles of issued work
 BACKLOG = 3000
 
 
-class Then:
-    """A commit that records what the finished MMAs released, then arrives."""
+def mma(sim, cycles, commits, finished=()):
+    """Queue MMAs on the in-order pipe.  What they release is recorded when
+    the pipe finishes them; their commits arrive after that.  Returns the
+    issuer's own delay."""
+    start = max(sim.now, sim.pipe_free)
+    sim.pipe_free = start + cycles
+    for fn in finished:
+        sim.at(sim.pipe_free - sim.now, fn)
+    for bar in commits:
+        sim.at(sim.pipe_free - sim.now + sim.rng.randint(0, 50),
+               lambda bar=bar: bar.arrive(sim, 1))
+    return ("delay", max(20, sim.pipe_free - sim.now - BACKLOG))
 
-    def __init__(self, fn, bar):
-        self.fn, self.bar, self.name = fn, bar, bar.name
 
-    def arrive(self, sim, weight=1, tx=0):
-        self.fn()
-        self.bar.arrive(sim, weight, tx)
+class Slots:
+    """A ring of pair slots: the pair a slot holds, whether its tiles have
+    landed, and whether the MMAs reading it have finished."""
+
+    def __init__(self, name, count):
+        self.name, self.count, self.held = name, count, {}
+
+    def load(self, p):
+        s = p % self.count
+        h = self.held.get(s)
+        if h is not None and not h["done"]:
+            raise Hazard("%s slot %d reloaded with pair %d while pair %d is in use"
+                         % (self.name, s, p, h["pair"]))
+        self.held[s] = {"pair": p, "landed": False, "done": False}
+
+    def land(self, p):
+        h = self.held[p % self.count]
+        if h["pair"] == p:
+            h["landed"] = True
+
+    def use(self, p, what):
+        h = self.held.get(p % self.count)
+        if h is None or h["pair"] != p or not h["landed"]:
+            raise Hazard("%s of pair %d read %s slot %d holding %s"
+                         % (what, p, self.name, p % self.count, h))
+
+    def release(self, p):
+        h = self.held[p % self.count]
+        if h["pair"] == p:
+            h["done"] = True
 
 
-def simulate(n, seed, member_rate, skip_xfree_wait=False, skip_empty_wait=False,
-             acc_cycles=300):
-    stages = NS
+def compute_time(rng):
+    lo = rng.choice([10, 300, 800])
+    return lo, lo + rng.choice([100, 2000, 8000])
+
+
+def simulate_dq(n, seed, member_rate, skip=None, acc_cycles=512):
     sim = Sim(seed)
     rng = sim.rng
-    full = [Barrier("full%d" % s, 1) for s in range(stages)]
-    empty = [Barrier("empty%d" % s, 1) for s in range(stages)]
-    s_ready = [Barrier("s_ready%d" % w, 1) for w in range(2)]
-    x_ready = [Barrier("x_ready%d" % w, 128) for w in range(2)]
-    x_free = [Barrier("x_free%d" % w, 1) for w in range(2)]
-    own = Barrier("own", 256)
-    # stage contents: step held, landed, accumulation finished
-    stage = {}
-    # tensor memory per group: the step whose S/dP the columns hold, how many
-    # of the group's four warps have read it, the step whose P/dS each warp
-    # has written over its own lanes, and whether the accumulation that reads
-    # them has finished
-    cols = [{"step": None, "read": 4, "x": [None] * 4, "x_used": True} for _ in range(2)]
+    pairs = (n + 1) // 2
+    kfull = [Barrier("kfull%d" % s, 1) for s in range(NK)]
+    kempty = [Barrier("kempty%d" % s, 1) for s in range(NK)]
+    vfull = [Barrier("vfull%d" % s, 1) for s in range(NV)]
+    vempty = [Barrier("vempty%d" % s, 1) for s in range(NV)]
+    sd_ready = Barrier("sd_ready", 1)
+    read = Barrier("read", 8)
+    x_ready = [Barrier("x_ready%d" % g, 4) for g in range(2)]
+    x_free = Barrier("x_free", 1)
+    own = Barrier("own", 8)
+    done = Barrier("done", 1)
+    kring, vring = Slots("K", NK), Slots("V", NV)
+    # tensor memory: the pair whose S / dP each group's columns hold and how
+    # many of its warps read them; each warp's dS rows: the pair written and
+    # whether the accumulation reading them has finished
+    sd = [{"pair": None, "read": 4} for _ in range(2)]
+    ds = [[{"pair": None, "free": True} for _ in range(4)] for _ in range(2)]
+    acc = {"done": 0}
 
-    def start_load(j):
-        s = j % stages
-        held = stage.get(s)
-        if held is not None and not held[2]:
-            raise Hazard("stage %d reloaded with step %d while step %d is unfinished"
-                         % (s, j, held[0]))
-        stage[s] = [j, False, False]
+    def steps_in(p):
+        return 2 if 2 * p + 1 < n else 1
 
-    def landed(j):
-        s = j % stages
-        if stage[s][0] == j:
-            stage[s][1] = True
+    def loader():
+        for p in range(pairs):
+            if p >= NK and skip != "kempty":
+                yield ("wait", kempty[p % NK], ((p - NK) // NK) & 1)
+            kring.load(p)
+            yield ("copy", kfull[p % NK], 100 * steps_in(p), lambda p=p: kring.land(p))
+            if p >= NV:
+                yield ("wait", vempty[p % NV], ((p - NV) // NV) & 1)
+            vring.load(p)
+            yield ("copy", vfull[p % NV], 100 * steps_in(p), lambda p=p: vring.land(p))
 
-    def use_stage(j):
-        held = stage.get(j % stages)
-        if held is None or held[0] != j or not held[1]:
-            raise Hazard("MMA of step %d read stage %d holding %s" % (j, j % stages, held))
+    def burst(p):
+        for g in range(2):
+            if sd[g]["pair"] is not None and sd[g]["read"] < 4:
+                raise Hazard("S/dP of pair %d overwrite group %d's unread pair %d"
+                             % (p, g, sd[g]["pair"]))
+            sd[g].update(pair=p, read=0)
+        kring.use(p, "S")
+        vring.use(p, "dP")
 
-    def burst(j):
-        w = j & 1
-        c = cols[w]
-        if c["step"] is not None and c["read"] < 4:
-            raise Hazard("S/dP of step %d overwrites group %d's unread step %d"
-                         % (j, w, c["step"]))
-        if not c["x_used"]:
-            raise Hazard("S/dP of step %d overwrites group %d's P/dS of steps %s before "
-                         "their accumulation" % (j, w, c["x"]))
-        use_stage(j)
-        c.update(step=j, read=0)
+    def accumulate_mma(q, g):
+        kring.use(q, "accumulation")
+        if any(x["pair"] != q for x in ds[g]):
+            raise Hazard("accumulation of pair %d reads group %d's dS of pairs %s"
+                         % (q, g, [x["pair"] for x in ds[g]]))
+        for x in ds[g]:
+            x["free"] = False
 
-    def accumulate_mma(j):
-        w = j & 1
-        use_stage(j)
-        c = cols[w]
-        if any(x != j for x in c["x"]):
-            raise Hazard("accumulation of step %d reads P/dS of steps %s" % (j, c["x"]))
-        c["x_used"] = False
-
-    def stage_done(j):
-        stage[j % stages][2] = True
-
-    def x_done(j):
-        cols[j & 1]["x_used"] = True
-
-    def mma(cycles, commits):
-        """Queue MMAs on the in-order pipe; their commits arrive when the pipe
-        reaches them.  Returns the issuer's own delay."""
-        start = max(sim.now, sim.pipe_free)
-        sim.pipe_free = start + cycles
-        for bar in commits:
-            sim.at(sim.pipe_free - sim.now + rng.randint(0, 50),
-                   lambda bar=bar: bar.arrive(sim, 1))
-        return ("delay", max(20, sim.pipe_free - sim.now - BACKLOG))
+    def acc_done(q):
+        for g in range(2):
+            for x in ds[g]:
+                if x["pair"] == q:
+                    x["free"] = True
+        acc["done"] += steps_in(q)
 
     def issuer():
         yield ("wait", own, 0)
-        if n > 0:
-            start_load(0)
-            yield ("copy", full[0], 100, lambda: landed(0))
 
-        def accumulate(j):
-            w = j & 1
-            yield ("wait", x_ready[w], (j >> 1) & 1)
-            accumulate_mma(j)
-            yield mma(acc_cycles, [Then(lambda j=j: x_done(j), x_free[w]),
-                            Then(lambda j=j: stage_done(j), empty[j % stages])])
+        def accumulate(q):
+            for g in range(steps_in(q)):
+                yield ("wait", x_ready[g], q & 1)
+                accumulate_mma(q, g)
+            yield mma(sim, acc_cycles * steps_in(q), [x_free, kempty[q % NK]],
+                      [lambda q=q: acc_done(q), lambda q=q: kring.release(q)])
 
-        for j in range(n):
-            w, k = j & 1, j >> 1
-            if j + 1 < n:
-                if j + 1 >= stages and not skip_empty_wait:
-                    yield ("wait", empty[(j + 1) % stages], ((j + 1 - stages) // stages) & 1)
-                start_load(j + 1)
-                yield ("copy", full[(j + 1) % stages], 100, lambda j=j: landed(j + 1))
-            if j >= 2:
-                yield from accumulate(j - 2)
-            yield ("wait", full[j % stages], (j // stages) & 1)
-            if k > 0 and not skip_xfree_wait:
-                yield ("wait", x_free[w], (k - 1) & 1)
-            burst(j)
-            yield mma(700, [s_ready[w]])
-        for jj in range(max(0, n - 2), n):
-            yield from accumulate(jj)
+        for p in range(pairs):
+            yield ("wait", kfull[p % NK], (p // NK) & 1)
+            yield ("wait", vfull[p % NV], (p // NV) & 1)
+            if p > 0 and skip != "read":
+                yield ("wait", read, (p - 1) & 1)
+            burst(p)
+            yield mma(sim, 1024, [sd_ready, vempty[p % NV]], [lambda p=p: vring.release(p)])
+            if p > 0:
+                yield from accumulate(p - 1)
+        if pairs > 0:
+            yield from accumulate(pairs - 1)
+        yield mma(sim, 10, [done])
 
-    def group_warp(w, quad):
+    def group_warp(g, quad):
         yield ("delay", rng.randint(50, 600))
-        yield ("arrive", own, 32)
-        lo = rng.choice([10, 300, 800])
-        hi = lo + rng.choice([100, 2000, 8000])
-        for k, j in enumerate(range(w, n, 2)):
-            yield ("wait", s_ready[w], k & 1)
-            c = cols[w]
-            if c["step"] != j:
-                raise Hazard("group %d read S/dP of step %s for step %d" % (w, c["step"], j))
-            yield ("delay", rng.randint(50, 150))
-            c["read"] += 1
+        yield ("arrive", own, 1)
+        lo, hi = compute_time(rng)
+        for p in range(pairs):
+            yield ("wait", sd_ready, p & 1)
+            mine = 2 * p + g < n
+            if mine:
+                if sd[g]["pair"] != p:
+                    raise Hazard("group %d read S/dP of pair %s for pair %d"
+                                 % (g, sd[g]["pair"], p))
+                yield ("delay", rng.randint(50, 150))
+                sd[g]["read"] += 1
+            yield ("arrive", read, 1)
+            if not mine:
+                continue
             busy = rng.random() < member_rate
             yield ("delay", rng.randint(lo, hi) if busy else rng.randint(20, 200))
-            # P/dS over the warp's own lanes of the S/dP columns just read
-            c["x"][quad] = j
+            if p > 0 and skip != "x_free":
+                yield ("wait", x_free, (p - 1) & 1)
+            x = ds[g][quad]
+            if not x["free"]:
+                raise Hazard("group %d warp %d overwrites dS of pair %s before its accumulation"
+                             % (g, quad, x["pair"]))
+            x["pair"] = p
             yield ("delay", rng.randint(30, 100))
-            yield ("arrive", x_ready[w], 32)
+            yield ("arrive", x_ready[g], 1)
+        yield ("wait", done, 0)
+        if acc["done"] != n:
+            raise Hazard("epilogue read dQ after %d of %d accumulations" % (acc["done"], n))
 
-    roles = {"issuer": issuer()}
-    for w in range(2):
+    roles = {"loader": loader(), "issuer": issuer()}
+    for g in range(2):
         for quad in range(4):
-            roles["group%d.%d" % (w, quad)] = group_warp(w, quad)
+            roles["group%d.%d" % (g, quad)] = group_warp(g, quad)
     sim.roles = roles
     return sim.run()
 
 
-STEP_COUNTS = (1, 2, 3, 4, 5, 7, 9, 16, 33, 60)
+def simulate_dkdv(n, seed, member_rate, skip=None, acc_cycles=512):
+    sim = Sim(seed)
+    rng = sim.rng
+    pairs = (n + 1) // 2
+    full = [Barrier("full%d" % s, 1) for s in range(NR)]
+    sd_ready = Barrier("sd_ready", 1)
+    p_ready = [Barrier("p_ready%d" % g, 4) for g in range(2)]
+    ds_ready = [Barrier("ds_ready%d" % g, 4) for g in range(2)]
+    xv_free = Barrier("xv_free", 1)
+    xk_free = Barrier("xk_free", 1)
+    own = Barrier("own", 8)
+    done = Barrier("done", 1)
+    ring = Slots("Q/dO", NR)
+    # tensor memory per group and warp (each warp writes its own rows): the
+    # S^T columns hold ("S", pair) until P^T is written over them, the dP^T
+    # columns ("dP", pair) until dS^T; "used" once the accumulation reading
+    # them has finished
+    st = [[{"what": None, "pair": None, "used": True} for _ in range(4)] for _ in range(2)]
+    dpt = [[{"what": None, "pair": None, "used": True} for _ in range(4)] for _ in range(2)]
+    acc = {"dv": 0, "dk": 0, "released": {}}
+
+    def steps_in(p):
+        return 2 if 2 * p + 1 < n else 1
+
+    def load(p):
+        ring.load(p)
+        yield ("copy", full[p % NR], 100 * steps_in(p), lambda p=p: ring.land(p))
+
+    def burst(cols, what, p, reader):
+        for g in range(2):
+            for x in cols[g]:
+                if not x["used"]:
+                    raise Hazard("%s of pair %d overwrites %s of pair %s before %s read it"
+                                 % (what, p, x["what"], x["pair"], reader))
+                x.update(what=what, pair=p, used=False)
+        ring.use(p, what)
+
+    def accumulate_mma(cols, what, q, g):
+        ring.use(q, "accumulation")
+        for x in cols[g]:
+            if x["what"] != what or x["pair"] != q:
+                raise Hazard("accumulation of pair %d reads %s/%s for %s"
+                             % (q, x["what"], x["pair"], what))
+
+    def finished(cols, q, kind):
+        for g in range(2):
+            for x in cols[g]:
+                if x["pair"] == q:
+                    x["used"] = True
+        acc[kind] += steps_in(q)
+        acc["released"][q] = acc["released"].get(q, 0) + 1
+        if acc["released"][q] == 2:
+            ring.release(q)
+
+    def issuer():
+        if pairs > 0:
+            yield from load(0)
+        if pairs > 1:
+            yield from load(1)
+        yield ("wait", own, 0)
+        for p in range(pairs):
+            yield ("wait", full[p % NR], (p // NR) & 1)
+            if p > 0 and skip != "xv_free":
+                yield ("wait", xv_free, (p - 1) & 1)
+            burst(st, "S", p, "dV")
+            yield mma(sim, 512, [])
+            if p > 0 and skip != "xk_free":
+                yield ("wait", xk_free, (p - 1) & 1)
+            burst(dpt, "dP", p, "dK")
+            yield mma(sim, 512, [sd_ready])
+            if 1 <= p and p + 1 < pairs:
+                yield from load(p + 1)
+            for g in range(steps_in(p)):
+                yield ("wait", p_ready[g], p & 1)
+                accumulate_mma(st, "P", p, g)
+            yield mma(sim, acc_cycles * steps_in(p), [xv_free],
+                      [lambda p=p: finished(st, p, "dv")])
+            for g in range(steps_in(p)):
+                yield ("wait", ds_ready[g], p & 1)
+                accumulate_mma(dpt, "dS", p, g)
+            yield mma(sim, acc_cycles * steps_in(p), [xk_free],
+                      [lambda p=p: finished(dpt, p, "dk")])
+        yield mma(sim, 10, [done])
+
+    def group_warp(g, quad):
+        yield ("delay", rng.randint(50, 600))
+        yield ("arrive", own, 1)
+        lo, hi = compute_time(rng)
+        for p in range(pairs):
+            yield ("wait", sd_ready, p & 1)
+            if 2 * p + g >= n:
+                continue
+            for cols, what in ((st, "S"), (dpt, "dP")):
+                x = cols[g][quad]
+                if x["what"] != what or x["pair"] != p:
+                    raise Hazard("group %d warp %d read %s/%s for %s of pair %d"
+                                 % (g, quad, x["what"], x["pair"], what, p))
+            yield ("delay", rng.randint(50, 150))
+            busy = rng.random() < member_rate
+            yield ("delay", rng.randint(lo, hi) if busy else rng.randint(20, 200))
+            st[g][quad]["what"] = "P"
+            yield ("arrive", p_ready[g], 1)
+            yield ("delay", rng.randint(30, 400))
+            dpt[g][quad]["what"] = "dS"
+            yield ("arrive", ds_ready[g], 1)
+        yield ("wait", done, 0)
+        if acc["dv"] != n or acc["dk"] != n:
+            raise Hazard("epilogue read dK/dV after %d/%d of %d accumulations"
+                         % (acc["dv"], acc["dk"], n))
+
+    roles = {"issuer": issuer()}
+    for g in range(2):
+        for quad in range(4):
+            roles["group%d.%d" % (g, quad)] = group_warp(g, quad)
+    sim.roles = roles
+    return sim.run()
+
+
+STEP_COUNTS = (0, 1, 2, 3, 4, 5, 7, 9, 16, 33, 60)
+KERNELS = {"dq": simulate_dq, "dkdv": simulate_dkdv}
 
 
 def schedules(count):
     for trial in range(count):
         rng = random.Random(trial)
         yield (rng.choice(STEP_COUNTS), 9100 + trial, rng.choice([0.3, 0.8, 1.0]),
-               rng.choice([300, 1500, 4000]))
+               rng.choice([200, 512, 1500, 4000]))
 
 
-def test_backward_protocol_has_no_hazard():
-    for n, seed, rate, acc in schedules(600):
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+def test_backward_protocol_has_no_hazard(kernel):
+    for n, seed, rate, acc in schedules(400):
         try:
-            result = simulate(n, seed, rate, acc_cycles=acc)
+            result = KERNELS[kernel](n, seed, rate, acc_cycles=acc)
         except Hazard as e:
-            pytest.fail("n=%d seed=%d: %s" % (n, seed, e))
-        assert result == "ok", "n=%d seed=%d: %s" % (n, seed, result)
+            pytest.fail("%s n=%d seed=%d: %s" % (kernel, n, seed, e))
+        assert result == "ok", "%s n=%d seed=%d: %s" % (kernel, n, seed, result)
 
 
-def test_burst_without_accumulation_wait_is_caught():
+@pytest.mark.parametrize("kernel,skip,what", [
+    ("dq", "x_free", "dS overwritten before its accumulation"),
+    ("dq", "read", "S/dP overwritten before both groups read them"),
+    ("dq", "kempty", "a K slot reloaded under its accumulation"),
+    ("dkdv", "xv_free", "P^T overwritten before dV read it"),
+    ("dkdv", "xk_free", "dS^T overwritten before dK read it"),
+])
+def test_planted_mistake_is_caught(kernel, skip, what):
     caught = 0
     for n, seed, rate, acc in schedules(300):
         try:
-            caught += simulate(n, seed, rate, skip_xfree_wait=True, acc_cycles=acc) != "ok"
+            caught += KERNELS[kernel](n, seed, rate, skip=skip, acc_cycles=acc) != "ok"
         except Hazard:
             caught += 1
-    assert caught > 0, "the model no longer sees P/dS overwritten before its accumulation"
-
-
-def test_reload_without_empty_wait_is_caught():
-    caught = 0
-    for n, seed, rate, acc in schedules(300):
-        try:
-            caught += simulate(n, seed, rate, skip_empty_wait=True, acc_cycles=acc) != "ok"
-        except Hazard:
-            caught += 1
-    assert caught > 0, "the model no longer sees a stage reloaded under its accumulation"
+    assert caught > 0, "the model no longer sees " + what
