@@ -31,8 +31,12 @@
 //        over its S^T columns (dV += P^T dO starts on it) and dS^T over its
 //        dP^T columns (dK += dS^T Q).  The two accumulators take half of
 //        tensor memory, so the next pair's S^T waits for dV and its dP^T for
-//        dK; the issuer loads the Q/dO ring (2 pairs, with the query rows'
+//        dK; S^T and dP^T signal separately, so a group starts P^T as soon
+//        as S^T is in, and dK is queued behind the next pair's S^T.  The
+//        burst thread loads the Q/dO ring (2 pairs, with the query rows'
 //        lse2 and D) one pair ahead.
+// In both kernels one thread issues the bursts and another the
+// accumulations, so that neither waits behind the other's barriers.
 // Every wait is bounded (2 s) and reports BSA_ERR_TIMEOUT as the forward.
 #include "bsa_internal.cuh"
 
@@ -169,8 +173,9 @@ __device__ __forceinline__ void bwd_walk(const Geo& g, const BwdIO& io, bool tra
 // ============================================================================
 template <int D>
 struct DqCfg {
-  // warps 0-3 / 4-7: row groups 0 / 1; 8: MMA issuer; 9: steps, then copies
-  static constexpr int kThreads = 320;
+  // warps 0-3 / 4-7: row groups 0 / 1; 8: S/dP issuer; 9: steps, then
+  // copies; 10: accumulation issuer
+  static constexpr int kThreads = 352;
   static constexpr int KB = D / 64;                // 64-column boxes
   static constexpr int NK = 3, NV = 2;             // K / V ring slots (pairs)
   static constexpr int TILE64 = 64 * D * 2;        // one step's 64-row tile
@@ -181,8 +186,8 @@ struct DqCfg {
   static constexpr int OFF_V = OFF_K + NK * PAIR;
   static constexpr int OFF_BAR = OFF_V + NV * PAIR;
   // kfull[NK] kempty[NK] vfull[NV] vempty[NV] sd_ready read x_ready[2]
-  // x_free own steps done drain
-  static constexpr int N_BARS = 2 * NK + 2 * NV + 10;
+  // x_free own steps done drain[2]
+  static constexpr int N_BARS = 2 * NK + 2 * NV + 11;
   static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;  // uint32 A, B, F [kMaxWords]
   static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
   static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
@@ -197,7 +202,7 @@ struct DqCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                        Geo g, const BwdIO io) {
   using C = DqCfg<D>;
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t vfull = kempty + 8 * NK, vempty = vfull + 8 * NV;
   const uint32_t sd_ready = vempty + 8 * NV, read = sd_ready + 8, x_ready = read + 8;
   const uint32_t x_free = x_ready + 16, own = x_free + 8, bar_steps = own + 8;
-  const uint32_t done = bar_steps + 8, drain = done + 8;
+  const uint32_t done = bar_steps + 8, drain = done + 8;  // drain[2]: one per issuer
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
   uint32_t* bmB = bmA + kMaxWords;
   uint32_t* bmF = bmA + 2 * kMaxWords;
@@ -240,8 +245,9 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(x_free, 1);
     mbar_init(own, 8);
     mbar_init(bar_steps, 32);
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     mbar_init(drain, 1);
+    mbar_init(drain + 8, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -302,32 +308,14 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else if (warp == 8) {
-    // ---- the issuer: per pair p, S/dP of p, then the accumulation of p-1
+    // ---- S and dP of each pair, once its tiles are in and both groups have
+    // read the previous pair's (they are overwritten)
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);  // S, dP: B K-major
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);   // dQ: B N-major
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);  // B K-major
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
       const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
       ok = ok && mbar_wait(own, 0, abort_flag);
-      // dQ += dS_g K_(2q+g): A = group g's dS, B = the K tile read N-major
-      auto accumulate = [&](int q) -> bool {
-        const int ns = 2 * q + 1 < n ? 2 : 1;
-        for (int h = 0; h < ns; ++h) {
-          if (!mbar_wait(x_ready + 8 * h, q & 1, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_DS + 32u * h + 8u * kk,
-                      sdesc_sw128(kslot(q) + h * C::BOX64 + kk * 2048, C::BOX128, 1024),
-                      idesc_acc, (q > 0 || h > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(x_free);
-        tc_commit(kempty + 8 * (q % NK));
-        return true;
-      };
       for (int p = 0; ok && p < np; ++p) {
-        // S and dP of pair p once its tiles are in and both groups have
-        // read pair p-1's (they are overwritten)
         if (!mbar_wait(kfull + 8 * (p % NK), (p / NK) & 1, abort_flag) ||
             !mbar_wait(vfull + 8 * (p % NV), (p / NV) & 1, abort_flag) ||
             (p > 0 && !mbar_wait(read, (p - 1) & 1, abort_flag))) {
@@ -345,13 +333,42 @@ __global__ void __launch_bounds__(320, 1)
         }
         tc_commit(sd_ready);
         tc_commit(vempty + 8 * (p % NV));
-        if (p > 0 && !accumulate(p - 1)) ok = false;
       }
-      if (ok && np > 0) ok = accumulate(np - 1);
       if (!ok) report_timeout(abort_flag, io.status);
       tc_commit(done);
       tc_commit(drain);
       mbar_wait(drain, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 10) {
+    // ---- the accumulations: dQ += dS_g K_(2q+g) as each group's dS is in;
+    // A = the group's dS columns, B = the K tile read N-major
+    if (lane == 0) {
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+      for (int q = 0; ok && q < np; ++q) {
+        const int ns = 2 * q + 1 < n ? 2 : 1;
+        for (int h = 0; h < ns; ++h) {
+          if (!mbar_wait(x_ready + 8 * h, q & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ts(tmem + C::COL_ACC, tmem + C::COL_DS + 32u * h + 8u * kk,
+                      sdesc_sw128(kslot(q) + h * C::BOX64 + kk * 2048, C::BOX128, 1024),
+                      idesc_acc, (q > 0 || h > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!ok) break;
+        tc_commit(x_free);
+        tc_commit(kempty + 8 * (q % NK));
+      }
+      if (!ok) report_timeout(abort_flag, io.status);
+      tc_commit(done);
+      tc_commit(drain + 8);
+      mbar_wait(drain + 8, 0, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
@@ -501,8 +518,9 @@ __global__ void __launch_bounds__(320, 1)
 // ============================================================================
 template <int D>
 struct DkdvCfg {
-  // warps 0-3 / 4-7: row groups 0 / 1; 8: issuer (MMAs and copies); 9: steps
-  static constexpr int kThreads = 320;
+  // warps 0-3 / 4-7: row groups 0 / 1; 8: S^T/dP^T issuer and copies;
+  // 9: steps; 10: accumulation issuer
+  static constexpr int kThreads = 352;
   static constexpr int KB = D / 64;
   static constexpr int NR = 2;                     // Q/dO ring slots (pairs)
   static constexpr int TILE64 = 64 * D * 2;
@@ -512,8 +530,9 @@ struct DkdvCfg {
   static constexpr int OFF_STG = 2 * PAIR;         // [slot][Q pair | dO pair]
   static constexpr int OFF_VEC = OFF_STG + NR * 2 * PAIR;  // [slot][lse2 128 | D 128] fp32
   static constexpr int OFF_BAR = OFF_VEC + NR * 1024;
-  // full[NR] sd_ready p_ready[2] ds_ready[2] xv_free xk_free own steps done drain
-  static constexpr int N_BARS = NR + 11;
+  // full[NR] s_ready dp_ready st_issued p_ready[2] ds_ready[2] xv_free
+  // xk_free own steps done drain[2]
+  static constexpr int N_BARS = NR + 14;
   static constexpr int OFF_BM = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_STEPS = OFF_BM + 3 * 4 * kMaxWords;
   static constexpr int OFF_MISC = OFF_STEPS + 2 * kAttnMaxBlocks;
@@ -527,7 +546,7 @@ struct DkdvCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq,
                          const __grid_constant__ CUtensorMap mdo, Geo g, const BwdIO io) {
   using C = DkdvCfg<D>;
@@ -537,10 +556,10 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
   const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
-  const uint32_t full = base + C::OFF_BAR, sd_ready = full + 8 * NR;
-  const uint32_t p_ready = sd_ready + 8, ds_ready = p_ready + 16;
+  const uint32_t full = base + C::OFF_BAR, s_ready = full + 8 * NR, dp_ready = s_ready + 8;
+  const uint32_t st_issued = dp_ready + 8, p_ready = st_issued + 8, ds_ready = p_ready + 16;
   const uint32_t xv_free = ds_ready + 16, xk_free = xv_free + 8, own = xk_free + 8;
-  const uint32_t bar_steps = own + 8, done = bar_steps + 8, drain = done + 8;
+  const uint32_t bar_steps = own + 8, done = bar_steps + 8, drain = done + 8;  // drain[2]
   uint32_t* bmA = reinterpret_cast<uint32_t*>(sm + C::OFF_BM);
   uint32_t* bmB = bmA + kMaxWords;
   uint32_t* bmF = bmA + 2 * kMaxWords;
@@ -556,7 +575,9 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NR; ++s) mbar_init(full + 8 * s, 1);
-    mbar_init(sd_ready, 1);
+    mbar_init(s_ready, 1);
+    mbar_init(dp_ready, 1);
+    mbar_init(st_issued, 1);
     for (int w = 0; w < 2; ++w) {
       mbar_init(p_ready + 8 * w, 4);
       mbar_init(ds_ready + 8 * w, 4);
@@ -565,8 +586,9 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(xk_free, 1);
     mbar_init(own, 8);
     mbar_init(bar_steps, 32);
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     mbar_init(drain, 1);
+    mbar_init(drain + 8, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -583,9 +605,9 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 9) {
     bwd_walk(g, io, true, pair, bh, b, nw, bmA, bmB, bmF, steps, n_steps_sm, bar_steps, lane);
   } else if (warp == 8) {
+    // ---- S^T and dP^T of each pair, and the copies
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
       tma_prefetch_desc(&mq);
       tma_prefetch_desc(&mdo);
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
@@ -610,9 +632,7 @@ __global__ void __launch_bounds__(320, 1)
       int loaded = 0;
       for (; loaded < np && loaded < NR; ++loaded) load(loaded);
       ok = ok && mbar_wait(own, 0, abort_flag);
-      int p = 0;
-      for (; ok && p < np; ++p) {
-        const int ns = 2 * p + 1 < n ? 2 : 1;
+      for (int p = 0; ok && p < np; ++p) {
         // S^T of pair p once dV has read P^T of pair p-1 from its columns
         if (!mbar_wait(full + 8 * (p % NR), (p / NR) & 1, abort_flag) ||
             (p > 0 && !mbar_wait(xv_free, (p - 1) & 1, abort_flag))) {
@@ -626,6 +646,8 @@ __global__ void __launch_bounds__(320, 1)
           tc_mma_ss(tmem + C::COL_ST, sdesc_sw128(sK + off, 16, 1024),
                     sdesc_sw128(qslot(p) + off, 16, 1024), idesc_s, kk > 0);
         }
+        tc_commit(s_ready);
+        mbar_arrive(st_issued);
         // dP^T once dK has read dS^T of pair p-1
         if (p > 0 && !mbar_wait(xk_free, (p - 1) & 1, abort_flag)) {
           ok = false;
@@ -638,13 +660,34 @@ __global__ void __launch_bounds__(320, 1)
           tc_mma_ss(tmem + C::COL_DPT, sdesc_sw128(sV + off, 16, 1024),
                     sdesc_sw128(doslot(p) + off, 16, 1024), idesc_s, kk > 0);
         }
-        tc_commit(sd_ready);
+        tc_commit(dp_ready);
         // pair p+1 into the slot of pair p-1, whose accumulations finished
         if (p >= 1 && p + 1 < np) {
           load(p + 1);
           loaded = p + 2;
         }
-        // dV += P^T_g dO_(2p+g) as each group's P^T is in
+      }
+      if (!ok) {
+        report_timeout(abort_flag, io.status);
+        // the newest copy into each slot may still be landing
+        for (int pp = loaded > NR ? loaded - NR : 0; pp < loaded; ++pp)
+          mbar_wait(full + 8 * (pp % NR), (pp / NR) & 1, nullptr, 200000000ull);
+      }
+      tc_commit(done);
+      tc_commit(drain);
+      mbar_wait(drain, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 10) {
+    // ---- the accumulations: dV += P^T_g dO_(2p+g) as each group's P^T is
+    // in, then (after the next pair's S^T, so that the groups' next P^T
+    // phase is not held up) dK += dS^T_g Q_(2p+g); B read N-major
+    if (lane == 0) {
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
+      bool ok = mbar_wait(bar_steps, 0, abort_flag);
+      const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+      for (int p = 0; ok && p < np; ++p) {
+        const int ns = 2 * p + 1 < n ? 2 : 1;
         for (int h = 0; h < ns && ok; ++h) {
           if (!mbar_wait(p_ready + 8 * h, p & 1, abort_flag)) {
             ok = false;
@@ -659,7 +702,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!ok) break;
         tc_commit(xv_free);
-        // dK += dS^T_g Q_(2p+g)
+        if (p + 1 < np && !mbar_wait(st_issued, (p + 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         for (int h = 0; h < ns && ok; ++h) {
           if (!mbar_wait(ds_ready + 8 * h, p & 1, abort_flag)) {
             ok = false;
@@ -675,15 +721,10 @@ __global__ void __launch_bounds__(320, 1)
         if (!ok) break;
         tc_commit(xk_free);
       }
-      if (!ok) {
-        report_timeout(abort_flag, io.status);
-        // the newest copy into each slot may still be landing
-        for (int pp = loaded > NR ? loaded - NR : 0; pp < loaded; ++pp)
-          mbar_wait(full + 8 * (pp % NR), (pp / NR) & 1, nullptr, 200000000ull);
-      }
+      if (!ok) report_timeout(abort_flag, io.status);
       tc_commit(done);
-      tc_commit(drain);
-      mbar_wait(drain, 0, nullptr, 200000000ull);
+      tc_commit(drain + 8);
+      mbar_wait(drain + 8, 0, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
@@ -710,7 +751,7 @@ __global__ void __launch_bounds__(320, 1)
     const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
     for (int p = 0; ok && p < np; ++p) {
       const int j = 2 * p + grp;
-      ok = __all_sync(0xffffffffu, mbar_wait(sd_ready, p & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_ready, p & 1, abort_flag));
       if (!ok || j >= n) continue;  // the last pair may hold one step
       tc_fence_after();
       const uint32_t entry = steps[j];
@@ -718,11 +759,8 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t flags = entry >> kFlagShift;
       const bool member = key_valid && ((flags >> half) & 1u);
       const bool dense = member && (flags & 4u);  // every query slot is a real token
-      // S^T, and the first half of dP^T (its second half is read after P^T
-      // is stored, which keeps the registers under the budget)
       uint32_t sv[64], dp[64];
       BSA_TMEM_LD64(tS, sv);
-      BSA_TMEM_LD32(tDP, dp);
       // query slots of block `tile`: real tokens only (pad queries have no output)
       const uint64_t qm = (flags & 4u) ? ~0ull : __ldg(io.bmask + int64_t(b) * g.nb + tile);
       const uint32_t lo = uint32_t(qm), hi = uint32_t(qm >> 32);
@@ -762,10 +800,15 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_ready + 8 * grp);
-      // dS^T = P^T * (dP^T - D) over dP^T
+      // dS^T = P^T * (dP^T - D) over dP^T, once dP^T is in (its burst runs
+      // while P^T is computed); dP^T read 32 columns at a time, which keeps
+      // the registers under the budget
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_ready, p & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        if (h2 == 1) BSA_TMEM_LD32(tDP + 32u, (dp + 32));
+        BSA_TMEM_LD32(tDP + 32u * h2, (dp + 32 * h2));
         uint32_t pk[16];
 #pragma unroll
         for (int c4 = 8 * h2; c4 < 8 * h2 + 8; ++c4) {

@@ -2,18 +2,20 @@
 only), in the style of the forward's model.  Both kernels of
 csrc/attention_bwd.cu take their steps in pairs: one N=128 burst per product
 covers steps 2p and 2p+1, and row group g takes step 2p+g from its half of
-the burst's columns.
+the burst's columns.  Two threads issue MMAs into the one in-order tensor
+pipe: one the bursts, one the accumulations.
 
 dQ:   a copy warp fills a K ring (3 pair slots, freed by the accumulation)
-      and a V ring (2 pair slots, freed by the dP burst); the issuer runs,
-      per pair p, S(p) and dP(p) once both groups have read pair p-1's S
-      and dP, then the accumulation of pair p-1 (dQ += dS K) from each
-      group's dS columns.  A group writes dS(p) into its own dS columns once
-      the accumulation of pair p-1 has finished.
-dKdV: the issuer loads a 2-slot ring itself; per pair p: S^T(p) once dV of
-      pair p-1 has finished (P^T is written over S^T), dP^T(p) once dK of
-      pair p-1 has finished (dS^T over dP^T), then dV(p) from each group's
-      P^T as it is stored and dK(p) from each group's dS^T.
+      and a V ring (2 pair slots, freed by the dP burst); S(p) and dP(p)
+      are issued once both groups have read pair p-1's S and dP, the
+      accumulation of pair p (dQ += dS K) from each group's dS columns once
+      the group has written them.  A group writes dS(p) into its own dS
+      columns once the accumulation of pair p-1 has finished.
+dKdV: the burst thread also loads a 2-slot ring; S^T(p) once dV of pair
+      p-1 has finished (P^T is written over S^T), dP^T(p) once dK of pair
+      p-1 has finished (dS^T over dP^T), with separate ready signals so the
+      groups start P^T on S^T alone.  dV(p) from each group's P^T as it is
+      stored; dK(p) from each group's dS^T, queued after S^T(p+1).
 
 Hazard checks: no ring slot is reloaded before the MMAs that read it have
 finished, every MMA reads a slot holding its own pair with its tiles
@@ -98,7 +100,7 @@ def simulate_dq(n, seed, member_rate, skip=None, acc_cycles=512):
     x_ready = [Barrier("x_ready%d" % g, 4) for g in range(2)]
     x_free = Barrier("x_free", 1)
     own = Barrier("own", 8)
-    done = Barrier("done", 1)
+    done = Barrier("done", 2)
     kring, vring = Slots("K", NK), Slots("V", NV)
     # tensor memory: the pair whose S / dP each group's columns hold and how
     # many of its warps read them; each warp's dS rows: the pair written and
@@ -145,16 +147,8 @@ def simulate_dq(n, seed, member_rate, skip=None, acc_cycles=512):
                     x["free"] = True
         acc["done"] += steps_in(q)
 
-    def issuer():
+    def burst_issuer():
         yield ("wait", own, 0)
-
-        def accumulate(q):
-            for g in range(steps_in(q)):
-                yield ("wait", x_ready[g], q & 1)
-                accumulate_mma(q, g)
-            yield mma(sim, acc_cycles * steps_in(q), [x_free, kempty[q % NK]],
-                      [lambda q=q: acc_done(q), lambda q=q: kring.release(q)])
-
         for p in range(pairs):
             yield ("wait", kfull[p % NK], (p // NK) & 1)
             yield ("wait", vfull[p % NV], (p // NV) & 1)
@@ -162,11 +156,16 @@ def simulate_dq(n, seed, member_rate, skip=None, acc_cycles=512):
                 yield ("wait", read, (p - 1) & 1)
             burst(p)
             yield mma(sim, 1024, [sd_ready, vempty[p % NV]], [lambda p=p: vring.release(p)])
-            if p > 0:
-                yield from accumulate(p - 1)
-        if pairs > 0:
-            yield from accumulate(pairs - 1)
-        yield mma(sim, 10, [done])
+        yield mma(sim, 1, [done])
+
+    def acc_issuer():
+        for q in range(pairs):
+            for g in range(steps_in(q)):
+                yield ("wait", x_ready[g], q & 1)
+                accumulate_mma(q, g)
+            yield mma(sim, acc_cycles * steps_in(q), [x_free, kempty[q % NK]],
+                      [lambda q=q: acc_done(q), lambda q=q: kring.release(q)])
+        yield mma(sim, 1, [done])
 
     def group_warp(g, quad):
         yield ("delay", rng.randint(50, 600))
@@ -199,7 +198,7 @@ def simulate_dq(n, seed, member_rate, skip=None, acc_cycles=512):
         if acc["done"] != n:
             raise Hazard("epilogue read dQ after %d of %d accumulations" % (acc["done"], n))
 
-    roles = {"loader": loader(), "issuer": issuer()}
+    roles = {"loader": loader(), "bursts": burst_issuer(), "accumulations": acc_issuer()}
     for g in range(2):
         for quad in range(4):
             roles["group%d.%d" % (g, quad)] = group_warp(g, quad)
@@ -212,13 +211,15 @@ def simulate_dkdv(n, seed, member_rate, skip=None, acc_cycles=512):
     rng = sim.rng
     pairs = (n + 1) // 2
     full = [Barrier("full%d" % s, 1) for s in range(NR)]
-    sd_ready = Barrier("sd_ready", 1)
+    s_ready = Barrier("s_ready", 1)
+    dp_ready = Barrier("dp_ready", 1)
+    st_issued = Barrier("st_issued", 1)
     p_ready = [Barrier("p_ready%d" % g, 4) for g in range(2)]
     ds_ready = [Barrier("ds_ready%d" % g, 4) for g in range(2)]
     xv_free = Barrier("xv_free", 1)
     xk_free = Barrier("xk_free", 1)
     own = Barrier("own", 8)
-    done = Barrier("done", 1)
+    done = Barrier("done", 2)
     ring = Slots("Q/dO", NR)
     # tensor memory per group and warp (each warp writes its own rows): the
     # S^T columns hold ("S", pair) until P^T is written over them, the dP^T
@@ -261,7 +262,7 @@ def simulate_dkdv(n, seed, member_rate, skip=None, acc_cycles=512):
         if acc["released"][q] == 2:
             ring.release(q)
 
-    def issuer():
+    def burst_issuer():
         if pairs > 0:
             yield from load(0)
         if pairs > 1:
@@ -272,52 +273,65 @@ def simulate_dkdv(n, seed, member_rate, skip=None, acc_cycles=512):
             if p > 0 and skip != "xv_free":
                 yield ("wait", xv_free, (p - 1) & 1)
             burst(st, "S", p, "dV")
-            yield mma(sim, 512, [])
+            yield mma(sim, 512, [s_ready])
+            yield ("arrive", st_issued, 1)
             if p > 0 and skip != "xk_free":
                 yield ("wait", xk_free, (p - 1) & 1)
             burst(dpt, "dP", p, "dK")
-            yield mma(sim, 512, [sd_ready])
+            yield mma(sim, 512, [dp_ready])
             if 1 <= p and p + 1 < pairs:
                 yield from load(p + 1)
+        yield mma(sim, 1, [done])
+
+    def acc_issuer():
+        for p in range(pairs):
             for g in range(steps_in(p)):
                 yield ("wait", p_ready[g], p & 1)
                 accumulate_mma(st, "P", p, g)
             yield mma(sim, acc_cycles * steps_in(p), [xv_free],
                       [lambda p=p: finished(st, p, "dv")])
+            # dK after the next pair's S^T, so that its P^T phase starts early
+            if p + 1 < pairs:
+                yield ("wait", st_issued, (p + 1) & 1)
             for g in range(steps_in(p)):
                 yield ("wait", ds_ready[g], p & 1)
                 accumulate_mma(dpt, "dS", p, g)
             yield mma(sim, acc_cycles * steps_in(p), [xk_free],
                       [lambda p=p: finished(dpt, p, "dk")])
-        yield mma(sim, 10, [done])
+        yield mma(sim, 1, [done])
 
     def group_warp(g, quad):
         yield ("delay", rng.randint(50, 600))
         yield ("arrive", own, 1)
         lo, hi = compute_time(rng)
         for p in range(pairs):
-            yield ("wait", sd_ready, p & 1)
+            yield ("wait", s_ready, p & 1)
             if 2 * p + g >= n:
                 continue
-            for cols, what in ((st, "S"), (dpt, "dP")):
-                x = cols[g][quad]
-                if x["what"] != what or x["pair"] != p:
-                    raise Hazard("group %d warp %d read %s/%s for %s of pair %d"
-                                 % (g, quad, x["what"], x["pair"], what, p))
+            x = st[g][quad]
+            if x["what"] != "S" or x["pair"] != p:
+                raise Hazard("group %d warp %d read %s/%s for S^T of pair %d"
+                             % (g, quad, x["what"], x["pair"], p))
             yield ("delay", rng.randint(50, 150))
             busy = rng.random() < member_rate
             yield ("delay", rng.randint(lo, hi) if busy else rng.randint(20, 200))
-            st[g][quad]["what"] = "P"
+            x["what"] = "P"
             yield ("arrive", p_ready[g], 1)
+            if skip != "dp_ready":
+                yield ("wait", dp_ready, p & 1)
+            x = dpt[g][quad]
+            if x["what"] != "dP" or x["pair"] != p:
+                raise Hazard("group %d warp %d read %s/%s for dP^T of pair %d"
+                             % (g, quad, x["what"], x["pair"], p))
             yield ("delay", rng.randint(30, 400))
-            dpt[g][quad]["what"] = "dS"
+            x["what"] = "dS"
             yield ("arrive", ds_ready[g], 1)
         yield ("wait", done, 0)
         if acc["dv"] != n or acc["dk"] != n:
             raise Hazard("epilogue read dK/dV after %d/%d of %d accumulations"
                          % (acc["dv"], acc["dk"], n))
 
-    roles = {"issuer": issuer()}
+    roles = {"bursts": burst_issuer(), "accumulations": acc_issuer()}
     for g in range(2):
         for quad in range(4):
             roles["group%d.%d" % (g, quad)] = group_warp(g, quad)
@@ -352,6 +366,7 @@ def test_backward_protocol_has_no_hazard(kernel):
     ("dq", "kempty", "a K slot reloaded under its accumulation"),
     ("dkdv", "xv_free", "P^T overwritten before dV read it"),
     ("dkdv", "xk_free", "dS^T overwritten before dK read it"),
+    ("dkdv", "dp_ready", "dP^T read before its burst finished"),
 ])
 def test_planted_mistake_is_caught(kernel, skip, what):
     caught = 0
