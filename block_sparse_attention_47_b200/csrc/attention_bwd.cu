@@ -648,10 +648,15 @@ __global__ void __launch_bounds__(352, 1)
         }
         tc_commit(s_ready);
         mbar_arrive(st_issued);
-        // dP^T once dK has read dS^T of pair p-1
+        // dP^T once dK has read dS^T of pair p-1; pair p+1 goes into the
+        // slot of pair p-1 as soon as both its accumulations have finished
         if (p > 0 && !mbar_wait(xk_free, (p - 1) & 1, abort_flag)) {
           ok = false;
           break;
+        }
+        if (p >= 1 && p + 1 < np) {
+          load(p + 1);
+          loaded = p + 2;
         }
         tc_fence_after();
 #pragma unroll
@@ -661,11 +666,6 @@ __global__ void __launch_bounds__(352, 1)
                     sdesc_sw128(doslot(p) + off, 16, 1024), idesc_s, kk > 0);
         }
         tc_commit(dp_ready);
-        // pair p+1 into the slot of pair p-1, whose accumulations finished
-        if (p >= 1 && p + 1 < np) {
-          load(p + 1);
-          loaded = p + 2;
-        }
       }
       if (!ok) {
         report_timeout(abort_flag, io.status);
@@ -758,7 +758,10 @@ __global__ void __launch_bounds__(352, 1)
       const int tile = int(entry & kTileMask);
       const uint32_t flags = entry >> kFlagShift;
       const bool member = key_valid && ((flags >> half) & 1u);
-      const bool dense = member && (flags & 4u);  // every query slot is a real token
+      // every query slot is a real token and every row of the warp a member:
+      // warp-uniform, since both paths below end in warp-wide tensor-memory
+      // stores
+      const bool dense = __all_sync(0xffffffffu, member && (flags & 4u));
       uint32_t sv[64], dp[64];
       BSA_TMEM_LD64(tS, sv);
       // query slots of block `tile`: real tokens only (pad queries have no output)
@@ -767,35 +770,53 @@ __global__ void __launch_bounds__(352, 1)
       const float* lse = reinterpret_cast<const float*>(sm + C::OFF_VEC + (p % NR) * 1024) + 64 * grp;
       const float* dlt = lse + 128;
       // P^T over S^T first, so that dV starts while dS^T is computed; the
-      // probabilities stay in sv.  32 query columns (16 packed) at a time.
+      // probabilities stay in sv.  32 query columns (16 packed) at a time,
+      // with the dense case in a branch-free loop of its own so that the
+      // exponentials of successive columns overlap.
+      if (dense) {
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t pk[16];
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[16];
+          float4 l4[8];
 #pragma unroll
-        for (int c4 = 8 * h2; c4 < 8 * h2 + 8; ++c4) {
-          const float4 l4 = reinterpret_cast<const float4*>(lse)[c4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          for (int i = 0; i < 8; ++i) l4[i] = reinterpret_cast<const float4*>(lse)[8 * h2 + i];
 #pragma unroll
-          for (int u = 0; u < 4; u += 2) {
-            const int c = 4 * c4 + u;
+          for (int i = 0; i < 8; ++i) {
+            const int c = 32 * h2 + 4 * i;
+            float x0, x1, x2, x3;
+            fma_f32x2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2,
+                      -l4[i].x, -l4[i].y);
+            fma_f32x2(x2, x3, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]), sl2, sl2,
+                      -l4[i].z, -l4[i].w);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+            sv[c] = __float_as_uint(p0);
+            sv[c + 1] = __float_as_uint(p1);
+            sv[c + 2] = __float_as_uint(p2);
+            sv[c + 3] = __float_as_uint(p3);
+            pk[2 * i] = pack_bf16x2(p0, p1);
+            pk[2 * i + 1] = pack_bf16x2(p2, p3);
+          }
+          BSA_TMEM_ST16(tS + 16u * h2, pk);
+        }
+      } else {
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 32 * h2; c < 32 * h2 + 32; c += 2) {
             float p0 = 0.f, p1 = 0.f;
-            if (dense) {
-              float x0, x1;
-              fma_f32x2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2,
-                        -lv[u], -lv[u + 1]);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            } else if (member) {
-              if (bit_of(lo, hi, c)) p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
+            if (member) {
+              if (bit_of(lo, hi, c)) p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse[c]));
               if (bit_of(lo, hi, c + 1))
-                p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lv[u + 1]));
+                p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse[c + 1]));
             }
             sv[c] = __float_as_uint(p0);
             sv[c + 1] = __float_as_uint(p1);
             pk[(c - 32 * h2) / 2] = pack_bf16x2(p0, p1);
           }
+          BSA_TMEM_ST16(tS + 16u * h2, pk);
         }
-        BSA_TMEM_ST16(tS + 16u * h2, pk);
       }
       tc_fence_before();
       __syncwarp();

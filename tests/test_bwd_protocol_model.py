@@ -277,10 +277,10 @@ def simulate_dkdv(n, seed, member_rate, skip=None, acc_cycles=512):
             yield ("arrive", st_issued, 1)
             if p > 0 and skip != "xk_free":
                 yield ("wait", xk_free, (p - 1) & 1)
-            burst(dpt, "dP", p, "dK")
-            yield mma(sim, 512, [dp_ready])
             if 1 <= p and p + 1 < pairs:
                 yield from load(p + 1)
+            burst(dpt, "dP", p, "dK")
+            yield mma(sim, 512, [dp_ready])
         yield mma(sim, 1, [done])
 
     def acc_issuer():
