@@ -294,13 +294,37 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y, b = bh / g.h;
 
-  // the step-table warp starts its first global loads (the two lists'
-  // lengths) before the set-up barrier, so their latency overlaps it
+  // the step-table warp issues all of its global loads before the set-up
+  // barrier, so that their latencies overlap it and one another: the two
+  // lists' lengths, their first 256 entries (read up to the lists' capacity,
+  // since the lengths are not known yet) and the full-block flags of the
+  // first 64 bitmap words
   int pre_cnt[2] = {-1, -1};
-  if (MODE == kModeLists && warp == 8) {
+  int pre_a[8], pre_b[8];
+  uint32_t pre_f[2][8];
+  if (warp == 8) {
+    if constexpr (MODE == kModeLists) {
+      const int32_t* srcA = idx + (int64_t(bh) * g.nb + 2 * pair) * g.kcap;
+      const bool has_b = 2 * pair + 1 < g.nb;
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf)
-      if (2 * pair + hf < g.nb) pre_cnt[hf] = __ldg(cnt + int64_t(bh) * g.nb + 2 * pair + hf);
+      for (int hf = 0; hf < 2; ++hf)
+        if (2 * pair + hf < g.nb) pre_cnt[hf] = __ldg(cnt + int64_t(bh) * g.nb + 2 * pair + hf);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = 32 * u + lane;
+        pre_a[u] = i < g.kcap ? __ldg(srcA + i) : -1;
+        pre_b[u] = i < g.kcap && has_b ? __ldg(srcA + g.kcap + i) : -1;
+      }
+    }
+    const uint32_t* f4 = reinterpret_cast<const uint32_t*>(bfull + int64_t(b) * g.nb);
+    const bool words = ((int64_t(b) * g.nb) & 3) == 0;  // 4-byte aligned flags
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int w = lane + 32 * r;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        pre_f[r][i] = words && 32 * w + 32 <= g.nb ? __ldg(f4 + 8 * w + i) : 0u;
+    }
   }
 
   if (threadIdx.x == 0) {
@@ -395,8 +419,9 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int i = base + 32 * u + lane;
-            va[u] = i < nA ? __ldg(srcA + i) : -1;
-            vb[u] = i < nB ? __ldg(srcB + i) : -1;
+            // the first 256 entries were loaded before the set-up barrier
+            va[u] = i >= nA ? -1 : (base == 0 ? pre_a[u] : __ldg(srcA + i));
+            vb[u] = i >= nB ? -1 : (base == 0 ? pre_b[u] : __ldg(srcB + i));
           }
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -411,11 +436,12 @@ __global__ void __launch_bounds__(512, 1)
       for (int w = lane; w < nw; w += 32) {
         uint32_t f = 0u;
         if (words && 32 * w + 32 <= g.nb) {
-          // eight 4-byte loads of the 32 flag bytes (each byte 0 or 1)
+          // eight 4-byte words of the 32 flag bytes (each byte 0 or 1); those
+          // of the first 64 bitmap words were loaded before the set-up barrier
           const uint32_t* f4 = reinterpret_cast<const uint32_t*>(full_row + 32 * w);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const uint32_t x = __ldg(f4 + i);
+            const uint32_t x = w < 32 ? pre_f[0][i] : (w < 64 ? pre_f[1][i] : __ldg(f4 + i));
             f |= (((x & 0xFFu) != 0u) | (((x >> 8) & 0xFFu) != 0u) << 1 |
                   (((x >> 16) & 0xFFu) != 0u) << 2 | ((x >> 24) != 0u) << 3) << (4 * i);
           }
