@@ -48,8 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # written), scaled by the number of (batch, head) problems.  Valid only for
 # the kernel source it was measured on and the 720p keep-480 fixed-block
 # workload on the permuted path; null otherwise.
-ATTN_TRAFFIC = {"sha256": "049ff65fc9c444e7de9b63a04d0dd7d36a92d669cfbfff03206733a198ad2296",
-                "bytes_per_bh": (2.118633e9 + 0.125721e9) / 4, "workload": ("720p", 0.25, 0)}
+ATTN_TRAFFIC = {"sha256": "4d2c4962edb62dac8bee4b4d4b3f9ff60c58d586771bb1c8242ce43d2a543feb",
+                "bytes_per_bh": (1.943522e9 + 0.124784e9) / 4, "workload": ("720p", 0.25, 0)}
 
 
 def attn_traffic(cfg, keep_ratio):
