@@ -346,7 +346,9 @@ __global__ void __launch_bounds__(352, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
-      const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+      // test hook: with stall_pv set no accumulation is issued, so the
+      // groups' wait for the first one runs out (the timeout path)
+      const int n = ok && !g.stall_pv ? *n_steps_sm : 0, np = (n + 1) >> 1;
       for (int q = 0; ok && q < np; ++q) {
         const int ns = 2 * q + 1 < n ? 2 : 1;
         for (int h = 0; h < ns; ++h) {
@@ -685,7 +687,9 @@ __global__ void __launch_bounds__(352, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
       bool ok = mbar_wait(bar_steps, 0, abort_flag);
-      const int n = ok ? *n_steps_sm : 0, np = (n + 1) >> 1;
+      // test hook: with stall_pv set no accumulation is issued, so the
+      // burst thread's wait for the first one runs out (the timeout path)
+      const int n = ok && !g.stall_pv ? *n_steps_sm : 0, np = (n + 1) >> 1;
       for (int p = 0; ok && p < np; ++p) {
         const int ns = 2 * p + 1 < n ? 2 : 1;
         for (int h = 0; h < ns && ok; ++h) {

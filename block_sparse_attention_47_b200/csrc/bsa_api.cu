@@ -60,7 +60,7 @@ bsa_status cuda_fail(cudaError_t e, const char* what) {
 // dev_status = NULL; read and cleared by bsa_take_default_status
 __device__ int32_t g_dev_status_sink;
 
-// test hook (bsa_debug_stall_pv): attention launches made by this thread
+// test hook (bsa_debug_stall_pv): attention launches (forward and backward) made by this thread
 // while it is set issue no PV; other threads' launches are unaffected
 thread_local int g_stall_pv = 0;
 
@@ -555,6 +555,7 @@ bsa_status bsa_sparse_attn_bwd(const bsa_problem* prob, const void* layout_buf,
     return fail(BSA_ERR_WORKSPACE, "workspace of %zu bytes; the backward needs %zu", ws_bytes,
                 need);
   BSA_TRY(check_device());
+  g.stall_pv = g_stall_pv;
   CUtensorMap maps[4];
   BSA_TRY(make_map(&maps[0], g, k_perm, 64));
   BSA_TRY(make_map(&maps[1], g, v_perm, 64));

@@ -375,13 +375,14 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
                             int32_t heads_per_group, int32_t* dev_status, void* stream);
 
 /* Test hook for the device-side timeout path.  While enabled (nonzero),
- * attention launches issue no PV product, so the softmax's bounded wait on
- * the first PV runs out after 2 s.  The kernel then writes BSA_ERR_TIMEOUT
- * to the status word, drains its copies and MMAs, frees tensor memory and
- * returns, and the CUDA context stays usable.  Output is undefined for
- * launches made while enabled.  The switch belongs to the calling thread:
- * only attention launches queued by that thread are affected, never
- * another thread's.  Off by default. */
+ * attention launches issue no PV product (forward) and no accumulation
+ * (backward: dQ += dS K, dV += P^T dO, dK += dS^T Q), so a bounded wait on
+ * the first of them runs out after 2 s.  The kernel then writes
+ * BSA_ERR_TIMEOUT to the status word, drains its copies and MMAs, frees
+ * tensor memory and returns, and the CUDA context stays usable.  Output is
+ * undefined for launches made while enabled.  The switch belongs to the
+ * calling thread: only attention launches queued by that thread are
+ * affected, never another thread's.  Off by default. */
 bsa_status bsa_debug_stall_pv(int32_t enable);
 
 /* The library-owned status word of the current device, which receives the

@@ -154,3 +154,31 @@ def test_backward_full_size_720p_identities_and_sampled_rows():
             want = scale * ds @ kp[keys]
             want[~O.slot_valid(geo, perm)[rows]] = 0.0
             grad_close(gq[b, hh, rows].cpu().numpy(), want, "720p dQ b%d h%d block %d" % (b, hh, i))
+
+
+def test_backward_stall_reports_timeout_and_context_survives():
+    """With the stall hook the backward issues no accumulation, so the row
+    groups' bounded waits run out: BSA_ERR_TIMEOUT in the status word, no
+    fault, and a normal backward afterwards gives the same gradients."""
+    cfg = SMALL["tiny"]
+    run, _, o, lse, dout, grads = run_backward(cfg, 5300)
+    good = [t.clone() for t in grads]
+    attn, prob = run.attn, run.prob
+    ws = torch.empty(bsa.bwd_workspace_bytes(prob), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stalled = [torch.empty_like(attn.op) for _ in range(3)]
+    bsa.debug_stall_pv(True)
+    try:
+        bsa.sparse_attn_bwd(prob, attn.layout_buf, attn.qp, attn.kp, attn.vp, o, dout, lse,
+                            attn.idx, attn.cnt, *stalled, ws, status)
+        torch.cuda.synchronize()        # returns: the kernels gave up, they did not hang
+    finally:
+        bsa.debug_stall_pv(False)
+    assert int(status.item()) == 6, "expected BSA_ERR_TIMEOUT"
+    again = [torch.full_like(attn.op, float("nan")) for _ in range(3)]
+    bsa.sparse_attn_bwd(prob, attn.layout_buf, attn.qp, attn.kp, attn.vp, o, dout, lse, attn.idx,
+                        attn.cnt, *again, ws, attn.status)
+    torch.cuda.synchronize()
+    attn.check_status()
+    for a, b_ in zip(again, good):
+        assert torch.equal(a, b_), "a normal backward after the timeout must be unaffected"
