@@ -722,10 +722,11 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_copy_mutex;
-cudaStream_t g_copy_in[kMaxDevices], g_copy_out[kMaxDevices];
+cudaStream_t g_copy_in[kMaxDevices], g_copy_out[kMaxDevices], g_compute[kMaxDevices];
 
-// the two copy streams of the current device, created on first use
-bsa_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
+// the library's streams of the current device (uploads, downloads and a
+// second compute stream), created on first use
+bsa_status side_streams(cudaStream_t* in, cudaStream_t* out, cudaStream_t* cmp) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -734,10 +735,12 @@ bsa_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
   if (!g_copy_in[dev]) {
     e = cudaStreamCreateWithFlags(&g_copy_in[dev], cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&g_copy_out[dev], cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&g_compute[dev], cudaStreamNonBlocking);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
   }
   *in = g_copy_in[dev];
   *out = g_copy_out[dev];
+  *cmp = g_compute[dev];
   return BSA_OK;
 }
 
@@ -789,8 +792,8 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
     return fail(BSA_ERR_INVALID_ARG, "heads_per_group %d must divide heads (%d)", heads_per_group,
                 g.h);
   BSA_TRY(check_device());
-  cudaStream_t st = static_cast<cudaStream_t>(stream), s_in, s_out;
-  BSA_TRY(copy_streams(&s_in, &s_out));
+  cudaStream_t st = static_cast<cudaStream_t>(stream), s_in, s_out, s_c2;
+  BSA_TRY(side_streams(&s_in, &s_out, &s_c2));
 
   const int groups = g.h / heads_per_group;
   bsa_problem sub = *prob;
@@ -807,10 +810,11 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
   const size_t cnt_elems = size_t(g.B) * heads_per_group * g.nb;
   const bool dynamic = g.mode == BSA_BLOCK_DYNAMIC_888;
 
-  EventSet es;  // start, k, in[groups], out[groups], done
-  cudaError_t e = es.make(3 + 2 * size_t(groups));
+  EventSet es;  // start, k, in[groups], out[groups], done, layout
+  cudaError_t e = es.make(4 + 2 * size_t(groups));
   if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags");
   cudaEvent_t ev_start = es.ev[0], ev_k = es.ev[1], ev_done = es.ev[2 + 2 * groups];
+  cudaEvent_t ev_layout = es.ev[3 + 2 * groups];
   auto ev_in = [&](int i) { return es.ev[2 + i]; };
   auto ev_out = [&](int i) { return es.ev[2 + groups + i]; };
   auto slab = [&](const void* base, int grp) {
@@ -834,6 +838,10 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
     BSA_CUDA(cudaStreamWaitEvent(st, ev_k, 0), "cudaStreamWaitEvent");
   }
   BSA_TRY(bsa_layout(prob, buf->k_raster, sb, sn, sh, buf->layout_buf, st));
+  // odd groups compute on the library's second stream, so that a group's
+  // first kernels fill the SMs that the previous group's last ones leave idle
+  BSA_CUDA(cudaEventRecord(ev_layout, st), "cudaEventRecord");
+  BSA_CUDA(cudaStreamWaitEvent(s_c2, ev_layout, 0), "cudaStreamWaitEvent");
 
   // uploads: every group's slabs, in order, on the input stream
   for (int i = 0; i < groups; ++i) {
@@ -849,7 +857,8 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
   }
   // computation of each group once its slabs have landed
   for (int i = 0; i < groups; ++i) {
-    BSA_CUDA(cudaStreamWaitEvent(st, ev_in(i), 0), "cudaStreamWaitEvent");
+    const cudaStream_t cs = (i & 1) ? s_c2 : st;
+    BSA_CUDA(cudaStreamWaitEvent(cs, ev_in(i), 0), "cudaStreamWaitEvent");
     const int64_t h0 = int64_t(i) * heads_per_group * g.d;  // element offset of the slab
     auto rq = static_cast<const __nv_bfloat16*>(buf->q_raster) + h0;
     auto rk = static_cast<const __nv_bfloat16*>(buf->k_raster) + h0;
@@ -864,19 +873,19 @@ bsa_status bsa_forward_host(const bsa_problem* prob, const void* q_host, const v
     int32_t* idx = buf->idx + i * idx_elems;
     int32_t* cnt = buf->cnt + i * cnt_elems;
     if (raster) {
-      BSA_TRY(bsa_pool_raster(&sub, buf->layout_buf, rq, rk, sb, sn, sh, qpool, kpool, st));
-      BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
+      BSA_TRY(bsa_pool_raster(&sub, buf->layout_buf, rq, rk, sb, sn, sh, qpool, kpool, cs));
+      BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, cs));
       BSA_TRY(bsa_sparse_attn_fwd_raster(&sub, buf->layout_buf, rq, rk, rv, sb, sn, sh, idx, cnt,
-                                         ro, sb, sn, sh, dev_status, st));
+                                         ro, sb, sn, sh, dev_status, cs));
     } else {
       BSA_TRY(bsa_permute_pool(&sub, buf->layout_buf, rq, rk, rv, sb, sn, sh, pq, pk, pv, qpool,
-                               kpool, st));
-      BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, st));
+                               kpool, cs));
+      BSA_TRY(bsa_select_topk(&sub, qpool, kpool, idx, cnt, cs));
       BSA_TRY(bsa_sparse_attn_fwd(&sub, buf->layout_buf, pq, pk, pv, idx, cnt, po, dev_status,
-                                  st));
-      BSA_TRY(bsa_unpermute(&sub, buf->layout_buf, po, ro, sb, sn, sh, st));
+                                  cs));
+      BSA_TRY(bsa_unpermute(&sub, buf->layout_buf, po, ro, sb, sn, sh, cs));
     }
-    BSA_CUDA(cudaEventRecord(ev_out(i), st), "cudaEventRecord");
+    BSA_CUDA(cudaEventRecord(ev_out(i), cs), "cudaEventRecord");
   }
   // downloads on the output stream; the caller's stream ends with the last one
   for (int i = 0; i < groups; ++i) {

@@ -352,8 +352,11 @@ typedef struct bsa_device_buffers {
  * transfers overlapped with the computation.  Heads are processed in groups
  * of `heads_per_group`.  Group g+1 is copied to the device while group g is
  * computed and group g-1's output is copied back, on two library-owned
- * copy streams tied to `stream` by events.  The dynamic layout needs every
- * head of K, so in dynamic mode K is copied whole first.
+ * copy streams tied to `stream` by events.  Even groups compute on `stream`,
+ * odd ones on a third library-owned stream, so that one group's first
+ * kernels run on the SMs that the previous group's last kernels leave idle.
+ * The dynamic layout needs every head of K, so in dynamic mode K is copied
+ * whole first.
  *   q_host, k_host, v_host  [B, N, heads, head_dim] bf16, contiguous, host
  *                           memory (page-locked memory lets copies overlap)
  *   o_host                  same layout, written; pad tokens are 0
