@@ -71,13 +71,23 @@ METRIC = "ms/call & effective TFLOP/s (kept tiles) at 122,880 tok, s=0.75; % BF1
 
 # ----------------------------------------------------------------------------
 def peaks():
+    """The measured peaks where the file gives them, each missing number
+    taken from the fallback figures; the kind says which the sustained bf16
+    figure (the roofline's denominator) is."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    p = dict(FALLBACK_PEAKS)
     try:
         with open(path) as f:
-            p = json.load(f)
-        return p, "measured"
+            got = json.load(f)
     except (OSError, ValueError):
-        return dict(FALLBACK_PEAKS), "fallback"
+        return p, "fallback"
+    if not isinstance(got, dict):
+        return p, "fallback"
+    for key in FALLBACK_PEAKS:
+        if isinstance(got.get(key), (int, float)) and got[key] > 0:
+            p[key] = float(got[key])
+    measured = isinstance(got.get("bf16_tflops_sustained"), (int, float))
+    return p, "measured" if measured else "fallback"
 
 
 # tcgen05 dense bf16 rate per SM and clock (4,096 multiply-adds; measured

@@ -85,3 +85,23 @@ def test_mma_rate_fraction_at_clock():
     assert bench.mma_rate_frac(606.208, {"sm_mhz": 1000.0}) == pytest.approx(0.5)
     assert bench.mma_rate_frac(500.0, None) is None
     assert bench.mma_rate_frac(500.0, {"sm_mhz": None}) is None
+
+
+def test_peaks_fall_back_per_missing_number(tmp_path, monkeypatch):
+    """The generated peaks file: each number it gives is used, each one it
+    lacks (or gives in an unusable form) comes from the fallback figures."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p, kind = bench.peaks()
+    assert kind == "fallback" and p == bench.FALLBACK_PEAKS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6464.9, "bf16_tflops": "n/a", "clocks": {"sm": 1965}}))
+    p, kind = bench.peaks()
+    assert kind == "fallback"
+    assert p["hbm_gbs"] == 6464.9 and p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6464.9, "bf16_tflops": 1641.7, "bf16_tflops_sustained": 1368.0}))
+    p, kind = bench.peaks()
+    assert kind == "measured" and p["bf16_tflops_sustained"] == 1368.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text("[1, 2]")
+    assert bench.peaks() == (bench.FALLBACK_PEAKS, "fallback")
