@@ -425,10 +425,12 @@ bsa_status bsa_select_topk(const bsa_problem* prob, const float* q_pool, const f
   BSA_TRY(check_ptr4(idx, "idx"));
   BSA_TRY(check_ptr4(cnt, "cnt"));
   BSA_TRY(check_device());
+  int32_t* status = nullptr;  // the library's word of this device
+  BSA_TRY(status_word(&status));
   CUtensorMap kmap;
   const bool tma = make_pool_map(&kmap, g, k_pool);
   cudaError_t e = bsa::launch_select(g, q_pool, k_pool, nullptr, tma ? &kmap : nullptr, idx, cnt,
-                                     static_cast<cudaStream_t>(stream));
+                                     status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_select_topk launch");
 }
 
@@ -445,10 +447,12 @@ bsa_status bsa_select_topk_gated(const bsa_problem* prob, const float* q_pool,
   BSA_TRY(check_ptr4(idx, "idx"));
   BSA_TRY(check_ptr4(cnt, "cnt"));
   BSA_TRY(check_device());
+  int32_t* status = nullptr;  // the library's word of this device
+  BSA_TRY(status_word(&status));
   CUtensorMap kmap;
   const bool tma = make_pool_map(&kmap, g, k_pool);
   cudaError_t e = bsa::launch_select(g, q_pool, k_pool, gate, tma ? &kmap : nullptr, idx, cnt,
-                                     static_cast<cudaStream_t>(stream));
+                                     status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e, "bsa_select_topk_gated launch");
 }
 

@@ -104,8 +104,10 @@ cudaError_t launch_pool(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* qp,
                         const __nv_bfloat16* kp, float* qpool, float* kpool, cudaStream_t st);
 // kmap (optional): 2-D map over the pooled keys [B*heads*nb rows, d] fp32,
 // 32 x 256 boxes, 128-byte swizzle (the TMA-fed score tiles)
+// status: where a bounded wait that runs out reports BSA_ERR_TIMEOUT
 cudaError_t launch_select(const Geo& g, const float* qpool, const float* kpool, const float* gate,
-                          const CUtensorMap* kmap, int32_t* idx, int32_t* cnt, cudaStream_t st);
+                          const CUtensorMap* kmap, int32_t* idx, int32_t* cnt, int32_t* status,
+                          cudaStream_t st);
 cudaError_t launch_pool_raster(const Geo& g, LayoutPtrs lp, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, int64_t sb, int64_t sn, int64_t sh,
                                float* qpool, float* kpool, cudaStream_t st);
