@@ -682,40 +682,6 @@ __device__ __forceinline__ void store_split(uint32_t hi_tile, uint32_t lo_tile, 
                                          __float_as_uint(l.z), __float_as_uint(l.w)));
 }
 
-// q~ = G q for the ROWS rows in sq, in place (the FMA kernels' arithmetic):
-// thread t takes channel c = t % d of rows t / d, t / d + NT / d, .., each
-// output one fmaf chain in e order
-template <int NT, int ROWS>
-__device__ __forceinline__ void gate_rows(const Geo& g, const float* __restrict__ gate, int bh,
-                                          float* sq) {
-  const float* G = gate + int64_t(bh % g.h) * g.d * g.d;
-  constexpr int MAXO = (ROWS * 128) / NT;
-  const int c = threadIdx.x % g.d, r0 = threadIdx.x / g.d, rstep = NT / g.d;
-  const int nout = ROWS * g.d / NT;
-  float acc[MAXO];
-#pragma unroll
-  for (int o = 0; o < MAXO; ++o) acc[o] = 0.f;
-  const float4* gr = reinterpret_cast<const float4*>(G + int64_t(c) * g.d);
-  for (int e4 = 0; e4 < g.d / 4; ++e4) {
-    const float4 gv = __ldg(gr + e4);
-#pragma unroll
-    for (int o = 0; o < MAXO; ++o) {
-      if (o < nout) {
-        const float4 qv = reinterpret_cast<const float4*>(sq + (r0 + rstep * o) * g.d)[e4];
-        acc[o] = fmaf(gv.x, qv.x, acc[o]);
-        acc[o] = fmaf(gv.y, qv.y, acc[o]);
-        acc[o] = fmaf(gv.z, qv.z, acc[o]);
-        acc[o] = fmaf(gv.w, qv.w, acc[o]);
-      }
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int o = 0; o < MAXO; ++o)
-    if (o < nout) sq[(r0 + rstep * o) * g.d + c] = acc[o];
-  __syncthreads();
-}
-
 __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads, 1)
     select_tc_kernel(Geo g, int KC, const float* __restrict__ qpool,
                      const float* __restrict__ kpool, const float* __restrict__ gate,
@@ -764,7 +730,46 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  if (gate) gate_rows<kTcThreads, kTcM>(g, gate, bh, sq);
+  if (gate) {
+    // q~ = G q: this CTA maps the 16 rows it owns (the FMA kernels' fmaf
+    // chains) and stores them into every CTA's copy of the rows, once every
+    // CTA has loaded its plain rows
+    cluster.sync();
+    const float* G = gate + int64_t(bh % g.h) * g.d * g.d;
+    constexpr int MAXO = kTcRows * 128 / kTcThreads;
+    const int c = threadIdx.x % g.d, q0 = threadIdx.x / g.d, qstep = kTcThreads / g.d;
+    const int nout = kTcRows * g.d / kTcThreads;
+    const int mine = crank * kTcRows;
+    float acc[MAXO];
+#pragma unroll
+    for (int o = 0; o < MAXO; ++o) acc[o] = 0.f;
+    const float4* gr = reinterpret_cast<const float4*>(G + int64_t(c) * g.d);
+    // eight loads of the gate row in flight (d / 4 is a multiple of 8)
+#pragma unroll 8
+    for (int e4 = 0; e4 < g.d / 4; ++e4) {
+      const float4 gv = __ldg(gr + e4);
+#pragma unroll
+      for (int o = 0; o < MAXO; ++o) {
+        if (o < nout) {
+          const float4 qv =
+              reinterpret_cast<const float4*>(sq + (mine + q0 + qstep * o) * g.d)[e4];
+          acc[o] = fmaf(gv.x, qv.x, acc[o]);
+          acc[o] = fmaf(gv.y, qv.y, acc[o]);
+          acc[o] = fmaf(gv.z, qv.z, acc[o]);
+          acc[o] = fmaf(gv.w, qv.w, acc[o]);
+        }
+      }
+    }
+    __syncthreads();  // this CTA's own rows are read before they are replaced
+#pragma unroll 1
+    for (int dst = 0; dst < kTcCluster; ++dst) {
+      float* rq = cluster.map_shared_rank(sq, dst);
+#pragma unroll
+      for (int o = 0; o < MAXO; ++o)
+        if (o < nout) rq[(mine + q0 + qstep * o) * g.d + c] = acc[o];
+    }
+    cluster.sync();  // every CTA's rows are mapped
+  }
   // the query rows as A tiles: [chunk][128 rows][32 channels], hi and lo
   for (int e = threadIdx.x; e < kTcM * g.d / 4; e += kTcThreads) {
     const int r = e / (g.d / 4), c4 = e % (g.d / 4);
