@@ -614,7 +614,8 @@ __global__ void __launch_bounds__(kSelThreads * RG) select_kernel(
 // channels per MMA, with every fp32 operand split as x = hi + lo (hi = x with
 // its low 13 mantissa bits cleared, a tf32 value, so the split is exact) and
 // S = qh.kh + qh.kl + ql.kh accumulated in fp32: the dropped ql.kl term and
-// the tf32 rounding of lo stay below 2^-20 of |q||k| per channel.  Each CTA
+// the tf32 truncation of each lo are each below 2^-20 |q||k| per channel,
+// so a product is within 3 * 2^-20 |q||k| of the exact one.  Each CTA
 // then stores every row's order keys into the shared memory of the CTA that
 // owns the row (rows 16 c' .. 16 c' + 15 belong to CTA c'), and after a
 // cluster barrier every CTA runs the same per-row top-k as the FMA kernels

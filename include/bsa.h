@@ -176,8 +176,8 @@ bsa_status bsa_permute_pool(const bsa_problem* prob, const void* layout_buf, con
  * cnt[i] = nbp + keep_blocks.  Prefix query blocks attend densely:
  * cnt = -1 and their idx row is left untouched (Ref2VA VSA, section
  * "조건 토큰은 왜 다르게 다루나").  Up to 2,048 video blocks the scores come
- * from the tensor cores (tf32 with every operand split into two tf32 parts,
- * within 2^-20 of |q||k| per channel of the fp32 dot product; lists can
+ * from the tensor cores (tf32 with every operand split into two tf32 parts:
+ * each channel's product within 3 * 2^-20 |q_c||k_c| of the exact one; lists can
  * differ from an fp32 FMA evaluation only between blocks whose scores are
  * that close); above that, from fp32 FMA chains.  A bounded internal wait
  * that runs out reports BSA_ERR_TIMEOUT through bsa_take_default_status. */
