@@ -39,7 +39,7 @@ def assert_close(got, want, what=""):
     return err, rel
 
 
-class GpuRun:
+class DeviceRun:
     """The whole six-call sequence on device buffers, kept for inspection."""
 
     def __init__(self, cfg, q, k, v, keep=None, dense=False, raster=False):

@@ -27,7 +27,7 @@ import torch
 import block_sparse_attention_47_b200 as bsa
 from gen import config, make_qkv
 from oracle import bsa_oracle as O
-from parity_helpers import GpuRun, matched_lists, to_np64
+from parity_helpers import DeviceRun, matched_lists, to_np64
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +59,7 @@ def grad_close(got, want, what):
 
 def run_backward(cfg, seed):
     q, k, v = make_qkv(cfg, seed, pad_fill=1e4, device="cuda")
-    run = GpuRun(cfg, q, k, v)
+    run = DeviceRun(cfg, q, k, v)
     attn, prob = run.attn, run.prob
     lse = torch.empty(attn.cnt.shape[:2] + (attn.sizes.n_tokens,), dtype=torch.float32,
                       device="cuda")

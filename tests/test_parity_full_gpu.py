@@ -14,7 +14,7 @@ import torch
 
 from gen import config, make_qkv
 from oracle import bsa_oracle as O
-from parity_helpers import (GpuRun, assert_close, decode_map, matched_lists, sample_blocks,
+from parity_helpers import (DeviceRun, assert_close, decode_map, matched_lists, sample_blocks,
                             scale_of, to_np64)
 
 pytestmark = pytest.mark.gpu
@@ -80,7 +80,7 @@ def check_full_size(name, over, raster=False):
     cfg = config(name, **over)
     rng = np.random.default_rng(1234)
     q, k, v = make_qkv(cfg, 42000 + len(name), pad_fill=1e4, device="cuda")
-    run = GpuRun(cfg, q, k, v, raster=raster)
+    run = DeviceRun(cfg, q, k, v, raster=raster)
     geo = O.Geometry(cfg)
     keep = run.prob.keep_blocks
     assert keep == O.keep_count(geo.nbv, cfg["keep_ratio"])

@@ -13,7 +13,7 @@ import torch
 import block_sparse_attention_47_b200 as bsa
 from gen import config
 from oracle import bsa_oracle as O
-from parity_helpers import (GpuRun, assert_close, check_list_row, decode_map, lists_to_device,
+from parity_helpers import (DeviceRun, assert_close, check_list_row, decode_map, lists_to_device,
                             oracle_bh, oracle_forward_matched, problem, scale_of, seeded_inputs,
                             to_np64)
 
@@ -44,7 +44,7 @@ def built(cuda_ok):
 def case(request):
     cfg = SMALL[request.param]
     (q, k, v), (qn, kn, vn) = seeded_inputs(cfg, seed=42000 + len(request.param))
-    run = GpuRun(cfg, q, k, v)
+    run = DeviceRun(cfg, q, k, v)
     geo = O.Geometry(cfg)
     lay = O.layout(cfg, kn)
     return dict(cfg=cfg, geo=geo, run=run, dev=(q, k, v), host=(qn, kn, vn), lay=lay)
@@ -253,7 +253,7 @@ def test_rescale_path_growing_logits(name):
     cfg = SMALL[name]
     q, k, v = growing_logit_inputs(cfg, 99)
     host = [to_np64(t) for t in (q, k, v)]
-    run = GpuRun(cfg, q, k, v)
+    run = DeviceRun(cfg, q, k, v)
     want = oracle_forward_matched(cfg, host, run.attn.idx.cpu().numpy(), run.prob.keep_blocks)
     assert_close(to_np64(run.out), want, name + " growing logits")
     assert int(run.attn.status.item()) == 0
@@ -267,7 +267,7 @@ def test_host_call_pipelined_by_head_groups(name, raster):
     oracle bar as the device path."""
     cfg = SMALL[name]
     (q, k, v), (qn, kn, vn) = seeded_inputs(cfg, seed=4242)
-    run = GpuRun(cfg, q, k, v)
+    run = DeviceRun(cfg, q, k, v)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     out = run.attn.host_call(qh, kh, vh, heads_per_group=1, raster=raster)
     torch.cuda.synchronize()

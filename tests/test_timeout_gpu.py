@@ -10,7 +10,7 @@ import torch
 
 import block_sparse_attention_47_b200 as bsa
 from gen import config
-from parity_helpers import GpuRun, seeded_inputs
+from parity_helpers import DeviceRun, seeded_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,7 @@ def built(cuda_ok):
 def test_stalled_wait_reports_timeout_and_context_survives():
     cfg = config("tiny")
     (q, k, v), _ = seeded_inputs(cfg, seed=777)
-    run = GpuRun(cfg, q, k, v)          # a normal call first
+    run = DeviceRun(cfg, q, k, v)          # a normal call first
     good = run.out.clone()
     attn = run.attn
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -51,7 +51,7 @@ def test_timeout_without_status_word_is_readable_from_the_default_word():
     bsa_take_default_status reports once and clears."""
     cfg = config("tiny")
     (q, k, v), _ = seeded_inputs(cfg, seed=778)
-    run = GpuRun(cfg, q, k, v)
+    run = DeviceRun(cfg, q, k, v)
     attn = run.attn
     assert bsa.take_default_status() == 0
     o = torch.empty_like(attn.op)
@@ -75,7 +75,7 @@ def test_stall_hook_affects_only_the_calling_thread():
     import threading
     cfg = config("tiny")
     (q, k, v), _ = seeded_inputs(cfg, seed=779)
-    run = GpuRun(cfg, q, k, v)
+    run = DeviceRun(cfg, q, k, v)
     attn = run.attn
     on = threading.Event()
     done = threading.Event()
